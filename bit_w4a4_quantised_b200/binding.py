@@ -1,0 +1,238 @@
+"""ctypes binding of libqwam.so (declared in include/qwam.h).
+
+Argument marshalling only: tensors are passed as raw device pointers, streams
+as cudaStream_t handles, and every step of the layer runs in the library's
+CUDA kernels.  There is no fallback: if the shared library is missing or a call
+fails, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqwam.so")
+
+#: Every entry point declared in include/qwam.h, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+SIGNATURES = {
+    "qwam_prepare_weight": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, ctypes.POINTER(_P)]),
+    "qwam_destroy": (_I, [_P]),
+    "qwam_linear": (_I, [_P, _I, _P, _P, _P]),
+    "qwam_prologue": (_I, [_P, _I, _P, _P]),
+    "qwam_gemm": (_I, [_I, _P, _P, _P]),
+    "qwam_handle_info": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                              ctypes.POINTER(_I), ctypes.POINTER(_F)]),
+    "qwam_export_weight": (_I, [_P, _P, _P, _P, _P]),
+    "qwam_debug_prepare_weight": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
+    "qwam_debug_prologue": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "qwam_quantize_fp32": (_I, [_P, _I, _I, _P, _P, _P, _P]),
+    "qwam_fp4_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "qwam_device_error": (_I, [ctypes.POINTER(ctypes.c_uint32)]),
+    "qwam_last_error": (ctypes.c_char_p, []),
+    "qwam_status_string": (ctypes.c_char_p, [_I]),
+    "qwam_version": (_I, []),
+}
+
+STATUS = {0: "QWAM_OK", 1: "QWAM_ERR_INVALID_ARG", 2: "QWAM_ERR_SHAPE", 3: "QWAM_ERR_ALIGN",
+          4: "QWAM_ERR_ARCH", 5: "QWAM_ERR_OOM", 6: "QWAM_ERR_CUDA", 7: "QWAM_ERR_TIMEOUT"}
+
+
+class QwamError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libqwam.so once.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m bit_w4a4_quantised_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise QwamError(status, load().qwam_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need(t, dtype, shape, name):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class Handle:
+    """A prepared layer (owns device memory inside the library)."""
+
+    def __init__(self, raw: int):
+        self._raw = raw
+        N, K, r, b, gw = _I(), _I(), _I(), _I(), _F()
+        _check(load().qwam_handle_info(raw, ctypes.byref(N), ctypes.byref(K), ctypes.byref(r),
+                                       ctypes.byref(b), ctypes.byref(gw)))
+        self.N, self.K, self.r, self.b, self.g_w = N.value, K.value, r.value, b.value, gw.value
+
+    @property
+    def raw(self) -> int:
+        if not self._raw:
+            raise ValueError("handle already destroyed")
+        return self._raw
+
+    def destroy(self) -> None:
+        if self._raw:
+            _check(load().qwam_destroy(self._raw))
+            self._raw = None
+
+    def __del__(self):
+        try:
+            if self._raw and _lib is not None:
+                _lib.qwam_destroy(self._raw)
+        except Exception:
+            pass
+
+
+def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None) -> Handle:
+    """W bf16 [N, K], s fp32 [K], V fp32 [K, r] or None, bias bf16 [N] or None."""
+    import torch
+    lib = load()
+    N, K = W.shape
+    _need(W, torch.bfloat16, (N, K), "W")
+    _need(s, torch.float32, (K,), "s")
+    r = 0 if V is None else V.shape[1]
+    if V is not None:
+        _need(V, torch.float32, (K, r), "V")
+    if bias is not None:
+        _need(bias, torch.bfloat16, (N,), "bias")
+    out = _P()
+    if wd_out is None:
+        _check(lib.qwam_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
+                                       _stream(stream), ctypes.byref(out)))
+    else:
+        _need(wd_out, torch.float32, (N, K), "wd_out")
+        _check(lib.qwam_debug_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
+                                             _ptr(wd_out), _stream(stream), ctypes.byref(out)))
+    return Handle(out.value)
+
+
+def linear(x, h: Handle, y=None, stream=None):
+    """y = the ASP NVFP4 layer applied to x (bf16 [M, K]) -> bf16 [M, N]."""
+    import torch
+    M = x.shape[0]
+    _need(x, torch.bfloat16, (M, h.K), "x")
+    if y is None:
+        y = torch.empty((M, h.N), dtype=torch.bfloat16, device=x.device)
+    _need(y, torch.bfloat16, (M, h.N), "y")
+    _check(load().qwam_linear(_ptr(x), M, h.raw, _ptr(y), _stream(stream)))
+    return y
+
+
+def prologue(x, h: Handle, stream=None) -> None:
+    import torch
+    _need(x, torch.bfloat16, (x.shape[0], h.K), "x")
+    _check(load().qwam_prologue(_ptr(x), x.shape[0], h.raw, _stream(stream)))
+
+
+def gemm(M: int, h: Handle, y, stream=None):
+    import torch
+    _need(y, torch.bfloat16, (M, h.N), "y")
+    _check(load().qwam_gemm(M, h.raw, _ptr(y), _stream(stream)))
+    return y
+
+
+def export_weight(h: Handle, stream=None) -> dict:
+    import torch
+    dev = torch.device("cuda")
+    codes = torch.empty((h.N, h.K // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty((-(-h.N // 128) * 128 * h.K // 16,), dtype=torch.uint8, device=dev)
+    L = torch.empty((h.N, max(h.r, 1)), dtype=torch.bfloat16, device=dev)
+    _check(load().qwam_export_weight(h.raw, _ptr(codes), _ptr(sf), _ptr(L) if h.r else None, _stream(stream)))
+    return {"codes": codes, "scales": sf, "L": L[:, :h.r], "g_w": h.g_w}
+
+
+def debug_prologue(x, h: Handle, stream=None) -> dict:
+    import torch
+    M = x.shape[0]
+    _need(x, torch.bfloat16, (M, h.K), "x")
+    dev = x.device
+    z = torch.empty((M, h.K), dtype=torch.float32, device=dev)
+    u = torch.empty((M, max(h.r, 1)), dtype=torch.float32, device=dev)
+    codes = torch.empty((M, h.K // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty((-(-M // 128) * 128 * h.K // 16,), dtype=torch.uint8, device=dev)
+    ub = torch.empty((M, max(h.r, 1)), dtype=torch.bfloat16, device=dev)
+    gx = torch.empty((1,), dtype=torch.float32, device=dev)
+    _check(load().qwam_debug_prologue(_ptr(x), M, h.raw, _ptr(z), _ptr(u) if h.r else None, _ptr(codes),
+                                      _ptr(sf), _ptr(ub) if h.r else None, _ptr(gx), _stream(stream)))
+    return {"z": z, "u": u[:, :h.r], "codes": codes, "scales": sf, "ub": ub[:, :h.r], "g_x": gx}
+
+
+def quantize_fp32(T, stream=None):
+    """Bare NVFP4 quantiser: T fp32 [rows, K] -> (codes [rows, K/2], tiled scales, g)."""
+    import torch
+    rows, K = T.shape
+    _need(T, torch.float32, (rows, K), "T")
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=T.device)
+    sf = torch.zeros((-(-rows // 128) * 128 * K // 16,), dtype=torch.uint8, device=T.device)
+    g = torch.empty((1,), dtype=torch.float32, device=T.device)
+    _check(load().qwam_quantize_fp32(_ptr(T), rows, K, _ptr(codes), _ptr(sf), _ptr(g), _stream(stream)))
+    return codes, sf, g
+
+
+def fp4_gemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, alpha: float = 1.0, stream=None):
+    """Bare block-scaled FP4 GEMM -> fp32 [M, N] (scales tiled; B rows padded to 256)."""
+    import torch
+    out = torch.empty((M, N), dtype=torch.float32, device=a_codes.device)
+    _check(load().qwam_fp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
+                                float(alpha), _ptr(out), _stream(stream)))
+    return out
+
+
+def device_error() -> int:
+    code = ctypes.c_uint32(0)
+    st = load().qwam_device_error(ctypes.byref(code))
+    if st not in (0, 7):
+        _check(st)
+    return code.value
+
+
+def version() -> int:
+    return load().qwam_version()

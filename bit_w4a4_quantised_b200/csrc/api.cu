@@ -1,0 +1,598 @@
+// C-ABI host layer of libqwam.so: argument checks, handle lifetime, the
+// per-device workspace, tensor-map construction and kernel launch order.
+// Declarations and the contract of every entry point: include/qwam.h.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "kernels.h"
+#include "qwam.h"
+
+using namespace qwam;
+
+namespace {
+
+constexpr uint32_t kMagic = 0x514d5731u;
+constexpr int kMaxDevices = 64;
+constexpr size_t kHeaderBytes = 256 + 65536;  // scalars, then split-K tile tickets
+constexpr int kMaxTiles = 16384;
+constexpr int kSMs = 148;
+
+thread_local std::string g_err;
+
+qwam_status fail(qwam_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+#define QW_CUDA(call)                                                                                     \
+  do {                                                                                                    \
+    cudaError_t e_ = (call);                                                                              \
+    if (e_ != cudaSuccess) return fail(QWAM_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));   \
+  } while (0)
+
+#define QW_TRY(expr)                    \
+  do {                                  \
+    qwam_status s_ = (expr);            \
+    if (s_ != QWAM_OK) return s_;       \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+qwam_status current_device(int* dev) {
+  QW_CUDA(cudaGetDevice(dev));
+  int major = 0;
+  QW_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev));
+  if (major != 10) return fail(QWAM_ERR_ARCH, "device %d is compute capability %d.x; this library is built for sm_100a", *dev, major);
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(QWAM_ERR_INVALID_ARG, "device index %d out of range", *dev);
+  return QWAM_OK;
+}
+
+// ---- tensor maps -----------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+qwam_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail(QWAM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QWAM_ERR_CUDA, "cuTensorMapEncodeTiled failed with code %d", static_cast<int>(r));
+  return QWAM_OK;
+}
+
+CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B; }
+
+// ---- GEMM launch plan ------------------------------------------------------
+struct Plan {
+  int bn, k_stages, splits, stages_per_split;
+};
+
+Plan plan_gemm(int M, int N, int K) {
+  Plan p{};
+  p.k_stages = (K + 255) / 256;
+  const int tiles_m = (M + 127) / 128;
+  p.bn = (M <= 128 || N < 256) ? 128 : 256;
+  const int tiles = tiles_m * ((N + p.bn - 1) / p.bn);
+  int splits = 1;
+  if (tiles < kSMs) splits = std::min(p.k_stages, std::max(1, kSMs / tiles));
+  p.stages_per_split = (p.k_stages + splits - 1) / splits;
+  p.splits = (p.k_stages + p.stages_per_split - 1) / p.stages_per_split;
+  return p;
+}
+
+// ---- per-device workspace --------------------------------------------------
+struct Arena {
+  uint8_t* base = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_arena_mu;
+Arena g_arena[kMaxDevices];
+
+struct Layout {
+  size_t codes, sf, u, ub, partial, total;
+};
+
+Layout layout_for(int M, int K, int N, int r, int splits) {
+  Layout L{};
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + std::max<size_t>(bytes, 16), 256);
+    return o;
+  };
+  const size_t Mp = round_up(static_cast<size_t>(M), 128);
+  const size_t rr = static_cast<size_t>(std::max(r, 1));
+  L.codes = take(Mp * K / 2);
+  L.sf = take(Mp * K / 16);
+  L.u = take(static_cast<size_t>(M) * rr * 4);
+  L.ub = take(Mp * rr * 2);
+  L.partial = take(splits > 1 ? static_cast<size_t>(splits) * M * N * 4 : 0);
+  L.total = off;
+  return L;
+}
+
+uint32_t* arena_amax(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base); }
+float* arena_gx(const Arena& a) { return reinterpret_cast<float*>(a.base + 4); }
+uint32_t* arena_err(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base + 8); }
+uint32_t* arena_counters(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base + 256); }
+
+qwam_status arena_get(int dev, size_t need, Arena** out) {
+  std::lock_guard<std::mutex> lock(g_arena_mu);
+  Arena& a = g_arena[dev];
+  if (a.bytes < need) {
+    if (a.base) {
+      QW_CUDA(cudaDeviceSynchronize());
+      QW_CUDA(cudaFree(a.base));
+      a.base = nullptr;
+      a.bytes = 0;
+    }
+    const size_t bytes = round_up(std::max(need, kHeaderBytes + (size_t(1) << 20)), size_t(1) << 20);
+    if (cudaMalloc(&a.base, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      a.base = nullptr;
+      return fail(QWAM_ERR_OOM, "workspace allocation of %zu bytes failed", bytes);
+    }
+    QW_CUDA(cudaMemset(a.base, 0, bytes));
+    QW_CUDA(cudaDeviceSynchronize());
+    a.bytes = bytes;
+  }
+  *out = &a;
+  return QWAM_OK;
+}
+
+int cluster_parts(int K) {
+  const int chunks = K / 128;
+  for (int c = std::min(8, chunks); c >= 1; --c)
+    if (chunks % c == 0) return c;
+  return 1;
+}
+
+}  // namespace
+
+struct qwam_layer {
+  uint32_t magic;
+  int N, K, r, b, dev;
+  uint8_t* codes;
+  uint8_t* sf;
+  uint16_t* L;
+  uint16_t *v_hi, *v_lo, *vt_hi, *vt_lo;
+  float* inv_s;
+  uint16_t* bias;
+  float g_w;
+  size_t sf_bytes;
+  CUtensorMap map_b128, map_b256, map_l128, map_l256;
+};
+
+namespace {
+
+void free_layer(qwam_layer* h) {
+  if (!h) return;
+  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->vt_hi, h->vt_lo, h->inv_s, h->bias};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  h->magic = 0;
+  delete h;
+}
+
+qwam_status check_handle(qwam_handle h) {
+  if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
+  int dev = -1;
+  QW_CUDA(cudaGetDevice(&dev));
+  if (dev != h->dev) return fail(QWAM_ERR_INVALID_ARG, "handle belongs to device %d, current device is %d", h->dev, dev);
+  return QWAM_OK;
+}
+
+qwam_status check_layer_shape(int N, int K, int r, int b) {
+  if (K <= 0 || K % 128) return fail(QWAM_ERR_SHAPE, "K=%d must be a positive multiple of 128", K);
+  if (b < 1 || b > 128 || (b & (b - 1))) return fail(QWAM_ERR_SHAPE, "hadamard_block=%d must be a power of two <= 128", b);
+  if (K % b) return fail(QWAM_ERR_SHAPE, "K=%d is not a multiple of hadamard_block=%d", K, b);
+  if (r != 0 && r != 16 && r != 32) return fail(QWAM_ERR_SHAPE, "rank r=%d must be 0, 16 or 32", r);
+  if (N < 16 || N % 16) return fail(QWAM_ERR_SHAPE, "N=%d must be a positive multiple of 16", N);
+  return QWAM_OK;
+}
+
+template <typename T>
+qwam_status dmalloc(T** p, size_t bytes) {
+  *p = nullptr;
+  if (cudaMalloc(reinterpret_cast<void**>(p), std::max<size_t>(bytes, 16)) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return fail(QWAM_ERR_OOM, "device allocation of %zu bytes failed", bytes);
+  }
+  return QWAM_OK;
+}
+
+// Stats + Quantise (any row count) or Fused (rows <= 64, when it fits).
+qwam_status run_rows(PrologueParams prm, int r, bool allow_fused, uint32_t* amax, cudaStream_t st) {
+  const int K = prm.K;
+  const int parts = cluster_parts(K);
+  const int chunks = K / 128 / parts;
+  if (allow_fused && prm.rows <= 64 && prologue_smem_bytes(r, PrologueMode::Fused, chunks) <= 200 * 1024) {
+    prm.chunks = chunks;
+    QW_CUDA(launch_prologue(prm, r, PrologueMode::Fused, parts, st));
+    return QWAM_OK;
+  }
+  QW_CUDA(cudaMemsetAsync(amax, 0, sizeof(uint32_t), st));
+  prm.amax_glob = amax;
+  prm.chunks = chunks;
+  QW_CUDA(launch_prologue(prm, r, PrologueMode::Stats, parts, st));
+  prm.chunks = 1;
+  QW_CUDA(launch_prologue(prm, r, PrologueMode::Quantise, 1, st));
+  return QWAM_OK;
+}
+
+qwam_status prepare_impl(const void* W, int N, int K, const float* s, const float* V, int r, const void* bias,
+                         int b, float* wd_out, void* stream, qwam_handle* out) {
+  if (!out) return fail(QWAM_ERR_INVALID_ARG, "out handle pointer is NULL");
+  *out = nullptr;
+  if (!W || !s) return fail(QWAM_ERR_INVALID_ARG, "W and s must be non-NULL");
+  QW_TRY(check_layer_shape(N, K, r, b));
+  if (r > 0 && !V) return fail(QWAM_ERR_INVALID_ARG, "V must be non-NULL when r > 0");
+  if (!aligned16(W) || !aligned16(s) || (V && !aligned16(V)) || (bias && !aligned16(bias)) ||
+      (wd_out && !aligned16(wd_out)))
+    return fail(QWAM_ERR_ALIGN, "device pointers must be 16-byte aligned");
+  int dev = 0;
+  QW_TRY(current_device(&dev));
+  cudaStream_t st = as_stream(stream);
+
+  qwam_layer* h = new qwam_layer();
+  std::memset(h, 0, sizeof(*h));
+  h->magic = kMagic;
+  h->N = N; h->K = K; h->r = r; h->b = b; h->dev = dev;
+  h->sf_bytes = round_up(static_cast<size_t>(N), 256) * K / 16;
+  float* u_tmp = nullptr;
+  uint32_t* scratch = nullptr;  // [0] amax, [1] err, [2] g_w (fp32)
+  auto cleanup = [&](qwam_status s) {
+    if (u_tmp) cudaFree(u_tmp);
+    if (scratch) cudaFree(scratch);
+    free_layer(h);
+    return s;
+  };
+  qwam_status s_;
+  const size_t rr = static_cast<size_t>(std::max(r, 1));
+  if ((s_ = dmalloc(&h->codes, static_cast<size_t>(N) * K / 2)) != QWAM_OK ||
+      (s_ = dmalloc(&h->sf, h->sf_bytes)) != QWAM_OK || (s_ = dmalloc(&h->L, static_cast<size_t>(N) * rr * 2)) != QWAM_OK ||
+      (s_ = dmalloc(&h->v_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->v_lo, K * rr * 2)) != QWAM_OK ||
+      (s_ = dmalloc(&h->vt_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->vt_lo, K * rr * 2)) != QWAM_OK ||
+      (s_ = dmalloc(&h->inv_s, static_cast<size_t>(K) * 4)) != QWAM_OK ||
+      (s_ = dmalloc(&u_tmp, static_cast<size_t>(N) * rr * 4)) != QWAM_OK || (s_ = dmalloc(&scratch, 64)) != QWAM_OK)
+    return cleanup(s_);
+  if (bias && (s_ = dmalloc(&h->bias, static_cast<size_t>(N) * 2)) != QWAM_OK) return cleanup(s_);
+
+#define QW_CUDA_CLEAN(call)                                                                                      \
+  do {                                                                                                           \
+    cudaError_t e_ = (call);                                                                                     \
+    if (e_ != cudaSuccess) return cleanup(fail(QWAM_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_))); \
+  } while (0)
+
+  QW_CUDA_CLEAN(cudaMemsetAsync(h->sf, 0, h->sf_bytes, st));
+  QW_CUDA_CLEAN(cudaMemsetAsync(scratch, 0, 64, st));
+  if (bias) QW_CUDA_CLEAN(cudaMemcpyAsync(h->bias, bias, static_cast<size_t>(N) * 2, cudaMemcpyDeviceToDevice, st));
+  QW_CUDA_CLEAN(launch_recip(s, h->inv_s, K, scratch + 1, st));
+  if (r > 0) QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, h->vt_hi, h->vt_lo, st));
+
+  PrologueParams prm{};
+  prm.x = W;
+  prm.chan = s;
+  prm.vt_hi = h->vt_hi; prm.vt_lo = h->vt_lo; prm.v_hi = h->v_hi; prm.v_lo = h->v_lo;
+  prm.rows = N;
+  prm.K = K;
+  prm.b = b;
+  prm.hscale = 1.0f / std::sqrt(static_cast<float>(b));
+  prm.u_glob = u_tmp;
+  prm.codes = h->codes;
+  prm.sf = h->sf;
+  prm.branch = h->L;
+  prm.branch_mode = 0;
+  prm.g_other = 1.0f;
+  prm.g_out = reinterpret_cast<float*>(scratch + 2);
+  prm.z_out = wd_out;
+  if ((s_ = run_rows(prm, r, false, scratch, st)) != QWAM_OK) return cleanup(s_);
+  uint32_t host_scr[4] = {0, 0, 0, 0};
+  QW_CUDA_CLEAN(cudaMemcpyAsync(host_scr, scratch, 16, cudaMemcpyDeviceToHost, st));
+  QW_CUDA_CLEAN(cudaStreamSynchronize(st));
+  if (host_scr[1]) return cleanup(fail(QWAM_ERR_INVALID_ARG, "smoothing vector s has an entry that is <= 0 or not finite"));
+  std::memcpy(&h->g_w, &host_scr[2], 4);
+
+  if ((s_ = make_map(&h->map_b128, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK ||
+      (s_ = make_map(&h->map_b256, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 128, 256,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK)
+    return cleanup(s_);
+  if (r > 0) {
+    if ((s_ = make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r))) !=
+            QWAM_OK ||
+        (s_ = make_map(&h->map_l256, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 256, branch_swizzle(r))) !=
+            QWAM_OK)
+      return cleanup(s_);
+  } else {
+    h->map_l128 = h->map_b128;
+    h->map_l256 = h->map_b256;
+  }
+  cudaFree(u_tmp);
+  cudaFree(scratch);
+#undef QW_CUDA_CLEAN
+  *out = h;
+  return QWAM_OK;
+}
+
+qwam_status check_linear_args(const void* x, int M, qwam_handle h) {
+  QW_TRY(check_handle(h));
+  if (M < 0) return fail(QWAM_ERR_SHAPE, "M=%d must be >= 0", M);
+  if (M > (1 << 24)) return fail(QWAM_ERR_SHAPE, "M=%d exceeds the supported maximum of 2^24", M);
+  if (M > 0 && !x) return fail(QWAM_ERR_INVALID_ARG, "x is NULL");
+  if (x && !aligned16(x)) return fail(QWAM_ERR_ALIGN, "x must be 16-byte aligned");
+  return QWAM_OK;
+}
+
+qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, float* u_out, cudaStream_t st,
+                          Arena** arena_out, Layout* lay_out) {
+  const Plan pl = plan_gemm(M, h->N, h->K);
+  const Layout lay = layout_for(M, h->K, h->N, h->r, pl.splits);
+  Arena* a = nullptr;
+  QW_TRY(arena_get(h->dev, lay.total, &a));
+  PrologueParams prm{};
+  prm.x = x;
+  prm.chan = h->inv_s;
+  prm.vt_hi = h->vt_hi; prm.vt_lo = h->vt_lo; prm.v_hi = h->v_hi; prm.v_lo = h->v_lo;
+  prm.rows = M;
+  prm.K = h->K;
+  prm.b = h->b;
+  prm.hscale = 1.0f / std::sqrt(static_cast<float>(h->b));
+  prm.u_glob = reinterpret_cast<float*>(a->base + lay.u);
+  prm.codes = a->base + lay.codes;
+  prm.sf = a->base + lay.sf;
+  prm.branch = reinterpret_cast<uint16_t*>(a->base + lay.ub);
+  prm.branch_mode = 1;
+  prm.g_other = h->g_w;
+  prm.g_out = arena_gx(*a);
+  prm.z_out = z_out;
+  prm.u_out = u_out;
+  QW_TRY(run_rows(prm, h->r, true, arena_amax(*a), st));
+  if (arena_out) *arena_out = a;
+  if (lay_out) *lay_out = lay;
+  return QWAM_OK;
+}
+
+qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
+  const Plan pl = plan_gemm(M, h->N, h->K);
+  const Layout lay = layout_for(M, h->K, h->N, h->r, pl.splits);
+  Arena* a = nullptr;
+  QW_TRY(arena_get(h->dev, lay.total, &a));
+  const int tiles = ((M + 127) / 128) * ((h->N + pl.bn - 1) / pl.bn);
+  if (pl.splits > 1 && tiles > kMaxTiles) return fail(QWAM_ERR_SHAPE, "too many output tiles for split-K");
+  GemmMaps maps{};
+  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->base + lay.codes, h->K / 2, M, h->K / 2, 128, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B));
+  maps.b = pl.bn == 256 ? h->map_b256 : h->map_b128;
+  if (h->r > 0) {
+    QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->base + lay.ub, h->r, M, h->r * 2, h->r, 128,
+                    branch_swizzle(h->r)));
+    maps.l = pl.bn == 256 ? h->map_l256 : h->map_l128;
+  } else {
+    maps.u = maps.a;
+    maps.l = maps.b;
+  }
+  GemmParams p{};
+  p.M = M; p.N = h->N; p.K = h->K;
+  p.k_stages = pl.k_stages;
+  p.stages_per_split = pl.stages_per_split;
+  p.splits = pl.splits;
+  p.sfa = a->base + lay.sf;
+  p.sfb = h->sf;
+  p.g_a_ptr = arena_gx(*a);
+  p.g_b = h->g_w;
+  p.has_branch = h->r > 0;
+  p.branch_k = h->r;
+  p.bias = h->bias;
+  p.y = y;
+  p.partial = reinterpret_cast<float*>(a->base + lay.partial);
+  p.counters = arena_counters(*a);
+  p.err = arena_err(*a);
+  QW_CUDA(launch_gemm(maps, p, pl.bn, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
+  return QWAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qwam_status qwam_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                const void* bias_bf16, int hadamard_block, void* stream, qwam_handle* out) {
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, nullptr, stream, out);
+}
+
+qwam_status qwam_debug_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                      const void* bias_bf16, int hadamard_block, float* Wd_f32, void* stream,
+                                      qwam_handle* out) {
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, Wd_f32, stream, out);
+}
+
+qwam_status qwam_destroy(qwam_handle h) {
+  if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
+  int prev = -1;
+  QW_CUDA(cudaGetDevice(&prev));
+  if (prev != h->dev) QW_CUDA(cudaSetDevice(h->dev));
+  QW_CUDA(cudaDeviceSynchronize());
+  free_layer(h);
+  if (prev != -1) cudaSetDevice(prev);
+  return QWAM_OK;
+}
+
+qwam_status qwam_prologue(const void* x_bf16, int M, qwam_handle h, void* stream) {
+  QW_TRY(check_linear_args(x_bf16, M, h));
+  if (M == 0) return QWAM_OK;
+  return prologue_impl(x_bf16, M, h, nullptr, nullptr, as_stream(stream), nullptr, nullptr);
+}
+
+qwam_status qwam_gemm(int M, qwam_handle h, void* y_bf16, void* stream) {
+  QW_TRY(check_handle(h));
+  if (M < 0) return fail(QWAM_ERR_SHAPE, "M=%d must be >= 0", M);
+  if (M == 0) return QWAM_OK;
+  if (!y_bf16) return fail(QWAM_ERR_INVALID_ARG, "y is NULL");
+  if (!aligned16(y_bf16)) return fail(QWAM_ERR_ALIGN, "y must be 16-byte aligned");
+  return gemm_impl(M, h, y_bf16, as_stream(stream));
+}
+
+qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream) {
+  QW_TRY(check_linear_args(x_bf16, M, h));
+  if (M == 0) return QWAM_OK;
+  if (!y_bf16) return fail(QWAM_ERR_INVALID_ARG, "y is NULL");
+  if (!aligned16(y_bf16)) return fail(QWAM_ERR_ALIGN, "y must be 16-byte aligned");
+  if (y_bf16 == x_bf16) return fail(QWAM_ERR_INVALID_ARG, "y must not alias x");
+  QW_TRY(prologue_impl(x_bf16, M, h, nullptr, nullptr, as_stream(stream), nullptr, nullptr));
+  return gemm_impl(M, h, y_bf16, as_stream(stream));
+}
+
+qwam_status qwam_handle_info(qwam_handle h, int* N, int* K, int* r, int* b, float* g_w) {
+  if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
+  if (N) *N = h->N;
+  if (K) *K = h->K;
+  if (r) *r = h->r;
+  if (b) *b = h->b;
+  if (g_w) *g_w = h->g_w;
+  return QWAM_OK;
+}
+
+qwam_status qwam_export_weight(qwam_handle h, void* codes, void* scales, void* L_bf16, void* stream) {
+  QW_TRY(check_handle(h));
+  cudaStream_t st = as_stream(stream);
+  if (codes) QW_CUDA(cudaMemcpyAsync(codes, h->codes, static_cast<size_t>(h->N) * h->K / 2, cudaMemcpyDeviceToDevice, st));
+  if (scales)
+    QW_CUDA(cudaMemcpyAsync(scales, h->sf, round_up(static_cast<size_t>(h->N), 128) * h->K / 16, cudaMemcpyDeviceToDevice, st));
+  if (L_bf16 && h->r > 0)
+    QW_CUDA(cudaMemcpyAsync(L_bf16, h->L, static_cast<size_t>(h->N) * h->r * 2, cudaMemcpyDeviceToDevice, st));
+  return QWAM_OK;
+}
+
+qwam_status qwam_debug_prologue(const void* x_bf16, int M, qwam_handle h, float* z_f32, float* u_f32, void* codes,
+                                void* scales, void* ubr_bf16, float* g_x, void* stream) {
+  QW_TRY(check_linear_args(x_bf16, M, h));
+  if (M == 0) return QWAM_OK;
+  if ((z_f32 && !aligned16(z_f32)) || (u_f32 && !aligned16(u_f32)))
+    return fail(QWAM_ERR_ALIGN, "debug outputs must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  Arena* a = nullptr;
+  Layout lay{};
+  QW_TRY(prologue_impl(x_bf16, M, h, z_f32, u_f32, st, &a, &lay));
+  if (codes) QW_CUDA(cudaMemcpyAsync(codes, a->base + lay.codes, static_cast<size_t>(M) * h->K / 2, cudaMemcpyDeviceToDevice, st));
+  if (scales)
+    QW_CUDA(cudaMemcpyAsync(scales, a->base + lay.sf, round_up(static_cast<size_t>(M), 128) * h->K / 16,
+                            cudaMemcpyDeviceToDevice, st));
+  if (ubr_bf16 && h->r > 0)
+    QW_CUDA(cudaMemcpyAsync(ubr_bf16, a->base + lay.ub, static_cast<size_t>(M) * h->r * 2, cudaMemcpyDeviceToDevice, st));
+  if (g_x) QW_CUDA(cudaMemcpyAsync(g_x, arena_gx(*a), 4, cudaMemcpyDeviceToDevice, st));
+  return QWAM_OK;
+}
+
+qwam_status qwam_quantize_fp32(const float* T, int rows, int K, void* codes, void* scales, float* g, void* stream) {
+  if (!T || !codes || !scales || !g) return fail(QWAM_ERR_INVALID_ARG, "NULL argument");
+  if (rows < 1 || K < 64 || K % 64) return fail(QWAM_ERR_SHAPE, "rows >= 1 and K a positive multiple of 64 required");
+  if (!aligned16(T) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(g) & 3))
+    return fail(QWAM_ERR_ALIGN, "buffers must be 16-byte aligned");
+  int dev = 0;
+  QW_TRY(current_device(&dev));
+  Arena* a = nullptr;
+  QW_TRY(arena_get(dev, kHeaderBytes, &a));
+  QW_CUDA(launch_quantize_fp32(T, rows, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), g,
+                               arena_amax(*a), as_stream(stream)));
+  return QWAM_OK;
+}
+
+qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales,
+                          int M, int N, int K, float alpha, float* out_f32, void* stream) {
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !out_f32) return fail(QWAM_ERR_INVALID_ARG, "NULL argument");
+  if (M < 1 || N < 16 || N % 16 || K < 128 || K % 128) return fail(QWAM_ERR_SHAPE, "bad GEMM shape M=%d N=%d K=%d", M, N, K);
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(out_f32))
+    return fail(QWAM_ERR_ALIGN, "buffers must be 16-byte aligned");
+  int dev = 0;
+  QW_TRY(current_device(&dev));
+  Arena* a = nullptr;
+  QW_TRY(arena_get(dev, kHeaderBytes, &a));
+  const int bn = N > 128 ? 256 : 128;
+  GemmMaps maps{};
+  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  QW_TRY(make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, K / 2, N, K / 2, 128, bn, CU_TENSOR_MAP_SWIZZLE_128B));
+  maps.u = maps.a;
+  maps.l = maps.b;
+  GemmParams p{};
+  p.M = M; p.N = N; p.K = K;
+  p.k_stages = (K + 255) / 256;
+  p.stages_per_split = p.k_stages;
+  p.splits = 1;
+  p.sfa = static_cast<const uint8_t*>(a_scales);
+  p.sfb = static_cast<const uint8_t*>(b_scales);
+  p.g_a_ptr = nullptr;
+  p.g_a = alpha;
+  p.g_b = 1.0f;
+  p.out_f32 = out_f32;
+  p.counters = arena_counters(*a);
+  p.err = arena_err(*a);
+  QW_CUDA(launch_gemm(maps, p, bn, GemmEpilogue::RawF32, as_stream(stream)));
+  return QWAM_OK;
+}
+
+qwam_status qwam_device_error(uint32_t* code) {
+  if (!code) return fail(QWAM_ERR_INVALID_ARG, "code is NULL");
+  *code = 0;
+  int dev = 0;
+  QW_CUDA(cudaGetDevice(&dev));
+  QW_CUDA(cudaDeviceSynchronize());
+  if (dev < 0 || dev >= kMaxDevices) return QWAM_OK;
+  std::lock_guard<std::mutex> lock(g_arena_mu);
+  const Arena& a = g_arena[dev];
+  if (!a.base) return QWAM_OK;
+  QW_CUDA(cudaMemcpy(code, arena_err(a), 4, cudaMemcpyDeviceToHost));
+  QW_CUDA(cudaMemset(arena_err(a), 0, 4));
+  if (*code) return fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired (flags 0x%x)", *code);
+  return QWAM_OK;
+}
+
+const char* qwam_last_error(void) { return g_err.c_str(); }
+
+const char* qwam_status_string(qwam_status s) {
+  switch (s) {
+    case QWAM_OK: return "QWAM_OK";
+    case QWAM_ERR_INVALID_ARG: return "QWAM_ERR_INVALID_ARG";
+    case QWAM_ERR_SHAPE: return "QWAM_ERR_SHAPE";
+    case QWAM_ERR_ALIGN: return "QWAM_ERR_ALIGN";
+    case QWAM_ERR_ARCH: return "QWAM_ERR_ARCH";
+    case QWAM_ERR_OOM: return "QWAM_ERR_OOM";
+    case QWAM_ERR_CUDA: return "QWAM_ERR_CUDA";
+    case QWAM_ERR_TIMEOUT: return "QWAM_ERR_TIMEOUT";
+  }
+  return "QWAM_UNKNOWN";
+}
+
+int qwam_version(void) { return 100; }
+
+}  // extern "C"

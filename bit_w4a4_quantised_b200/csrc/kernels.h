@@ -1,0 +1,85 @@
+// Internal launch interface between the C-ABI host layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace qwam {
+
+// One "rows" job of the activation prologue / weight prepare:
+//   T~ = (T * chan) H,  c = T~ V,  Z = T~ - c V^T,  quantise(Z),
+// with T = x, chan = 1/s on the activation side and T = W, chan = s on the
+// weight side.
+struct PrologueParams {
+  const void* x;          // bf16 [rows, K]
+  const float* chan;      // fp32 [K]
+  const uint16_t* vt_hi;  // bf16 bits [r, K]  (V^T, high part)
+  const uint16_t* vt_lo;  // bf16 bits [r, K]  (V^T, low part)
+  const uint16_t* v_hi;   // bf16 bits [K, r]
+  const uint16_t* v_lo;   // bf16 bits [K, r]
+  int rows;
+  int K;
+  int b;                  // Hadamard block (power of two, <= 128)
+  int chunks;             // 128-column chunks per CTA
+  float hscale;           // fp32(1 / sqrt(b))
+  float* u_glob;          // fp32 [rows, r]: written by phase 1, read by phase 2
+  uint32_t* amax_glob;    // fp32 bits of max|Z|: atomicMax'd by phase 1
+  uint8_t* codes;         // [rows, K/2]
+  uint8_t* sf;            // tiled scales, rows padded to 128
+  uint16_t* branch;       // bf16 bits [rows, r]
+  int branch_mode;        // 0: bf16(c)   1: bf16(c / (g * g_other))
+  float g_other;
+  float* g_out;           // fp32 scalar: the per-tensor scale of Z
+  float* z_out;           // optional fp32 [rows, K] (debug export of Z)
+  float* u_out;           // optional fp32 [rows, r] (debug export of c)
+};
+
+enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2 };
+
+// Fused: one cluster row group holds every row (rows <= 64); Stats/Quantise:
+// the two-launch form for any row count (Stats needs *amax_glob == 0).
+cudaError_t launch_prologue(const PrologueParams& p, int r, PrologueMode mode, int cluster, cudaStream_t st);
+size_t prologue_smem_bytes(int r, PrologueMode mode, int chunks);
+
+cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st);
+cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, uint16_t* vt_hi,
+                           uint16_t* vt_lo, cudaStream_t st);
+cudaError_t launch_quantize_fp32(const float* T, int rows, int K, uint8_t* codes, uint8_t* sf, float* g_out,
+                                 uint32_t* amax_scratch, cudaStream_t st);
+
+// Block-scaled FP4 GEMM.
+enum class GemmEpilogue { Bf16 = 0, RawF32 = 1, SplitK = 2 };
+
+struct GemmParams {
+  int M, N, K;
+  int k_stages;            // ceil(K / 256)
+  int stages_per_split;
+  int splits;
+  const uint8_t* sfa;      // tiled, rows padded to 128
+  const uint8_t* sfb;      // tiled, rows padded to 256
+  const float* g_a_ptr;    // device scalar (activation scale) or nullptr
+  float g_a;               // used when g_a_ptr == nullptr
+  float g_b;
+  int has_branch;          // rank-r branch in the accumulator (r = branch_k)
+  int branch_k;
+  const void* bias;        // bf16 [N] or nullptr
+  void* y;                 // bf16 [M, N]
+  float* out_f32;          // fp32 [M, N] (raw epilogue)
+  float* partial;          // fp32 [splits, M, N]
+  uint32_t* counters;      // one per output tile, zero between launches
+  uint32_t* err;
+};
+
+struct GemmMaps {
+  CUtensorMap a;  // codes A [M, K/2] u8, box 128 B x 128 rows, 128B swizzle
+  CUtensorMap b;  // codes B [N, K/2] u8, box 128 B x BN rows, 128B swizzle
+  CUtensorMap u;  // branch A [M, r] bf16, box r x 128 rows
+  CUtensorMap l;  // branch B [N, r] bf16, box r x BN rows
+};
+
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int bn, GemmEpilogue epi, cudaStream_t st);
+size_t gemm_smem_bytes(int bn);
+
+}  // namespace qwam

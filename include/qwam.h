@@ -1,0 +1,164 @@
+/*
+ * qwam — the Action-Subspace-Protected (deflated form) NVFP4 W4A4 linear
+ * layer on NVIDIA B200 (sm_100a), as a C-ABI shared library (libqwam.so).
+ *
+ * The layer ("FastWAM UR3 3-task — 4-bit quantisations", model card, section
+ * "What ASP is, and what the deflated form means"):
+ *
+ *     x~ = (x / s) H
+ *     y  = (x~ V)(W~ V)^T + NVFP4GEMM((I - V V^T) x~, W~ (I - V V^T)) + bias
+ *
+ * s: per-input-channel smoothing vector; H: block Hadamard (blocks of b,
+ * Sylvester order, scaled by 1/sqrt(b)); V: K x r basis with orthonormal
+ * columns; W~ = W diag(s) H (H on both sides so the branch pairs x~V with W~V
+ * in the same coordinates).  NVFP4 ("numeric format" row of the card's top
+ * table): E2M1 elements in blocks of 16 along K with E4M3 block scales, plus a
+ * fp32 per-tensor scale g = amax / 2688.  The rank-r branch stays bf16 ("The
+ * rank-32 branch stays in bf16 by design"; the Q-WAM abstract's "16-bit
+ * low-rank branch").
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Pointers marked "device" are CUDA device pointers on the current device;
+ *    "host" pointers are ordinary CPU memory.  Every pointer is BORROWED: the
+ *    library never frees caller memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Device work is enqueued on it in order; outputs are valid once the stream
+ *    reaches that point.
+ *  - Matrices are row-major and contiguous.  Device pointers must be 16-byte
+ *    aligned.
+ *  - Every call returns a qwam_status.  On any status other than QWAM_OK no
+ *    output has been written (argument checks happen before any launch) and
+ *    qwam_last_error() returns a message for the calling thread.  Nothing
+ *    traps on the device; a bounded device-side wait that runs out sets a
+ *    flag read by qwam_device_error().
+ *  - Shape limits: K % 128 == 0, K % b == 0, b in {1,2,4,...,128},
+ *    r in {0, 16, 32}, N % 16 == 0, N >= 16, M >= 0 (M == 0 is a no-op).
+ *  - Requires a compute capability 10.0 device (B200).
+ */
+#ifndef QWAM_H
+#define QWAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct qwam_layer* qwam_handle;
+
+typedef enum {
+  QWAM_OK = 0,
+  QWAM_ERR_INVALID_ARG = 1, /* null pointer, bad value (e.g. s <= 0), bad handle */
+  QWAM_ERR_SHAPE = 2,       /* a shape limit above is violated */
+  QWAM_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+  QWAM_ERR_ARCH = 4,        /* current device is not compute capability 10.x */
+  QWAM_ERR_OOM = 5,         /* device allocation failed */
+  QWAM_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed */
+  QWAM_ERR_TIMEOUT = 7      /* a bounded device wait expired (qwam_device_error) */
+} qwam_status;
+
+/* ---------------------------------------------------------------------------
+ * Weight side (offline).  Card sections "What ASP is..." (deflated form: the
+ * branch carries the exact W~V, the FP4 weight holds W~(I - VV^T)) and "Files"
+ * (E4M3 scales pre-swizzled to the 128x4 tensor-core tile layout).
+ *
+ *   W_bf16  device bf16 [N, K]          weight
+ *   s       device fp32 [K]             smoothing vector, every entry > 0 and finite
+ *   V       device fp32 [K, r]          basis; may be NULL iff r == 0
+ *   bias    device bf16 [N] or NULL
+ *   out     host   receives the new handle
+ *
+ * Computes W~ = W diag(s) H, L = W~V (stored bf16 [N, r]), W_d = W~ - L V^T,
+ * and quantises W_d (packed E2M1 codes [N, K/2], tiled E4M3 scales, fp32 g_w).
+ * The handle owns copies of everything it needs (1/s, V split into bf16
+ * hi/lo parts, bias); the caller may free W, s, V and bias when this returns.
+ * The call synchronises `stream`.
+ * ------------------------------------------------------------------------- */
+qwam_status qwam_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                const void* bias_bf16, int hadamard_block, void* stream, qwam_handle* out);
+
+/* Release a handle and its device memory (synchronises the device). */
+qwam_status qwam_destroy(qwam_handle h);
+
+/* ---------------------------------------------------------------------------
+ * Activation side (per call).  y = the layer above for x.
+ *
+ *   x_bf16  device bf16 [M, K]   (read only)
+ *   y_bf16  device bf16 [M, N]   (written; must not alias x)
+ *
+ * Runs the fused prologue (x/s, block FWHT, u = x~V, z = x~ - uV^T, per-tensor
+ * amax, NVFP4 quantisation of z, u' = bf16(u / (g_x g_w))) and the tcgen05
+ * block-scaled FP4 GEMM whose epilogue adds u' L^T and the bias and rounds
+ * once to bf16.  Scratch comes from a per-device workspace inside the library
+ * that grows on first use of a larger shape (that call allocates and
+ * synchronises the device, so it must not be stream-captured; a call at the
+ * largest M first makes later calls allocation-free).  Calls that share the
+ * workspace must be ordered: do not run two qwam_linear calls concurrently on
+ * different streams of the same device.
+ * ------------------------------------------------------------------------- */
+qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream);
+
+/* The two halves of qwam_linear, for measurement: qwam_linear(x, M, h, y, st)
+ * == qwam_prologue(x, M, h, st) followed by qwam_gemm(M, h, y, st) on the same
+ * stream with nothing else using the workspace in between. */
+qwam_status qwam_prologue(const void* x_bf16, int M, qwam_handle h, void* stream);
+qwam_status qwam_gemm(int M, qwam_handle h, void* y_bf16, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Inspection and test exports (not on the hot path).
+ * ------------------------------------------------------------------------- */
+
+/* Host outputs (each may be NULL): N, K, r, b and the weight scale g_w. */
+qwam_status qwam_handle_info(qwam_handle h, int* N, int* K, int* r, int* b, float* g_w);
+
+/* Copy the handle's weight operands into caller device buffers (each may be
+ * NULL): codes [N, K/2] bytes; scales: the tiled layout, round_up(N,128)*K/16
+ * bytes; L: bf16 [N, r]. */
+qwam_status qwam_export_weight(qwam_handle h, void* codes, void* scales, void* L_bf16, void* stream);
+
+/* Same as qwam_prepare_weight, and also writes W_d (the exact fp32 tensor the
+ * weight quantiser consumed) to Wd_f32 (device fp32 [N, K]). */
+qwam_status qwam_debug_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                      const void* bias_bf16, int hadamard_block, float* Wd_f32, void* stream,
+                                      qwam_handle* out);
+
+/* Run the activation prologue and copy its products to caller device buffers
+ * (each may be NULL): z fp32 [M, K] (the exact quantiser input), u fp32 [M, r],
+ * codes [M, K/2], scales (tiled, round_up(M,128)*K/16 bytes), u' bf16 [M, r],
+ * g_x fp32 scalar. */
+qwam_status qwam_debug_prologue(const void* x_bf16, int M, qwam_handle h, float* z_f32, float* u_f32,
+                                void* codes, void* scales, void* ubr_bf16, float* g_x, void* stream);
+
+/* The bare NVFP4 quantiser on a device fp32 tensor T [rows, K] (K % 64 == 0):
+ * codes [rows, K/2], scales in the tiled layout (round_up(rows,128)*K/16 bytes;
+ * padding rows are not written), g (device fp32 scalar). */
+qwam_status qwam_quantize_fp32(const float* T, int rows, int K, void* codes, void* scales, float* g, void* stream);
+
+/* The bare block-scaled FP4 GEMM: out[m,n] = alpha * sum_k deq(A)[m,k] deq(B)[n,k]
+ * with deq = e2m1(code) * e4m3(scale) (no per-tensor scales).  a_codes [M, K/2],
+ * b_codes [N, K/2]; a_scales / b_scales in the tiled layout with rows padded to
+ * 128 (A) and 256 (B), padding bytes zero; out fp32 [M, N] device.  K % 128 == 0. */
+qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales,
+                          int M, int N, int K, float alpha, float* out_f32, void* stream);
+
+/* Synchronise the current device, then return (and clear) the device error
+ * word set by bounded waits: *code == 0 means none expired.  Returns
+ * QWAM_ERR_TIMEOUT when *code != 0. */
+qwam_status qwam_device_error(uint32_t* code);
+
+/* Message for the last failing call on this thread ("" if none). */
+const char* qwam_last_error(void);
+
+/* Static name of a status code. */
+const char* qwam_status_string(qwam_status s);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int qwam_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QWAM_H */
