@@ -30,6 +30,8 @@ SIGNATURES = {
     "qwam_debug_prologue": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "qwam_quantize_fp32": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "qwam_fp4_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "qwam_plan_info": (_I, [_I, _P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                            ctypes.POINTER(_I)]),
     "qwam_device_error": (_I, [ctypes.POINTER(ctypes.c_uint32)]),
     "qwam_last_error": (ctypes.c_char_p, []),
     "qwam_status_string": (ctypes.c_char_p, [_I]),
@@ -224,6 +226,14 @@ def fp4_gemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, alpha
     _check(load().qwam_fp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
                                 float(alpha), _ptr(out), _stream(stream)))
     return out
+
+
+def plan_info(M: int, h: Handle) -> dict:
+    """How qwam_linear runs M rows of this layer: kernel launches per call,
+    single-launch prologue or not, GEMM K splits and tile width."""
+    k, f, sp, bn = _I(), _I(), _I(), _I()
+    _check(load().qwam_plan_info(M, h.raw, ctypes.byref(k), ctypes.byref(f), ctypes.byref(sp), ctypes.byref(bn)))
+    return {"kernels": k.value, "fused": bool(f.value), "splits": sp.value, "bn": bn.value}
 
 
 def device_error() -> int:

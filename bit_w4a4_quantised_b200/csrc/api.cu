@@ -89,6 +89,14 @@ qwam_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
   return QWAM_OK;
 }
 
+// Scale buffer of `rows_padded` rows (multiple of 128) and K columns in the tiled
+// layout, viewed as u8 [rows_padded * K / 16 / 256, 256]: one GEMM stage (two
+// 512-byte atoms) is a 256 x 4 box.
+qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, int K) {
+  const uint64_t total = static_cast<uint64_t>(rows_padded) * K / 16;
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, total / 256, 256, 256, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B; }
 
 // ---- GEMM launch plan ------------------------------------------------------
@@ -98,7 +106,7 @@ struct Plan {
 
 Plan plan_gemm(int M, int N, int K) {
   Plan p{};
-  p.k_stages = (K + 255) / 256;
+  p.k_stages = (K + 127) / 128;
   const int tiles_m = (M + 127) / 128;
   p.bn = (M <= 128 || N < 256) ? 128 : 256;
   const int tiles = tiles_m * ((N + p.bn - 1) / p.bn);
@@ -189,7 +197,8 @@ struct qwam_layer {
   uint16_t* bias;
   float g_w;
   size_t sf_bytes;
-  CUtensorMap map_b128, map_b256, map_l128, map_l256;
+  CUtensorMap map_b128, map_b256, map_l128, map_l256, map_sfb;
+  ProMaps vmaps;  // V^T and V (hi/lo) tensor maps for the prologue; x is per call
 };
 
 namespace {
@@ -231,22 +240,27 @@ qwam_status dmalloc(T** p, size_t bytes) {
   return QWAM_OK;
 }
 
-// Stats + Quantise (any row count) or Fused (rows <= 64, when it fits).
-qwam_status run_rows(PrologueParams prm, int r, bool allow_fused, uint32_t* amax, cudaStream_t st) {
+bool use_fused(int rows) { return rows <= 128; }
+
+// Stats + Quantise (any row count) or Fused (rows <= 128).  T is the bf16
+// [rows, K] input (x or W); vmaps holds the handle's V tensor maps.
+qwam_status run_rows(const void* T, PrologueParams prm, int r, const ProMaps& vmaps, bool allow_fused,
+                     uint32_t* amax, cudaStream_t st) {
   const int K = prm.K;
   const int parts = cluster_parts(K);
-  const int chunks = K / 128 / parts;
-  if (allow_fused && prm.rows <= 64 && prologue_smem_bytes(r, PrologueMode::Fused, chunks) <= 200 * 1024) {
-    prm.chunks = chunks;
-    QW_CUDA(launch_prologue(prm, r, PrologueMode::Fused, parts, st));
+  ProMaps maps = vmaps;
+  QW_TRY(make_map(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, K, prm.rows, static_cast<uint64_t>(K) * 2, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B));
+  if (r == 0) maps.vt_hi = maps.vt_lo = maps.v_hi = maps.v_lo = maps.x;
+  prm.chunks = K / 128 / parts;
+  prm.amax_glob = amax;
+  if (allow_fused && use_fused(prm.rows)) {
+    QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Fused, parts, st));
     return QWAM_OK;
   }
   QW_CUDA(cudaMemsetAsync(amax, 0, sizeof(uint32_t), st));
-  prm.amax_glob = amax;
-  prm.chunks = chunks;
-  QW_CUDA(launch_prologue(prm, r, PrologueMode::Stats, parts, st));
-  prm.chunks = 1;
-  QW_CUDA(launch_prologue(prm, r, PrologueMode::Quantise, 1, st));
+  QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Stats, parts, st));
+  QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Quantise, parts, st));
   return QWAM_OK;
 }
 
@@ -300,10 +314,19 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   QW_CUDA_CLEAN(launch_recip(s, h->inv_s, K, scratch + 1, st));
   if (r > 0) QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, h->vt_hi, h->vt_lo, st));
 
+  if (r > 0) {
+    if ((s_ = make_map(&h->vmaps.vt_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->vt_hi, K, r, static_cast<uint64_t>(K) * 2,
+                       64, r, CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK ||
+        (s_ = make_map(&h->vmaps.vt_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->vt_lo, K, r, static_cast<uint64_t>(K) * 2,
+                       64, r, CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK ||
+        (s_ = make_map(&h->vmaps.v_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_hi, r, K, r * 2, r, 128,
+                       branch_swizzle(r))) != QWAM_OK ||
+        (s_ = make_map(&h->vmaps.v_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_lo, r, K, r * 2, r, 128,
+                       branch_swizzle(r))) != QWAM_OK)
+      return cleanup(s_);
+  }
   PrologueParams prm{};
-  prm.x = W;
   prm.chan = s;
-  prm.vt_hi = h->vt_hi; prm.vt_lo = h->vt_lo; prm.v_hi = h->v_hi; prm.v_lo = h->v_lo;
   prm.rows = N;
   prm.K = K;
   prm.b = b;
@@ -316,18 +339,21 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   prm.g_other = 1.0f;
   prm.g_out = reinterpret_cast<float*>(scratch + 2);
   prm.z_out = wd_out;
-  if ((s_ = run_rows(prm, r, false, scratch, st)) != QWAM_OK) return cleanup(s_);
+  prm.err = scratch + 3;
+  if ((s_ = run_rows(W, prm, r, h->vmaps, false, scratch, st)) != QWAM_OK) return cleanup(s_);
   uint32_t host_scr[4] = {0, 0, 0, 0};
   QW_CUDA_CLEAN(cudaMemcpyAsync(host_scr, scratch, 16, cudaMemcpyDeviceToHost, st));
   QW_CUDA_CLEAN(cudaStreamSynchronize(st));
   if (host_scr[1]) return cleanup(fail(QWAM_ERR_INVALID_ARG, "smoothing vector s has an entry that is <= 0 or not finite"));
+  if (host_scr[3]) return cleanup(fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired in prepare (flags 0x%x)", host_scr[3]));
   std::memcpy(&h->g_w, &host_scr[2], 4);
 
-  if ((s_ = make_map(&h->map_b128, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 128, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK ||
-      (s_ = make_map(&h->map_b256, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 128, 256,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK)
+  if ((s_ = make_map(&h->map_b128, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_64B)) != QWAM_OK ||
+      (s_ = make_map(&h->map_b256, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 64, 256,
+                     CU_TENSOR_MAP_SWIZZLE_64B)) != QWAM_OK)
     return cleanup(s_);
+  if ((s_ = make_sf_map(&h->map_sfb, h->sf, round_up(static_cast<size_t>(N), 256), K)) != QWAM_OK) return cleanup(s_);
   if (r > 0) {
     if ((s_ = make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r))) !=
             QWAM_OK ||
@@ -361,9 +387,7 @@ qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, flo
   Arena* a = nullptr;
   QW_TRY(arena_get(h->dev, lay.total, &a));
   PrologueParams prm{};
-  prm.x = x;
   prm.chan = h->inv_s;
-  prm.vt_hi = h->vt_hi; prm.vt_lo = h->vt_lo; prm.v_hi = h->v_hi; prm.v_lo = h->v_lo;
   prm.rows = M;
   prm.K = h->K;
   prm.b = h->b;
@@ -377,7 +401,8 @@ qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, flo
   prm.g_out = arena_gx(*a);
   prm.z_out = z_out;
   prm.u_out = u_out;
-  QW_TRY(run_rows(prm, h->r, true, arena_amax(*a), st));
+  prm.err = arena_err(*a);
+  QW_TRY(run_rows(x, prm, h->r, h->vmaps, true, arena_amax(*a), st));
   if (arena_out) *arena_out = a;
   if (lay_out) *lay_out = lay;
   return QWAM_OK;
@@ -391,9 +416,11 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   const int tiles = ((M + 127) / 128) * ((h->N + pl.bn - 1) / pl.bn);
   if (pl.splits > 1 && tiles > kMaxTiles) return fail(QWAM_ERR_SHAPE, "too many output tiles for split-K");
   GemmMaps maps{};
-  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->base + lay.codes, h->K / 2, M, h->K / 2, 128, 128,
-                  CU_TENSOR_MAP_SWIZZLE_128B));
+  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->base + lay.codes, h->K / 2, M, h->K / 2, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_64B));
   maps.b = pl.bn == 256 ? h->map_b256 : h->map_b128;
+  QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K));
+  maps.sfb = h->map_sfb;
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
@@ -402,6 +429,11 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
     maps.u = maps.a;
     maps.l = maps.b;
   }
+  if (pl.splits == 1)
+    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B));
+  else
+    maps.y = maps.a;
   GemmParams p{};
   p.M = M; p.N = h->N; p.K = h->K;
   p.k_stages = pl.k_stages;
@@ -540,13 +572,16 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   QW_TRY(arena_get(dev, kHeaderBytes, &a));
   const int bn = N > 128 ? 256 : 128;
   GemmMaps maps{};
-  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B));
-  QW_TRY(make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, K / 2, N, K / 2, 128, bn, CU_TENSOR_MAP_SWIZZLE_128B));
+  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B));
+  QW_TRY(make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, K / 2, N, K / 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_64B));
   maps.u = maps.a;
   maps.l = maps.b;
+  maps.y = maps.a;
+  QW_TRY(make_sf_map(&maps.sfa, a_scales, round_up(static_cast<size_t>(M), 128), K));
+  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), bn), K));
   GemmParams p{};
   p.M = M; p.N = N; p.K = K;
-  p.k_stages = (K + 255) / 256;
+  p.k_stages = (K + 127) / 128;
   p.stages_per_split = p.k_stages;
   p.splits = 1;
   p.sfa = static_cast<const uint8_t*>(a_scales);
@@ -558,6 +593,18 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   p.counters = arena_counters(*a);
   p.err = arena_err(*a);
   QW_CUDA(launch_gemm(maps, p, bn, GemmEpilogue::RawF32, as_stream(stream)));
+  return QWAM_OK;
+}
+
+qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* splits, int* bn) {
+  if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
+  if (M < 0) return fail(QWAM_ERR_SHAPE, "M=%d must be >= 0", M);
+  const bool f = use_fused(M);
+  const Plan pl = plan_gemm(std::max(M, 1), h->N, h->K);
+  if (kernels) *kernels = M == 0 ? 0 : (f ? 2 : 3);
+  if (fused) *fused = f ? 1 : 0;
+  if (splits) *splits = pl.splits;
+  if (bn) *bn = pl.bn;
   return QWAM_OK;
 }
 

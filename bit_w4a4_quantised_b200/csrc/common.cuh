@@ -27,9 +27,17 @@ enum : uint32_t {
   DEVERR_BRANCH_WAIT = 1u << 4,
 };
 
-// About 2^26 polls; every poll of try_wait may also suspend the thread for a
-// hardware-chosen interval, so this is far beyond any legitimate wait.
-constexpr uint32_t kWaitLimit = 1u << 26;
+// A bounded wait gives up after this long (device global timer, nanoseconds).
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// Each try may suspend the waiting thread in hardware for up to this long; it is
+// woken as soon as the phase completes, so waiters do not poll shared memory.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -67,23 +75,26 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(addr), "r"(parity)
+      : "r"(addr), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 // Bounded wait for the phase with the given parity.  Returns false (and sets
-// `code` in the device error word) if the limit runs out.
+// `code` in the device error word) if kWaitLimitNs pass first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code) {
   const uint32_t addr = smem_u32(bar);
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(addr, parity)) return true;
+  if (mbar_try_wait(addr, parity, kSuspendHintNs)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait(addr, parity, kSuspendHintNs)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) break;
   }
   if (err) atomicOr(err, code);
   return false;
@@ -108,6 +119,42 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                    smem_u32(dst)),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
+}
+
+// Shared -> global tiled store (bulk group); the smem tile must be complete and
+// made visible to the async proxy (fence_proxy_async) before the call.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N committed bulk groups are still in flight (writes done).
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Generic-proxy shared-memory writes -> visible to TMA / tensor-core reads.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Barrier over the first `count` threads of the CTA (id 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  cluster_arrive();
+  cluster_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -157,6 +204,21 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, ui
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
+}
+// Instruction descriptor of kind::f16 with bf16 A/B, fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+// Instruction descriptor of kind::mxf4nvf4 (E2M1 A/B, UE4M3 scales, K = 64).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// tcgen05 smem-descriptor swizzle code and TMA-layout chunk permutation for a
+// K-major tile whose rows are W bytes (W = 32, 64 or 128, one swizzle atom).
+__host__ __device__ constexpr uint32_t umma_swizzle_code(int W) { return W == 128 ? 2u : (W == 64 ? 4u : 6u); }
+__device__ __forceinline__ int swz_chunk(int row, int chunk, int W) {
+  return chunk ^ ((row * W / 128) & (W / 16 - 1));
 }
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 operands, fp32 accumulate, K = 16.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,

@@ -12,13 +12,25 @@
 // quantisations", section "What ASP is...": y = (x~V)(W~V)^T + NVFP4GEMM(...) +
 // bias; branch kept in bf16).
 //
-// CTA = 6 warps: warp 0 issues TMA (tiles) and bulk copies (scales) into a
-// STAGES-deep shared-memory ring, warp 1 owns TMEM and issues tcgen05.cp (scales
-// -> TMEM) and tcgen05.mma, warps 2-5 drain the accumulator (tcgen05.ld).  Tile
-// 128 x BN, 256 K per stage (128 bytes of packed E2M1 per row = one 128B-swizzle
-// atom), K64 per MMA.  Split-K (small M): each split stores fp32 partials, the
-// last split to finish a tile (atomic ticket) sums them in split order and runs
-// the epilogue.  No TMA multicast.
+// Persistent kernel, one CTA per SM, tiles of 128 x BN (K in 128-element
+// stages, one 64B-swizzle atom of packed E2M1 per row, K64 per MMA; 6-8 stages
+// in flight to cover the ~0.7 us TMA latency).  Roles:
+//   producer warps  one per shared-memory ring slot; each stage is one
+//                   converged TMA instruction (A, B and their scale blocks on
+//                   four or five lanes).  A TMA instruction holds its warp for a
+//                   fixed ~600 cycles, so the slots have their own warps.
+//   MMA warp        owns TMEM; issues only tcgen05.mma (bf16 branch, then FP4).
+//   epilogue warps  eight, two per TMEM lane quarter (column halves).  While a
+//                   tile accumulates they copy each stage's scale blocks into the
+//                   slot's TMEM scale columns (tcgen05.cp; a warp's copies run one
+//                   after another, so eight warps share them and the copies run
+//                   beside the MMAs, not between them).  Then they drain the
+//                   accumulator to registers, release it to the next tile, add
+//                   bias, round to bf16, stage through 128B-swizzled smem and
+//                   store with TMA (ragged M / N are clipped by the tensor map).
+// Split-K (small M): fp32 partials; the last split of a tile (atomic ticket)
+// sums them in split order and writes y.  Every mbarrier wait is bounded.  No
+// TMA multicast.
 #include <algorithm>
 
 #include "common.cuh"
@@ -28,76 +40,100 @@ namespace qwam {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kStageBytes = 128;    // bytes per row per stage
-constexpr int kThreads = 192;
+constexpr int kStageBytes = 64;   // bytes per row per stage: 128 E2M1 codes, one 64B-swizzle atom
+constexpr int kK64 = 2;           // K64 MMA steps per stage
+constexpr int kEpiWarps = 8;
 
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 3 : 4;
+  static constexpr int STAGES = BN == 256 ? 6 : 8;
+  static constexpr int NSF = 1 + BN / 128;                  // scale block columns (A, B halves)
+  static constexpr int MMA_WARP = STAGES;
+  static constexpr int EPI_WARP0 = MMA_WARP + 1;
+  static constexpr int THREADS = 32 * (EPI_WARP0 + kEpiWarps);
   static constexpr int A_BYTES = kBM * kStageBytes;
   static constexpr int B_BYTES = BN * kStageBytes;
-  static constexpr int SFA_BYTES = 4 * 512;
-  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+  static constexpr int SFA_BYTES = kK64 * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * kK64 * 512;
   static constexpr int U_BYTES = kBM * 64;
   static constexpr int L_BYTES = BN * 64;
+  static constexpr int STG_BYTES = 4096;                    // per epilogue warp: 32 rows x 128 B
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
   static constexpr int OFF_U = OFF_SFB + STAGES * SFB_BYTES;
   static constexpr int OFF_L = OFF_U + U_BYTES;
-  static constexpr int OFF_BAR = OFF_L + L_BYTES;
-  static constexpr int NBAR = 2 * STAGES + 2;
+  static constexpr int OFF_STG = OFF_L + L_BYTES;
+  static constexpr int OFF_BAR = OFF_STG + kEpiWarps * STG_BYTES;
+  static constexpr int NBAR = 3 * STAGES + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  // TMEM columns: accumulator [0, BN), then per stage 4 K64 steps of scale
+  // TMEM columns: accumulator [0, BN), then per slot kK64 steps of scale
   // factors: A needs 4 columns per step (128 rows), B needs BN/32.
-  static constexpr int SF_COLS = 4 * 4 + 4 * (BN / 32);
+  static constexpr int SF_A_COLS = kK64 * 4;
+  static constexpr int SF_COLS = SF_A_COLS + kK64 * (BN / 32);
   static constexpr int TMEM_USED = BN + STAGES * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return pack2(bf16_bits_rn(a), bf16_bits_rn(b));
 }
 
+struct TileCoord {
+  int m0, n0, split;
+};
+
+// Tiles run M-fastest so consecutive CTAs reuse the same weight tile from L2.
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bn) {
+  const int mt = t % tiles_m;
+  const int rest = t / tiles_m;
+  return {mt * kBM, (rest % tiles_n) * bn, rest / tiles_n};
+}
+
 template <int BN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmSA,
+                    const __grid_constant__ CUtensorMap tmSB, const GemmParams p) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* empty = full + C::STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // TMA landed
+  uint64_t* sf_ready = full + C::STAGES;                            // scale copies done
+  uint64_t* empty = sf_ready + C::STAGES;                           // MMAs done with slot
   uint64_t* branch_full = empty + C::STAGES;
-  uint64_t* acc_full = branch_full + 1;
+  uint64_t* branch_empty = branch_full + 1;
+  uint64_t* acc_full = branch_empty + 1;
+  uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   uint32_t* last_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM, split = blockIdx.z;
-  const int s_begin = split * p.stages_per_split;
-  const int s_end = min(s_begin + p.stages_per_split, p.k_stages);
-  const int n_st = max(0, s_end - s_begin);
+  const int tiles_m = (p.M + kBM - 1) / kBM;
+  const int tiles_n = (p.N + BN - 1) / BN;
+  const int n_tiles = tiles_m * tiles_n * p.splits;
   const int k64_total = p.K / 64;
-  const bool do_branch = p.has_branch && split == 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
+      mbar_init(&sf_ready[i], kEpiWarps);
       mbar_init(&empty[i], 1);
     }
     mbar_init(branch_full, 1);
+    mbar_init(branch_empty, 1);
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiWarps);
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -106,178 +142,316 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- producer ----------------
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    if (do_branch) {
-      tma_prefetch_desc(&tmU);
-      tma_prefetch_desc(&tmL);
-      mbar_arrive_expect_tx(branch_full, static_cast<uint32_t>((kBM + BN) * p.branch_k * 2));
-      tma_load_2d(smem + C::OFF_U, &tmU, branch_full, 0, m0);
-      tma_load_2d(smem + C::OFF_L, &tmL, branch_full, 0, n0);
+  // stage range [s_begin, s_begin + n_st) of a split
+  auto stage_range = [&](int split, int& s_begin, int& n_st) {
+    s_begin = split * p.stages_per_split;
+    const int s_end = min(s_begin + p.stages_per_split, p.k_stages);
+    n_st = max(0, s_end - s_begin);
+  };
+
+  if (warp < C::MMA_WARP) {
+    // ------------------------------------------------ producers: warp st owns slot st
+    const int st = warp;
+    if (lane == 0 && st == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      tma_prefetch_desc(&tmSA);
+      tma_prefetch_desc(&tmSB);
+      if (p.has_branch) {
+        tma_prefetch_desc(&tmU);
+        tma_prefetch_desc(&tmL);
+      }
     }
-    int issued = 0;
-    for (int i = 0; i < n_st; ++i) {
-      const int st = i % C::STAGES;
-      const uint32_t ph = (i / C::STAGES) & 1;
-      if (!mbar_wait(&empty[st], ph ^ 1u, p.err, DEVERR_PRODUCER_WAIT)) break;
-      const int s = s_begin + i;
-      const int nk = min(4, k64_total - 4 * s);
-      const uint32_t sfb = static_cast<uint32_t>(nk) * 512u;
-      mbar_arrive_expect_tx(&full[st], C::A_BYTES + C::B_BYTES + sfb * (1 + BN / 128));
-      tma_load_2d(smem + C::OFF_A + st * C::A_BYTES, &tmA, &full[st], s * kStageBytes, m0);
-      tma_load_2d(smem + C::OFF_B + st * C::B_BYTES, &tmB, &full[st], s * kStageBytes, n0);
-      bulk_load(smem + C::OFF_SFA + st * C::SFA_BYTES,
-                p.sfa + (static_cast<size_t>(m0 / 128) * k64_total + 4 * s) * 512, sfb, &full[st]);
-#pragma unroll
-      for (int j = 0; j < BN / 128; ++j)
-        bulk_load(smem + C::OFF_SFB + st * C::SFB_BYTES + j * 2048,
-                  p.sfb + (static_cast<size_t>(n0 / 128 + j) * k64_total + 4 * s) * 512, sfb, &full[st]);
-      ++issued;
-    }
-    // every copy this CTA started must land before it exits
-    for (int i = max(0, issued - C::STAGES); i < issued; ++i)
-      mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
-    if (do_branch) mbar_wait(branch_full, 0, p.err, DEVERR_DRAIN_WAIT);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer ----------------
-    const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                               (static_cast<uint32_t>(kBM >> 4) << 24);
-    uint32_t accum = 0;
+    int g = 0;  // global stage counter of this CTA
+    int last = -1, nbranch = 0;
     bool ok = true;
-    if (do_branch) {
-      ok = mbar_wait(branch_full, 0, p.err, DEVERR_BRANCH_WAIT);
-      if (ok) {
-        tc_fence_after();
-        const uint32_t idesc_bf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                                    (static_cast<uint32_t>(kBM >> 4) << 24);
-        const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
-        const uint32_t sbo = 8u * p.branch_k * 2u;
-        const uint32_t us = smem_u32(smem + C::OFF_U), ls = smem_u32(smem + C::OFF_L);
-        for (int kk = 0; kk < p.branch_k / 16; ++kk) {
-          mma_bf16(tmem, smem_desc(us + kk * 32, 16, sbo, layout), smem_desc(ls + kk * 32, 16, sbo, layout),
-                   idesc_bf16, accum);
-          accum = 1;
+    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN);
+      int s_begin, n_st;
+      stage_range(tc.split, s_begin, n_st);
+      if (p.has_branch && tc.split == 0 && st == C::STAGES - 1) {
+        // branch operands of this tile, once the previous tile's branch MMAs are done
+        int bok = 1;
+        if (lane == 0) {
+          bok = (nbranch == 0 || mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_PRODUCER_WAIT)) ? 1 : 0;
+          if (bok) mbar_arrive_expect_tx(branch_full, static_cast<uint32_t>((kBM + BN) * p.branch_k * 2));
         }
+        bok = __shfl_sync(0xffffffffu, bok, 0);
+        if (!bok) break;
+        if (lane < 2)
+          tma_load_2d(smem + (lane ? C::OFF_L : C::OFF_U), lane ? &tmL : &tmU, branch_full, 0, lane ? tc.n0 : tc.m0);
+        ++nbranch;
+      }
+      for (int i = 0; i < n_st; ++i, ++g) {
+        if (g % C::STAGES != st) continue;
+        const uint32_t ph = (g / C::STAGES) & 1;
+        int wok = 1;
+        if (lane == 0) wok = mbar_wait(&empty[st], ph ^ 1u, p.err, DEVERR_PRODUCER_WAIT) ? 1 : 0;
+        wok = __shfl_sync(0xffffffffu, wok, 0);
+        if (!wok) {
+          ok = false;
+          break;
+        }
+        const int s = s_begin + i;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
+        __syncwarp();
+        // one converged instruction: A, B, A scales, B scales (1 + BN/128 blocks of 1 KB)
+        if (lane < 3 + BN / 128) {
+          const CUtensorMap* m;
+          uint8_t* dst;
+          int x, y;
+          if (lane == 0) {
+            m = &tmA; dst = smem + C::OFF_A + st * C::A_BYTES; x = s * kStageBytes; y = tc.m0;
+          } else if (lane == 1) {
+            m = &tmB; dst = smem + C::OFF_B + st * C::B_BYTES; x = s * kStageBytes; y = tc.n0;
+          } else if (lane == 2) {
+            m = &tmSA; dst = smem + C::OFF_SFA + st * C::SFA_BYTES; x = 0;
+            y = 2 * ((tc.m0 / 128) * k64_total + kK64 * s);
+          } else {
+            const int j = lane - 3;
+            m = &tmSB; dst = smem + C::OFF_SFB + st * C::SFB_BYTES + j * (kK64 * 512); x = 0;
+            y = 2 * ((tc.n0 / 128 + j) * k64_total + kK64 * s);
+          }
+          tma_load_2d(dst, m, &full[st], x, y);
+        }
+        last = g;
       }
     }
-    for (int i = 0; ok && i < n_st; ++i) {
-      const int st = i % C::STAGES;
-      const uint32_t ph = (i / C::STAGES) & 1;
-      if (!mbar_wait(&full[st], ph, p.err, DEVERR_MMA_WAIT)) break;
-      tc_fence_after();
-      const int s = s_begin + i;
-      const int nk = min(4, k64_total - 4 * s);
-      const uint32_t sfa_col = BN + st * C::SF_COLS;
-      const uint32_t sfb_col = sfa_col + 16;
-      const uint32_t sfa_s = smem_u32(smem + C::OFF_SFA + st * C::SFA_BYTES);
-      const uint32_t sfb_s = smem_u32(smem + C::OFF_SFB + st * C::SFB_BYTES);
-      for (int kk = 0; kk < nk; ++kk) {
-        tmem_cp_32x128b_x4(tmem + sfa_col + kk * 4, smem_desc(sfa_s + kk * 512, 0, 128, 0));
-#pragma unroll
-        for (int j = 0; j < BN / 128; ++j)
-          tmem_cp_32x128b_x4(tmem + sfb_col + kk * (BN / 32) + j * 4,
-                             smem_desc(sfb_s + j * 2048 + kk * 512, 0, 128, 0));
-      }
-      const uint32_t a_s = smem_u32(smem + C::OFF_A + st * C::A_BYTES);
-      const uint32_t b_s = smem_u32(smem + C::OFF_B + st * C::B_BYTES);
-      for (int kk = 0; kk < nk; ++kk) {
-        mma_mxf4nvf4(tmem, smem_desc(a_s + kk * 32, 16, 1024, 2), smem_desc(b_s + kk * 32, 16, 1024, 2), idesc_fp4,
-                     tmem + sfa_col + kk * 4, tmem + sfb_col + kk * (BN / 32), accum);
-        accum = 1;
-      }
-      tc_commit(&empty[st]);
+    // every copy this warp started must land before the CTA exits
+    if (lane == 0) {
+      if (last >= 0) mbar_wait(&full[st], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
+      if (nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
     }
-    tc_commit(acc_full);
-  } else if (warp >= 2) {
-    // ---------------- epilogue ----------------
-    const int qd = warp & 3;  // TMEM lane quarter this warp may access
-    const bool ok = mbar_wait(acc_full, 0, p.err, DEVERR_EPILOGUE_WAIT);
     __syncwarp();
-    tc_fence_after();
-    const int row = m0 + qd * 32 + lane;
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_fp4 = idesc_mxf4(kBM, BN);
+      const uint32_t idesc_br = idesc_bf16(kBM, BN);
+      const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
+      const uint32_t sbo = 8u * p.branch_k * 2u;
+      const uint32_t us = smem_u32(smem + C::OFF_U), ls = smem_u32(smem + C::OFF_L);
+      int g = 0, tl = 0, nbranch = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tl) {
+        const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN);
+        int s_begin, n_st;
+        stage_range(tc.split, s_begin, n_st);
+        // the epilogue must have drained the previous tile's accumulator
+        if (!mbar_wait(acc_empty, (tl & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) break;
+        tc_fence_after();
+        uint32_t accum = 0;
+        if (p.has_branch && tc.split == 0) {
+          if (!mbar_wait(branch_full, nbranch & 1, p.err, DEVERR_BRANCH_WAIT)) break;
+          tc_fence_after();
+          for (int kk = 0; kk < p.branch_k / 16; ++kk) {
+            mma_bf16(tmem, smem_desc(us + kk * 32, 16, sbo, layout), smem_desc(ls + kk * 32, 16, sbo, layout),
+                     idesc_br, accum);
+            accum = 1;
+          }
+          tc_commit(branch_empty);
+          ++nbranch;
+        }
+        for (int i = 0; i < n_st; ++i, ++g) {
+          const int st = g % C::STAGES;
+          const uint32_t ph = (g / C::STAGES) & 1;
+          if (!mbar_wait(&sf_ready[st], ph, p.err, DEVERR_MMA_WAIT) ||
+              !mbar_wait(&full[st], ph, p.err, DEVERR_MMA_WAIT)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int s = s_begin + i;
+          const int nk = min(kK64, k64_total - kK64 * s);
+          const uint32_t sf_col = BN + st * C::SF_COLS;
+          const uint32_t a_s = smem_u32(smem + C::OFF_A + st * C::A_BYTES);
+          const uint32_t b_s = smem_u32(smem + C::OFF_B + st * C::B_BYTES);
+          for (int kk = 0; kk < nk; ++kk) {
+            mma_mxf4nvf4(tmem, smem_desc(a_s + kk * 32, 16, 512, 4), smem_desc(b_s + kk * 32, 16, 512, 4), idesc_fp4,
+                         tmem + sf_col + kk * 4, tmem + sf_col + C::SF_A_COLS + kk * (BN / 32), accum);
+            accum = 1;
+          }
+          tc_commit(&empty[st]);
+        }
+        tc_commit(acc_full);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue
+    const int ew = warp - C::EPI_WARP0;  // 0..7
+    const int qd = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = ew >> 2;            // column half [half*BN/2, (half+1)*BN/2)
+    const int et = threadIdx.x - 32 * C::EPI_WARP0;
+    constexpr int HC = BN / 2;           // columns per thread
     const float gs = __fmul_rn(p.g_a_ptr ? *p.g_a_ptr : p.g_a, p.g_b);
     const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
-    if (ok) {
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + c * 32, r);
-        tmem_ld_wait();
-        const int n = n0 + c * 32;
-        if (row >= p.M || n >= p.N) continue;
-        const int nvalid = min(32, p.N - n);  // 16 or 32 (N % 16 == 0)
-        if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
-          uint16_t* y = static_cast<uint16_t*>(p.y) + static_cast<size_t>(row) * p.N + n;
-          for (int h = 0; h < nvalid / 16; ++h) {
-            float bv[16];
+    uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
+    int tl = 0, g = 0;
+    bool sf_ok = true;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN);
+      // Scale blocks of this tile's stages: smem -> TMEM.  A warp's tcgen05.cp
+      // instructions run one after another (~115 cycles each), so the 4 * NSF
+      // copies of a stage are spread over the eight epilogue warps, which are
+      // otherwise idle while the tile accumulates.
+      {
+        int s_begin, n_st;
+        stage_range(tc.split, s_begin, n_st);
+        for (int i = 0; i < n_st; ++i, ++g) {
+          const int st = g % C::STAGES;
+          int wok = 1;
+          if (lane == 0) wok = (sf_ok && mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_EPILOGUE_WAIT)) ? 1 : 0;
+          wok = __shfl_sync(0xffffffffu, wok, 0);
+          if (!wok) {
+            sf_ok = false;
+            continue;
+          }
+          if (lane == 0) {
+            tc_fence_after();
+            const int s = s_begin + i;
+            const int nk = min(kK64, k64_total - kK64 * s);
+            const uint32_t sf_col = BN + st * C::SF_COLS;
+            for (int c = ew; c < kK64 * C::NSF; c += kEpiWarps) {
+              const int col = c / kK64, kk = c % kK64;
+              if (kk >= nk) continue;
+              if (col == 0)
+                tmem_cp_32x128b_x4(tmem + sf_col + kk * 4,
+                                   smem_desc(smem_u32(smem + C::OFF_SFA + st * C::SFA_BYTES) + kk * 512, 0, 128, 0));
+              else
+                tmem_cp_32x128b_x4(
+                    tmem + sf_col + C::SF_A_COLS + kk * (BN / 32) + (col - 1) * 4,
+                    smem_desc(smem_u32(smem + C::OFF_SFB + st * C::SFB_BYTES) + (col - 1) * (kK64 * 512) + kk * 512, 0,
+                              128, 0));
+            }
+            tc_commit(&sf_ready[st]);
+          }
+          __syncwarp();
+        }
+      }
+      const bool ok = sf_ok && mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      __syncwarp();
+      tc_fence_after();
+      const int row = tc.m0 + qd * 32 + lane;
+      const int c0 = tc.n0 + half * HC;
+      if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
+        // drain: fp32 accumulator -> bf16 pairs in registers, then release
+        uint32_t packed[HC / 2];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) bv[j] = bias ? bf16_bits_to_float(__ldg(bias + n + 16 * h + j)) : 0.0f;
-            uint32_t o[8];
+        for (int q = 0; q < HC / 32; ++q) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + q * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 braw = make_uint4(0u, 0u, 0u, 0u);
+            if (bias && c0 + q * 32 + 8 * j < p.N) braw = __ldg(reinterpret_cast<const uint4*>(bias + c0 + q * 32 + 8 * j));
+            const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              packed[q * 16 + 4 * j + k] =
+                  pack_bf16x2(__fmaf_rn(__uint_as_float(r[8 * j + 2 * k]), gs, __uint_as_float(bw[k] << 16)),
+                              __fmaf_rn(__uint_as_float(r[8 * j + 2 * k + 1]), gs, __uint_as_float(bw[k] & 0xffff0000u)));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        if (ok) {
+          // stage 64 columns (32 rows x 128 B, 128B swizzle) per TMA store
+#pragma unroll
+          for (int cc = 0; cc < HC / 64; ++cc) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              o[j] = pack_bf16x2(__fmaf_rn(__uint_as_float(r[16 * h + 2 * j]), gs, bv[2 * j]),
-                                 __fmaf_rn(__uint_as_float(r[16 * h + 2 * j + 1]), gs, bv[2 * j + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(y + 16 * h);
-            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(packed[cc * 32 + 4 * j], packed[cc * 32 + 4 * j + 1], packed[cc * 32 + 4 * j + 2],
+                             packed[cc * 32 + 4 * j + 3]);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, stg, c0 + cc * 64, tc.m0 + qd * 32);
+              bulk_commit();
+            }
           }
-        } else {
+        }
+      } else {
+        // fp32 out (raw or split-K partial): direct row stores
+        const float sc = (EPI == static_cast<int>(GemmEpilogue::RawF32)) ? gs : 1.0f;
+#pragma unroll 1
+        for (int q = 0; q < HC / 32; ++q) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + q * 32, r);
+          tmem_ld_wait();
+          const int n = c0 + q * 32;
+          if (!ok || row >= p.M || n >= p.N) continue;
           float* dst = (EPI == static_cast<int>(GemmEpilogue::RawF32))
                            ? p.out_f32 + static_cast<size_t>(row) * p.N + n
-                           : p.partial + (static_cast<size_t>(split) * p.M + row) * p.N + n;
-          const float sc = (EPI == static_cast<int>(GemmEpilogue::RawF32)) ? gs : 1.0f;
-          for (int j = 0; j < nvalid; j += 4)
-            *reinterpret_cast<float4*>(dst + j) =
-                make_float4(__fmul_rn(__uint_as_float(r[j]), sc), __fmul_rn(__uint_as_float(r[j + 1]), sc),
-                            __fmul_rn(__uint_as_float(r[j + 2]), sc), __fmul_rn(__uint_as_float(r[j + 3]), sc));
+                           : p.partial + (static_cast<size_t>(tc.split) * p.M + row) * p.N + n;
+          float4* d4 = reinterpret_cast<float4*>(dst);
+          const int nv = min(32, p.N - n) / 4;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k < nv)
+              d4[k] = make_float4(__fmul_rn(__uint_as_float(r[4 * k]), sc), __fmul_rn(__uint_as_float(r[4 * k + 1]), sc),
+                                  __fmul_rn(__uint_as_float(r[4 * k + 2]), sc),
+                                  __fmul_rn(__uint_as_float(r[4 * k + 3]), sc));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        if constexpr (EPI == static_cast<int>(GemmEpilogue::SplitK)) {
+          __threadfence();
+          epi_bar();
+          const int tile = tc.m0 / kBM + tiles_m * (tc.n0 / BN);
+          if (et == 0) {
+            const uint32_t prev = atomicAdd(&p.counters[tile], 1u);
+            *last_flag = (prev == static_cast<uint32_t>(p.splits - 1)) ? 1u : 0u;
+          }
+          epi_bar();
+          if (*last_flag) {
+            __threadfence();
+            const int rows_v = min(kBM, p.M - tc.m0), cols_v = min(BN, p.N - tc.n0);
+            const int c4 = cols_v / 4;
+            uint16_t* y = static_cast<uint16_t*>(p.y);
+            for (int idx = et; idx < rows_v * c4; idx += 32 * kEpiWarps) {
+              const int m = tc.m0 + idx / c4, n = tc.n0 + (idx % c4) * 4;
+              float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int sp = 0; sp < p.splits; ++sp) {
+                const float4 v =
+                    __ldcg(reinterpret_cast<const float4*>(p.partial + (static_cast<size_t>(sp) * p.M + m) * p.N + n));
+                sacc.x = __fadd_rn(sacc.x, v.x);
+                sacc.y = __fadd_rn(sacc.y, v.y);
+                sacc.z = __fadd_rn(sacc.z, v.z);
+                sacc.w = __fadd_rn(sacc.w, v.w);
+              }
+              float b4[4] = {0.f, 0.f, 0.f, 0.f};
+              if (bias) {
+                const uint2 braw = __ldg(reinterpret_cast<const uint2*>(bias + n));
+                b4[0] = __uint_as_float(braw.x << 16);
+                b4[1] = __uint_as_float(braw.x & 0xffff0000u);
+                b4[2] = __uint_as_float(braw.y << 16);
+                b4[3] = __uint_as_float(braw.y & 0xffff0000u);
+              }
+              *reinterpret_cast<uint2*>(y + static_cast<size_t>(m) * p.N + n) =
+                  make_uint2(pack_bf16x2(__fmaf_rn(sacc.x, gs, b4[0]), __fmaf_rn(sacc.y, gs, b4[1])),
+                             pack_bf16x2(__fmaf_rn(sacc.z, gs, b4[2]), __fmaf_rn(sacc.w, gs, b4[3])));
+            }
+            if (et == 0) p.counters[tile] = 0u;
+          }
+          epi_bar();  // the ticket flag is reused by the next tile
         }
       }
     }
-    if constexpr (EPI == static_cast<int>(GemmEpilogue::SplitK)) {
-      __threadfence();
-      epi_bar();
-      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-      if (threadIdx.x == 64) {
-        const uint32_t prev = atomicAdd(&p.counters[tile], 1u);
-        *last_flag = (prev == static_cast<uint32_t>(p.splits - 1)) ? 1u : 0u;
-      }
-      epi_bar();
-      if (*last_flag) {
-        __threadfence();
-        const int t = threadIdx.x - 64;
-        const int rows_v = min(kBM, p.M - m0), cols_v = min(BN, p.N - n0);
-        const int c4 = cols_v / 4;
-        uint16_t* y = static_cast<uint16_t*>(p.y);
-        for (int idx = t; idx < rows_v * c4; idx += 128) {
-          const int m = m0 + idx / c4, n = n0 + (idx % c4) * 4;
-          float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int sp = 0; sp < p.splits; ++sp) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(p.partial + (static_cast<size_t>(sp) * p.M + m) * p.N + n));
-            s.x = __fadd_rn(s.x, v.x);
-            s.y = __fadd_rn(s.y, v.y);
-            s.z = __fadd_rn(s.z, v.z);
-            s.w = __fadd_rn(s.w, v.w);
-          }
-          float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-          if (bias) {
-            b0 = bf16_bits_to_float(__ldg(bias + n));
-            b1 = bf16_bits_to_float(__ldg(bias + n + 1));
-            b2 = bf16_bits_to_float(__ldg(bias + n + 2));
-            b3 = bf16_bits_to_float(__ldg(bias + n + 3));
-          }
-          *reinterpret_cast<uint2*>(y + static_cast<size_t>(m) * p.N + n) =
-              make_uint2(pack_bf16x2(__fmaf_rn(s.x, gs, b0), __fmaf_rn(s.y, gs, b1)),
-                         pack_bf16x2(__fmaf_rn(s.z, gs, b2), __fmaf_rn(s.w, gs, b3)));
-        }
-        if (t == 0) p.counters[tile] = 0u;
-      }
+    if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
+      if (lane == 0) bulk_wait<0>();
+      __syncwarp();
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     __syncwarp();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -287,10 +461,16 @@ template <int BN, int EPI>
 cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   using C = Cfg<BN>;
   auto kern = fp4_gemm_kernel<BN, EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  dim3 grid((p.N + BN - 1) / BN, (p.M + kBM - 1) / kBM, p.splits);
-  kern<<<grid, kThreads, C::SMEM, st>>>(m.a, m.b, m.u, m.l, p);
+  static const cudaError_t smem_attr =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (smem_attr != cudaSuccess) return smem_attr;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN) * p.splits;
+  const int grid = std::min(tiles, sms);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(m.a, m.b, m.u, m.l, m.y, m.sfa, m.sfb, p);
   return cudaGetLastError();
 }
 

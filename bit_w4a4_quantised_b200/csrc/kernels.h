@@ -11,21 +11,24 @@ namespace qwam {
 // One "rows" job of the activation prologue / weight prepare:
 //   T~ = (T * chan) H,  c = T~ V,  Z = T~ - c V^T,  quantise(Z),
 // with T = x, chan = 1/s on the activation side and T = W, chan = s on the
-// weight side.
+// weight side.  T and V reach the kernel through TMA tensor maps.
+struct ProMaps {
+  CUtensorMap x;      // T bf16 [rows, K], box 64 x 128 rows, 128B swizzle
+  CUtensorMap vt_hi;  // V^T bf16 [r, K], box 64 x r, 128B swizzle
+  CUtensorMap vt_lo;
+  CUtensorMap v_hi;   // V bf16 [K, r], box r x 128 rows, 2r-byte swizzle
+  CUtensorMap v_lo;
+};
+
 struct PrologueParams {
-  const void* x;          // bf16 [rows, K]
   const float* chan;      // fp32 [K]
-  const uint16_t* vt_hi;  // bf16 bits [r, K]  (V^T, high part)
-  const uint16_t* vt_lo;  // bf16 bits [r, K]  (V^T, low part)
-  const uint16_t* v_hi;   // bf16 bits [K, r]
-  const uint16_t* v_lo;   // bf16 bits [K, r]
   int rows;
   int K;
   int b;                  // Hadamard block (power of two, <= 128)
   int chunks;             // 128-column chunks per CTA
   float hscale;           // fp32(1 / sqrt(b))
-  float* u_glob;          // fp32 [rows, r]: written by phase 1, read by phase 2
-  uint32_t* amax_glob;    // fp32 bits of max|Z|: atomicMax'd by phase 1
+  float* u_glob;          // fp32 [rows, r]: written by Stats, read by Quantise
+  uint32_t* amax_glob;    // fp32 bits of max|Z|: atomicMax'd by Stats
   uint8_t* codes;         // [rows, K/2]
   uint8_t* sf;            // tiled scales, rows padded to 128
   uint16_t* branch;       // bf16 bits [rows, r]
@@ -34,14 +37,16 @@ struct PrologueParams {
   float* g_out;           // fp32 scalar: the per-tensor scale of Z
   float* z_out;           // optional fp32 [rows, K] (debug export of Z)
   float* u_out;           // optional fp32 [rows, r] (debug export of c)
+  uint32_t* err;          // device error word for bounded waits
 };
 
 enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2 };
 
-// Fused: one cluster row group holds every row (rows <= 64); Stats/Quantise:
-// the two-launch form for any row count (Stats needs *amax_glob == 0).
-cudaError_t launch_prologue(const PrologueParams& p, int r, PrologueMode mode, int cluster, cudaStream_t st);
-size_t prologue_smem_bytes(int r, PrologueMode mode, int chunks);
+// Grid: parts x ceil(rows / 128) CTAs; Fused and Stats (r > 0) launch the
+// parts of a row tile as one cluster.  Fused requires rows <= 128; Stats
+// requires *amax_glob == 0.
+cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode, int parts,
+                            cudaStream_t st);
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st);
 cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, uint16_t* vt_hi,
@@ -73,10 +78,13 @@ struct GemmParams {
 };
 
 struct GemmMaps {
-  CUtensorMap a;  // codes A [M, K/2] u8, box 128 B x 128 rows, 128B swizzle
-  CUtensorMap b;  // codes B [N, K/2] u8, box 128 B x BN rows, 128B swizzle
+  CUtensorMap a;  // codes A [M, K/2] u8, box 64 B x 128 rows, 64B swizzle
+  CUtensorMap b;  // codes B [N, K/2] u8, box 64 B x BN rows, 64B swizzle
   CUtensorMap u;  // branch A [M, r] bf16, box r x 128 rows
   CUtensorMap l;  // branch B [N, r] bf16, box r x BN rows
+  CUtensorMap y;    // output y [M, N] bf16, box 64 x 32 rows, 128B swizzle (bf16 epilogue)
+  CUtensorMap sfa;  // A scales viewed as u8 [atoms * 2, 256], box 256 x 4 (one stage, 1 KB)
+  CUtensorMap sfb;  // B scales, same view
 };
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int bn, GemmEpilogue epi, cudaStream_t st);

@@ -1,0 +1,95 @@
+// Kernels outside the per-call hot path: the standalone NVFP4 quantiser (used by
+// tests and tools on arbitrary fp32 tensors) and the prepare-time helpers that
+// derive 1/s and the bf16 hi/lo split of V stored in a layer handle.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "quant.cuh"
+
+namespace qwam {
+namespace {
+
+// --- standalone quantiser (tests and tools) -------------------------------
+__global__ void amax_kernel(const float* __restrict__ T, size_t n, uint32_t* amax) {
+  float m = 0.0f;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    m = fmaxf(m, fabsf(T[i]));
+  const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax, w);
+}
+
+__global__ void quantize_blocks_kernel(const float* __restrict__ T, int rows, int K, uint8_t* codes, uint8_t* sf,
+                                       const uint32_t* amax, float* g_out) {
+  const size_t nblk = static_cast<size_t>(rows) * (K / 16);
+  const float g = global_scale_from_amax(__uint_as_float(*amax));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  for (size_t bi = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; bi < nblk;
+       bi += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(bi / (K / 16));
+    const int kb = static_cast<int>(bi % (K / 16));
+    float v[16];
+    const float4* src = reinterpret_cast<const float4*>(T + static_cast<size_t>(row) * K + kb * 16);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 t = src[j];
+      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+    }
+    uint32_t c2[2];
+    const uint32_t S = quant_block16(v, g, c2);
+    *reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2) + kb * 8) = make_uint2(c2[0], c2[1]);
+    sf[sf_offset(row, kb, K)] = static_cast<uint8_t>(S);
+  }
+}
+
+// --- prepare helpers -------------------------------------------------------
+__global__ void recip_kernel(const float* __restrict__ s, float* __restrict__ inv_s, int K, uint32_t* err) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= K) return;
+  const float v = s[i];
+  if (!(v > 0.0f) || !isfinite(v)) atomicOr(err, 1u);
+  inv_s[i] = __frcp_rn(v);
+}
+
+__global__ void split_v_kernel(const float* __restrict__ V, int K, int r, uint16_t* v_hi, uint16_t* v_lo,
+                               uint16_t* vt_hi, uint16_t* vt_lo) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= K * r) return;
+  const int k = i / r, j = i % r;
+  uint16_t hi, lo;
+  split_bf16(V[i], hi, lo);
+  v_hi[i] = hi;
+  v_lo[i] = lo;
+  vt_hi[static_cast<size_t>(j) * K + k] = hi;
+  vt_lo[static_cast<size_t>(j) * K + k] = lo;
+}
+
+}  // namespace
+
+cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st) {
+  recip_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, uint16_t* vt_hi,
+                           uint16_t* vt_lo, cudaStream_t st) {
+  const int n = K * r;
+  split_v_kernel<<<(n + 255) / 256, 256, 0, st>>>(V, K, r, v_hi, v_lo, vt_hi, vt_lo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_fp32(const float* T, int rows, int K, uint8_t* codes, uint8_t* sf, float* g_out,
+                                 uint32_t* amax_scratch, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(amax_scratch, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  const size_t n = static_cast<size_t>(rows) * K;
+  const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 8));
+  amax_kernel<<<blocks, 256, 0, st>>>(T, n, amax_scratch);
+  const size_t nblk = static_cast<size_t>(rows) * (K / 16);
+  const int qblocks = static_cast<int>(std::min<size_t>((nblk + 255) / 256, 148 * 8));
+  quantize_blocks_kernel<<<qblocks, 256, 0, st>>>(T, rows, K, codes, sf, amax_scratch, g_out);
+  return cudaGetLastError();
+}
+
+}  // namespace qwam

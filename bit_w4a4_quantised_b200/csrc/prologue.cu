@@ -1,28 +1,32 @@
-// Activation prologue and weight prepare kernels.
+// Activation prologue and weight prepare: one row pipeline for both sides of
+// the deflated ASP layer ("FastWAM UR3 3-task — 4-bit quantisations", section
+// "What ASP is, and what the deflated form means"):
 //
-// Both sides of the deflated ASP layer ("FastWAM UR3 3-task — 4-bit
-// quantisations", section "What ASP is, and what the deflated form means") run
-// the same row pipeline:
+//   T~ = (T * chan) H           per-channel scale, block FWHT (one thread = one row)
+//   c  = T~ V                   rank-r coordinates, tcgen05 bf16 MMA into TMEM
+//   Z  = T~ - c V^T             deflation, tcgen05 bf16 MMA into TMEM
+//   amax(Z) -> g, quantise(Z)   NVFP4 codes + 128x4-tiled E4M3 scales
+//   branch operand              bf16(c)  (weight side: W~V)  or
+//                               bf16(c / (g_x g_w))  (activation side)
 //
-//   T~ = (T * chan) H            per-channel scale, then block-FWHT in registers
-//   c  = T~ V                    rank-r coordinates (bf16x3 split warp MMA)
-//   Z  = T~ - c V^T              deflation, again bf16x3
-//   amax(Z) -> g,  quantise(Z)   NVFP4 codes + tiled E4M3 scales
-//   branch operand               bf16(c) (weights: W~V) or bf16(c / (g_x g_w))
+// T = x and chan = 1/s on the activation side, T = W and chan = s on the weight
+// side.  Both rank-r products run on the tensor cores with a hi/lo bf16 split of
+// each operand (three MMAs per K step; plain bf16 flips ~0.2 % of the FP4 codes
+// against a float64 reference, the split keeps it below 0.01 %).
 //
-// Work split: a CTA of 4 warps owns 64 rows x (chunks * 128) columns; warp w
-// owns 16 rows.  The CTAs of one row group form a thread-block cluster along
-// K; their partial c sums are exchanged through distributed shared memory in a
-// fixed rank order (deterministic).  With <= 64 rows one cluster covers the
-// whole tensor, so the per-tensor amax is a cluster reduction and the kernel
-// finishes in one launch (Fused).  Otherwise a Stats launch writes c and
-// atomically maxes amax, and a Quantise launch recomputes Z bit-identically
-// (same code path, explicit round-to-nearest intrinsics, same fp32 c) and
-// quantises it.
+// CTA = 128 rows (one TMEM lane per row) x `chunks` 128-column chunks, 7 warps:
+//   warps 0-3  row threads: read their row of x from a TMA-filled ring, scale,
+//              FWHT in registers, write T~ (hi/lo) as the MMA A operand, read
+//              u and Z from TMEM, reduce amax, quantise in registers;
+//   warps 4, 6 TMA producers (x tiles, V tiles, chan), one per ring slot;
+//   warp 5     TMEM owner and MMA issuer.
+// The CTAs of a row tile form a cluster along K: partial c is summed across it
+// through distributed shared memory in rank order (deterministic).
 //
-// The rank-r products use the legacy m16n8k16 warp MMA with a hi/lo bf16 split
-// of both operands (three products per step): plain bf16 flips ~0.2 % of the
-// FP4 codes against a float64 reference, the split keeps it below 0.01 %.
+// Modes: Fused (rows <= 128: the cluster holds the whole tensor, so amax is a
+// cluster reduction and one launch finishes the job), Stats (c to global,
+// atomic amax) and Quantise (reads c and amax, recomputes Z bit-identically from
+// the same code and data, quantises).  Every wait on an mbarrier is bounded.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -34,499 +38,588 @@ namespace cg = cooperative_groups;
 namespace qwam {
 namespace {
 
-constexpr int kGroupRows = 64;
+constexpr int kRows = 128;
 constexpr int kChunk = 128;
-constexpr int kPad = 8;  // row stride = 8 (mod 32) floats: conflict-free float2 fragment reads
+constexpr int kThreads = 224;  // 4 row warps, producer warps 4 and 6, MMA warp 5
 
-__device__ __forceinline__ uint32_t ldg_u32(const uint16_t* p) {
-  return __ldg(reinterpret_cast<const unsigned int*>(p));
+template <int R, int MODE>
+struct PCfg {
+  static constexpr bool kMMA = R > 0;
+  static constexpr bool kProj = R > 0 && MODE != 2;        // sweep computing c
+  static constexpr bool kA = MODE != 2 && R > 0;           // cluster exchange of c
+  static constexpr bool kB = MODE == 0;                    // cluster exchange of amax
+  static constexpr bool kC = kA || kB;                     // keep smem alive for peers
+  static constexpr int X_BYTES = kRows * kChunk * 2;       // two 64-column SW128 boxes
+  static constexpr int V_BYTES = 512 * R;                  // V^T hi/lo (sweep 1) or V hi/lo
+  static constexpr int CH_BYTES = kChunk * 4;
+  static constexpr int SLOT = (X_BYTES + V_BYTES + CH_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_XT = 2 * SLOT;                  // T~ hi/lo as MMA A, 4 x 16 KB
+  static constexpr int XT_BYTES = kProj ? 4 * 16384 : 0;
+  static constexpr int OFF_UA = OFF_XT + XT_BYTES;         // c hi/lo as MMA A
+  static constexpr int UA_BYTES = kMMA ? 512 * R : 0;
+  static constexpr int OFF_BAR = OFF_UA + UA_BYTES;
+  static constexpr int OFF_MISC = OFF_BAR + 128;
+  static constexpr int SMEM = OFF_MISC + 64 + 1024;
+  static constexpr int UP_STRIDE = R + 4;                  // fp32 partial c rows (aliases T~)
+  static constexpr uint32_t TMEM_COLS = kMMA ? (MODE == 2 ? 128u : 256u) : 32u;
+  static_assert(!kProj || kRows * UP_STRIDE * 4 <= 32768, "partial and parked c must fit in the T~ area");
+};
+
+__device__ __forceinline__ void unpack8(uint4 w, float* o) {
+  o[0] = __uint_as_float(w.x << 16); o[1] = __uint_as_float(w.x & 0xffff0000u);
+  o[2] = __uint_as_float(w.y << 16); o[3] = __uint_as_float(w.y & 0xffff0000u);
+  o[4] = __uint_as_float(w.z << 16); o[5] = __uint_as_float(w.z & 0xffff0000u);
+  o[6] = __uint_as_float(w.w << 16); o[7] = __uint_as_float(w.w & 0xffff0000u);
 }
 
-// In-register fast Walsh-Hadamard transform over blocks of b columns; this lane
-// holds 4 consecutive columns, partner lanes are reached with xor shuffles.
-// Natural (Sylvester) order: (lo, hi) -> (lo + hi, lo - hi).
-__device__ __forceinline__ void fwht_lane4(float (&v)[4], int b, int lane) {
-  if (b >= 2) {
-    const float a0 = __fadd_rn(v[0], v[1]), a1 = __fsub_rn(v[0], v[1]);
-    const float a2 = __fadd_rn(v[2], v[3]), a3 = __fsub_rn(v[2], v[3]);
-    v[0] = a0; v[1] = a1; v[2] = a2; v[3] = a3;
-  }
-  if (b >= 4) {
-    const float a0 = __fadd_rn(v[0], v[2]), a2 = __fsub_rn(v[0], v[2]);
-    const float a1 = __fadd_rn(v[1], v[3]), a3 = __fsub_rn(v[1], v[3]);
-    v[0] = a0; v[1] = a1; v[2] = a2; v[3] = a3;
-  }
-  for (int h = 4; h < b; h <<= 1) {
-    const int m = h >> 2;
-    const bool upper = (lane & m) != 0;
+// This thread's row of one chunk: x (bf16, SW128 TMA tile) * chan, then the
+// block FWHT in registers (Sylvester order, butterflies (lo+hi, lo-hi)), then
+// the 1/sqrt(b) scale.  Identical code and op order in every sweep.
+__device__ __forceinline__ void rotate_row(const uint8_t* slot, const float* chan, int t, int b, float hscale,
+                                           float (&v)[kChunk]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+  for (int h = 0; h < 2; ++h) {
+    const uint8_t* rowp = slot + h * 16384 + t * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((j ^ (t & 7)) << 4));
+      unpack8(w, v + h * 64 + j * 8);
     }
   }
-}
-
-// Rotate the warp's 16 rows of one 128-column chunk into shared memory.
-// Rows past p.rows read as zero.  Returns this lane's max |T~|.
-__device__ __forceinline__ float rotate_rows(const PrologueParams& p, int row0, int col, float* xt, int stride,
-                                             int lane) {
-  const float4 c = __ldg(reinterpret_cast<const float4*>(p.chan + col) + lane);
-  const uint16_t* x = static_cast<const uint16_t*>(p.x);
-  float amax = 0.0f;
-#pragma unroll 4
-  for (int i = 0; i < 16; ++i) {
-    const int row = row0 + i;
-    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (row < p.rows) {
-      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + static_cast<size_t>(row) * p.K + col) + lane);
-      v[0] = __fmul_rn(__uint_as_float(raw.x << 16), c.x);
-      v[1] = __fmul_rn(__uint_as_float(raw.x & 0xffff0000u), c.y);
-      v[2] = __fmul_rn(__uint_as_float(raw.y << 16), c.z);
-      v[3] = __fmul_rn(__uint_as_float(raw.y & 0xffff0000u), c.w);
-    }
-    fwht_lane4(v, p.b, lane);
-    float4 o;
-    o.x = __fmul_rn(v[0], p.hscale);
-    o.y = __fmul_rn(v[1], p.hscale);
-    o.z = __fmul_rn(v[2], p.hscale);
-    o.w = __fmul_rn(v[3], p.hscale);
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
-    *reinterpret_cast<float4*>(xt + i * stride + 4 * lane) = o;
-  }
-  return amax;
-}
-
-__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
-  uint16_t ah, al, bh, bl;
-  split_bf16(a, ah, al);
-  split_bf16(b, bh, bl);
-  hi = pack2(ah, bh);
-  lo = pack2(al, bl);
-}
-
-// c[16 x R] += T~[16 x 128] * V[col.., 0..R) for the warp's rows (C fragments).
-template <int R>
-__device__ __forceinline__ void project(const PrologueParams& p, const float* xt, int stride, int col, int lane,
-                                        float (&u)[R / 8][4]) {
-  const int g = lane >> 2, q = lane & 3;
-#pragma unroll 2
-  for (int ks = 0; ks < kChunk / 16; ++ks) {
-    const float* r0 = xt + g * stride + ks * 16 + 2 * q;
-    const float* r1 = r0 + 8 * stride;
-    const float2 x00 = *reinterpret_cast<const float2*>(r0);
-    const float2 x10 = *reinterpret_cast<const float2*>(r1);
-    const float2 x01 = *reinterpret_cast<const float2*>(r0 + 8);
-    const float2 x11 = *reinterpret_cast<const float2*>(r1 + 8);
-    uint32_t ahi[4], alo[4];
-    split_pair(x00.x, x00.y, ahi[0], alo[0]);
-    split_pair(x10.x, x10.y, ahi[1], alo[1]);
-    split_pair(x01.x, x01.y, ahi[2], alo[2]);
-    split_pair(x11.x, x11.y, ahi[3], alo[3]);
-    const int kc = col + ks * 16 + 2 * q;
 #pragma unroll
-    for (int nt = 0; nt < R / 8; ++nt) {
-      const size_t off = static_cast<size_t>(nt * 8 + g) * p.K + kc;
-      const uint32_t bh0 = ldg_u32(p.vt_hi + off), bh1 = ldg_u32(p.vt_hi + off + 8);
-      const uint32_t bl0 = ldg_u32(p.vt_lo + off), bl1 = ldg_u32(p.vt_lo + off + 8);
-      mma16816(u[nt], alo, bh0, bh1);
-      mma16816(u[nt], ahi, bl0, bl1);
-      mma16816(u[nt], ahi, bh0, bh1);
+  for (int i = 0; i < kChunk; i += 4) {
+    const float4 c = *reinterpret_cast<const float4*>(chan + i);
+    v[i] = __fmul_rn(v[i], c.x);
+    v[i + 1] = __fmul_rn(v[i + 1], c.y);
+    v[i + 2] = __fmul_rn(v[i + 2], c.z);
+    v[i + 3] = __fmul_rn(v[i + 3], c.w);
+  }
+#pragma unroll
+  for (int s = 0; s < 7; ++s) {
+    const int hh = 1 << s;
+    if (hh < b) {
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) {
+        if (!(i & hh)) {
+          const float a = v[i], c = v[i + hh];
+          v[i] = __fadd_rn(a, c);
+          v[i + hh] = __fsub_rn(a, c);
+        }
+      }
     }
   }
+#pragma unroll
+  for (int i = 0; i < kChunk; ++i) v[i] = __fmul_rn(v[i], hscale);
 }
 
-// Z = T~ - c V^T on one 128-column chunk, in place; returns the lane's max |Z|.
-template <int R>
-__device__ __forceinline__ float deflate(const PrologueParams& p, float* xt, int stride, int col, int lane,
-                                         const float (&u)[R / 8][4]) {
-  const int g = lane >> 2, q = lane & 3;
-  uint32_t ahi[R / 16][4], alo[R / 16][4];
-#pragma unroll
-  for (int ks = 0; ks < R / 16; ++ks) {
-    split_pair(u[2 * ks][0], u[2 * ks][1], ahi[ks][0], alo[ks][0]);
-    split_pair(u[2 * ks][2], u[2 * ks][3], ahi[ks][1], alo[ks][1]);
-    split_pair(u[2 * ks + 1][0], u[2 * ks + 1][1], ahi[ks][2], alo[ks][2]);
-    split_pair(u[2 * ks + 1][2], u[2 * ks + 1][3], ahi[ks][3], alo[ks][3]);
-  }
-  float amax = 0.0f;
-#pragma unroll 4
-  for (int nt = 0; nt < kChunk / 8; ++nt) {
-    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const size_t vrow = static_cast<size_t>(col + nt * 8 + g) * R;
-#pragma unroll
-    for (int ks = 0; ks < R / 16; ++ks) {
-      const size_t off = vrow + ks * 16 + 2 * q;
-      const uint32_t bh0 = ldg_u32(p.v_hi + off), bh1 = ldg_u32(p.v_hi + off + 8);
-      const uint32_t bl0 = ldg_u32(p.v_lo + off), bl1 = ldg_u32(p.v_lo + off + 8);
-      mma16816(d, alo[ks], bh0, bh1);
-      mma16816(d, ahi[ks], bl0, bl1);
-      mma16816(d, ahi[ks], bh0, bh1);
-    }
-    float* p0 = xt + g * stride + nt * 8 + 2 * q;
-    float* p1 = p0 + 8 * stride;
-    float2 x0 = *reinterpret_cast<float2*>(p0);
-    float2 x1 = *reinterpret_cast<float2*>(p1);
-    x0.x = __fsub_rn(x0.x, d[0]);
-    x0.y = __fsub_rn(x0.y, d[1]);
-    x1.x = __fsub_rn(x1.x, d[2]);
-    x1.y = __fsub_rn(x1.y, d[3]);
-    *reinterpret_cast<float2*>(p0) = x0;
-    *reinterpret_cast<float2*>(p1) = x1;
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x1.x), fabsf(x1.y))));
-  }
-  return amax;
+// Row t of a K-major bf16 operand tile with W-byte rows (one swizzle atom wide):
+// write 8 consecutive elements (16 bytes) as logical chunk j.
+__device__ __forceinline__ void put16(uint8_t* tile, int t, int j, int W, uint4 w) {
+  *reinterpret_cast<uint4*>(tile + t * W + (swz_chunk(t, j, W) << 4)) = w;
 }
 
-// Quantise the warp's 16 rows of one chunk (Z in shared memory): lane l takes
-// row l/2 and 64 columns (4 blocks); 32 code bytes and 4 scale bytes per lane.
-__device__ __forceinline__ void quantise_rows(const PrologueParams& p, const float* xt, int stride, int row0,
-                                              int col, float g, int lane) {
-  const int i = lane >> 1, half = lane & 1;
-  const int row = row0 + i;
-  if (row >= p.rows) return;
-  const float* src = xt + i * stride + half * 64;
-  const int c0 = col + half * 64;
-  uint32_t codes[8];
-  uint32_t sf4 = 0;
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
 #pragma unroll
-  for (int bb = 0; bb < 4; ++bb) {
-    float v[16];
+  for (int k = 0; k < 4; ++k) {
+    uint16_t h0, l0, h1, l1;
+    split_bf16(v[2 * k], h0, l0);
+    split_bf16(v[2 * k + 1], h1, l1);
+    h[k] = pack2(h0, h1);
+    l[k] = pack2(l0, l1);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Quantise this thread's 128 values of row `row`, columns [col, col+128).
+__device__ __forceinline__ void quantise_row(const PrologueParams& p, const float (&v)[kChunk], int row, int col,
+                                             float g) {
+  uint32_t cw[16];
+  uint32_t sfw[2] = {0u, 0u};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 t = *reinterpret_cast<const float4*>(src + bb * 16 + 4 * j);
-      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
-    }
+  for (int k = 0; k < 8; ++k) {
+    float blk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) blk[e] = v[16 * k + e];
     uint32_t c2[2];
-    const uint32_t S = quant_block16(v, g, c2);
-    codes[2 * bb] = c2[0];
-    codes[2 * bb + 1] = c2[1];
-    sf4 |= S << (8 * bb);
-    if (p.z_out) {
-      float4* z = reinterpret_cast<float4*>(p.z_out + static_cast<size_t>(row) * p.K + c0 + bb * 16);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) z[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-    }
+    const uint32_t S = quant_block16(blk, g, c2);
+    cw[2 * k] = c2[0];
+    cw[2 * k + 1] = c2[1];
+    sfw[k >> 2] |= S << (8 * (k & 3));
   }
-  uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + c0 / 2);
-  dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-  dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-  *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, c0 / 16, p.K)) = sf4;
+  uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + col / 2);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dst[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
+  *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, col / 16, p.K)) = sfw[0];
+  *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, col / 16 + 4, p.K)) = sfw[1];
+  if (p.z_out) {
+    float4* z = reinterpret_cast<float4*>(p.z_out + static_cast<size_t>(row) * p.K + col);
+#pragma unroll
+    for (int k = 0; k < kChunk / 4; ++k) z[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  }
 }
 
-// Branch operand and optional fp32 export of c for the warp's rows.
 template <int R>
-__device__ __forceinline__ void write_branch(const PrologueParams& p, int row0, const float (&u)[R / 8][4], float g,
-                                             int lane) {
-  const int g4 = lane >> 2, q = lane & 3;
-  const float gs = __fmul_rn(g, p.g_other);
+__device__ __forceinline__ void write_branch(const PrologueParams& p, const float (&u)[R > 0 ? R : 1], int row,
+                                             float g) {
+  if constexpr (R > 0) {
+    const float gs = __fmul_rn(g, p.g_other);
+    uint32_t w[R / 2];
 #pragma unroll
-  for (int nt = 0; nt < R / 8; ++nt) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = row0 + g4 + 8 * h;
-      if (row >= p.rows) continue;
-      float a = u[nt][2 * h], b = u[nt][2 * h + 1];
-      const size_t off = static_cast<size_t>(row) * R + nt * 8 + 2 * q;
-      if (p.u_out) *reinterpret_cast<float2*>(p.u_out + off) = make_float2(a, b);
+    for (int j = 0; j < R / 2; ++j) {
+      float a = u[2 * j], b = u[2 * j + 1];
       if (p.branch_mode == 1) {
         a = __fdiv_rn(a, gs);
         b = __fdiv_rn(b, gs);
       }
-      *reinterpret_cast<uint32_t*>(p.branch + off) = pack2(bf16_bits_rn(a), bf16_bits_rn(b));
+      w[j] = pack2(bf16_bits_rn(a), bf16_bits_rn(b));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.branch + static_cast<size_t>(row) * R);
+#pragma unroll
+    for (int j = 0; j < R / 8; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    if (p.u_out) {
+      float4* o = reinterpret_cast<float4*>(p.u_out + static_cast<size_t>(row) * R);
+#pragma unroll
+      for (int j = 0; j < R / 4; ++j) o[j] = make_float4(u[4 * j], u[4 * j + 1], u[4 * j + 2], u[4 * j + 3]);
     }
   }
-}
-
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 template <int R, int MODE>
-__global__ void __launch_bounds__(128) prologue_kernel(const PrologueParams p) {
-  extern __shared__ __align__(16) float smem[];
-  constexpr int NT = (R > 0 ? R / 8 : 1);
+__global__ void __launch_bounds__(kThreads, 1)
+    prologue_kernel(const __grid_constant__ ProMaps maps, const PrologueParams p) {
+  using C = PCfg<R, MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* xs_full = bars;      // [2] TMA landed
+  uint64_t* xs_free = bars + 2;  // [2] rows (and MMA) done with the slot
+  uint64_t* xt_full = bars + 4;  // rows wrote T~ for the next projection
+  uint64_t* xt_free = bars + 5;  // projection MMAs done with T~
+  uint64_t* u_full = bars + 6;   // all projection MMAs done
+  uint64_t* ua_full = bars + 7;  // rows wrote c hi/lo
+  uint64_t* d2_full = bars + 8;  // deflation MMAs done
+  uint64_t* d2_free = bars + 9;  // rows read the deflation result
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_MISC + 16);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g4 = lane >> 2, q = lane & 3;
   const int part = blockIdx.x;
-  const int row0 = blockIdx.y * kGroupRows + warp * 16;
-  const bool active = row0 < p.rows;
-  const int ncols = p.chunks * kChunk;
-  const int col_base = part * ncols;
-  const int stride = (MODE == 0 ? ncols : kChunk) + kPad;
-  float* xt_w = smem + warp * 16 * stride;
-  float* upart = smem + kGroupRows * stride;
-  float* red = upart + kGroupRows * (R > 0 ? R : 4);
+  const int m0 = blockIdx.y * kRows;
+  const int nch = p.chunks;
+  const int col0 = part * nch * kChunk;
 
-  float u[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.0f;
-
-  float g = 1.0f;
-  if constexpr (MODE == 2) {
-    g = global_scale_from_amax(__uint_as_float(*p.amax_glob));
-    if constexpr (R > 0) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int row = row0 + g4 + 8 * h;
-          if (row < p.rows) {
-            const float2 t = *reinterpret_cast<const float2*>(p.u_glob + static_cast<size_t>(row) * R + nt * 8 + 2 * q);
-            u[nt][2 * h] = t.x;
-            u[nt][2 * h + 1] = t.y;
-          }
-        }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&xs_full[i], 1);
+      mbar_init(&xs_free[i], kRows + (C::kMMA ? 1 : 0));
+    }
+    mbar_init(xt_full, kRows);
+    mbar_init(xt_free, 1);
+    mbar_init(u_full, 1);
+    mbar_init(ua_full, kRows);
+    mbar_init(d2_full, 1);
+    mbar_init(d2_free, kRows);
+    fence_barrier_init();
+  }
+  if constexpr (C::kMMA) {
+    if (warp == 5) {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
     }
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = C::kMMA ? *tmem_slot : 0u;
+  const uint32_t d2_tmem = tmem;
+  const uint32_t u_tmem = tmem + 128;
 
-  // Sweep 1 (Fused / Stats with r > 0): rotate and project every chunk, then
-  // sum the partial coordinates across the cluster in rank order.
-  if constexpr (MODE != 2 && R > 0) {
-    if (active) {
-      for (int c = 0; c < p.chunks; ++c) {
-        float* xc = xt_w + (MODE == 0 ? c * kChunk : 0);
-        rotate_rows(p, row0, col_base + c * kChunk, xc, stride, lane);
-        __syncwarp();
-        project<R>(p, xc, stride, col_base + c * kChunk, lane, u);
-        __syncwarp();
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------ producers
+    // A TMA instruction occupies its warp for a fixed ~600 cycles whatever its
+    // size: every slot has its own producer warp (4: even loads, 6: odd loads)
+    // and a slot's tiles (x, V^T or V) go out as one converged instruction.
+    const int my_slot = warp == 4 ? 0 : 1;
+    int i = 0, last = -1;
+    auto load = [&](int c, bool proj) {
+      const int slot = i & 1;
+      if (slot != my_slot) {
+        ++i;
+        return true;
       }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float* d0 = upart + (warp * 16 + g4) * R + nt * 8 + 2 * q;
-      *reinterpret_cast<float2*>(d0) = make_float2(u[nt][0], u[nt][1]);
-      *reinterpret_cast<float2*>(d0 + 8 * R) = make_float2(u[nt][2], u[nt][3]);
-    }
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const int nranks = static_cast<int>(cluster.num_blocks());
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.0f;
-    for (int rk = 0; rk < nranks; ++rk) {
-      const float* rp = cluster.map_shared_rank(upart, rk);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float* s0 = rp + (warp * 16 + g4) * R + nt * 8 + 2 * q;
-        const float2 a = *reinterpret_cast<const float2*>(s0);
-        const float2 b = *reinterpret_cast<const float2*>(s0 + 8 * R);
-        u[nt][0] = __fadd_rn(u[nt][0], a.x);
-        u[nt][1] = __fadd_rn(u[nt][1], a.y);
-        u[nt][2] = __fadd_rn(u[nt][2], b.x);
-        u[nt][3] = __fadd_rn(u[nt][3], b.y);
-      }
-    }
-    if constexpr (MODE == 1) cluster_arrive();  // remote reads of upart are done
-  }
-
-  // Sweep 2: deflate (recomputing T~ unless it is still resident), track amax,
-  // and in the Quantise launch quantise each chunk straight away.
-  float amax = 0.0f;
-  if (active) {
-    for (int c = 0; c < p.chunks; ++c) {
-      float* xc = xt_w + (MODE == 0 ? c * kChunk : 0);
-      const int col = col_base + c * kChunk;
-      float m;
-      if (MODE == 0 && R > 0) {
-        m = 0.0f;
-      } else {
-        m = rotate_rows(p, row0, col, xc, stride, lane);
-        __syncwarp();
-      }
-      if constexpr (R > 0) m = deflate<R>(p, xc, stride, col, lane, u);
-      amax = fmaxf(amax, m);
+      int ok = 1;
+      if (lane == 0 && i >= 2)
+        ok = mbar_wait(&xs_free[slot], ((i >> 1) & 1) ^ 1u, p.err, DEVERR_PRODUCER_WAIT) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      uint8_t* s = smem + slot * C::SLOT;
+      const int col = col0 + c * kChunk;
+      if (lane == 0) mbar_arrive_expect_tx(&xs_full[slot], C::X_BYTES + C::V_BYTES + C::CH_BYTES);
       __syncwarp();
-      if constexpr (MODE == 2) {
-        quantise_rows(p, xc, stride, row0, col, g, lane);
-        __syncwarp();
+      const CUtensorMap* m = nullptr;
+      uint8_t* dst = s;
+      int x = 0, y = 0;
+      if (lane < 2) {
+        m = &maps.x; dst = s + lane * 16384; x = col + 64 * lane; y = m0;
+      } else if (R > 0 && proj && lane < 6) {
+        const int pp = (lane - 2) >> 1, kb = (lane - 2) & 1;
+        m = pp ? &maps.vt_lo : &maps.vt_hi; dst = s + C::X_BYTES + (pp * 2 + kb) * R * 128; x = col + kb * 64; y = 0;
+      } else if (R > 0 && !proj && lane < 4) {
+        const int pp = lane - 2;
+        m = pp ? &maps.v_lo : &maps.v_hi; dst = s + C::X_BYTES + pp * 256 * R; x = 0; y = col;
+      }
+      if (m) tma_load_2d(dst, m, &xs_full[slot], x, y);
+      if (lane == 0) bulk_load(s + C::X_BYTES + C::V_BYTES, p.chan + col, C::CH_BYTES, &xs_full[slot]);
+      last = i;
+      ++i;
+      return true;
+    };
+    bool ok = true;
+    if (lane == 0 && warp == 4) {
+      tma_prefetch_desc(&maps.x);
+      if constexpr (R > 0) {
+        tma_prefetch_desc(&maps.vt_hi); tma_prefetch_desc(&maps.vt_lo);
+        tma_prefetch_desc(&maps.v_hi); tma_prefetch_desc(&maps.v_lo);
       }
     }
-  }
-
-  if constexpr (MODE == 2) {
-    if constexpr (R > 0)
-      if (part == 0) write_branch<R>(p, row0, u, g, lane);
-    if (part == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = g;
-    return;
-  } else {
-    const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
-    if (lane == 0) red[warp] = __uint_as_float(wmax);
-    __syncthreads();
-    if constexpr (MODE == 1) {
-      if (threadIdx.x == 0) {
-        const float cmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        atomicMax(p.amax_glob, __float_as_uint(cmax));
-      }
-      if constexpr (R > 0) {
-        if (part == 0 && active) {
+    __syncwarp();
+    if constexpr (C::kA) cluster_arrive();
+    if constexpr (C::kProj)
+      for (int c = 0; ok && c < nch; ++c) ok = load(c, true);
+    for (int c = 0; ok && c < nch; ++c) ok = load(c, false);
+    __syncwarp();
+    if constexpr (C::kA) cluster_wait();
+    if constexpr (C::kB) {
+      cluster_arrive();
+      for (int c = 0; ok && c < nch; ++c) ok = load(c, false);
+      __syncwarp();
+    }
+    if (lane == 0 && last >= 0) mbar_wait(&xs_full[last & 1], (last >> 1) & 1, p.err, DEVERR_DRAIN_WAIT);
+    __syncwarp();
+    if constexpr (C::kB) cluster_wait();
+    if constexpr (C::kC) {
+      cluster_arrive();
+      cluster_wait();
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if constexpr (C::kMMA) {
+      int i = 0, j = 0;
+      bool ok = true;
+      const uint32_t sbo_u = 8u * 2u * R;
+      const uint32_t swz_u = umma_swizzle_code(2 * R);
+      // deflation of one chunk: D2[128 x 128] = c (hi/lo) . V_chunk^T (hi/lo)
+      auto deflate_chunk = [&]() {
+        const int slot = i & 1;
+        if (!mbar_wait(&xs_full[slot], (i >> 1) & 1, p.err, DEVERR_MMA_WAIT)) return false;
+        if (!mbar_wait(d2_free, (j & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) return false;
+        tc_fence_after();
+        const uint32_t vs = smem_u32(smem + slot * C::SLOT + C::X_BYTES);
+        const uint32_t ua = smem_u32(smem + C::OFF_UA);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int row = row0 + g4 + 8 * h;
-              if (row < p.rows)
-                *reinterpret_cast<float2*>(p.u_glob + static_cast<size_t>(row) * R + nt * 8 + 2 * q) =
-                    make_float2(u[nt][2 * h], u[nt][2 * h + 1]);
-            }
+        for (int k = 0; k < R / 16; ++k) {
+          const uint64_t ah = smem_desc(ua + k * 32, 16, sbo_u, swz_u);
+          const uint64_t al = smem_desc(ua + 256 * R + k * 32, 16, sbo_u, swz_u);
+          const uint64_t bh = smem_desc(vs + k * 32, 16, sbo_u, swz_u);
+          const uint64_t bl = smem_desc(vs + 256 * R + k * 32, 16, sbo_u, swz_u);
+          mma_bf16(d2_tmem, al, bh, idesc_bf16(128, 128), k > 0 ? 1u : 0u);
+          mma_bf16(d2_tmem, ah, bl, idesc_bf16(128, 128), 1u);
+          mma_bf16(d2_tmem, ah, bh, idesc_bf16(128, 128), 1u);
         }
-        cluster_wait();  // no CTA leaves while a peer may still read its upart
+        tc_commit(d2_full);
+        tc_commit(&xs_free[slot]);
+        ++i;
+        ++j;
+        return true;
+      };
+      if constexpr (C::kProj) {
+        if (lane == 0) {
+          uint32_t acc = 0;
+          for (int c = 0; ok && c < nch; ++c) {
+            const int slot = i & 1;
+            ok = mbar_wait(&xs_full[slot], (i >> 1) & 1, p.err, DEVERR_MMA_WAIT) &&
+                 mbar_wait(xt_full, c & 1, p.err, DEVERR_MMA_WAIT);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t vs = smem_u32(smem + slot * C::SLOT + C::X_BYTES);
+            const uint32_t xt = smem_u32(smem + C::OFF_XT);
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ah = smem_desc(xt + kb * 16384 + k * 32, 16, 1024, 2);
+                const uint64_t al = smem_desc(xt + (2 + kb) * 16384 + k * 32, 16, 1024, 2);
+                const uint64_t bh = smem_desc(vs + kb * R * 128 + k * 32, 16, 1024, 2);
+                const uint64_t bl = smem_desc(vs + (2 + kb) * R * 128 + k * 32, 16, 1024, 2);
+                mma_bf16(u_tmem, al, bh, idesc_bf16(128, R), acc);
+                mma_bf16(u_tmem, ah, bl, idesc_bf16(128, R), 1u);
+                mma_bf16(u_tmem, ah, bh, idesc_bf16(128, R), 1u);
+                acc = 1u;
+              }
+            tc_commit(xt_free);
+            tc_commit(&xs_free[slot]);
+            ++i;
+          }
+          tc_commit(u_full);
+        }
+        __syncwarp();
+      }
+      if constexpr (C::kA) cluster_arrive();
+      if (lane == 0) {
+        ok = ok && mbar_wait(ua_full, 0, p.err, DEVERR_MMA_WAIT);
+        for (int c = 0; ok && c < nch; ++c) ok = deflate_chunk();
+      }
+      __syncwarp();
+      if constexpr (C::kA) cluster_wait();
+      if constexpr (C::kB) {
+        cluster_arrive();
+        if (lane == 0)
+          for (int c = 0; ok && c < nch; ++c) ok = deflate_chunk();
+        __syncwarp();
+        cluster_wait();
       }
     } else {
-      // Fused: the cluster holds every row, so its amax is the tensor amax.
-      cg::cluster_group cluster = cg::this_cluster();
-      if (threadIdx.x == 0) red[4] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      cluster.sync();
-      float A = 0.0f;
-      const int nranks = static_cast<int>(cluster.num_blocks());
-      for (int rk = 0; rk < nranks; ++rk) A = fmaxf(A, cluster.map_shared_rank(red, rk)[4]);
+      if constexpr (C::kB) cluster_sync_all();
+    }
+    if constexpr (C::kC) {
       cluster_arrive();
-      g = global_scale_from_amax(A);
-      if (active) {
-        for (int c = 0; c < p.chunks; ++c) quantise_rows(p, xt_w + c * kChunk, stride, row0, col_base + c * kChunk, g, lane);
-        if constexpr (R > 0)
-          if (part == 0) write_branch<R>(p, row0, u, g, lane);
+      cluster_wait();
+    }
+  } else {
+    // ------------------------------------------------------------ row threads
+    const int t = threadIdx.x;  // 0..127 = TMEM lane = row within the tile
+    const int row = m0 + t;
+    const bool valid = row < p.rows;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float v[kChunk];
+    float u[R > 0 ? R : 1];
+#pragma unroll
+    for (int k = 0; k < (R > 0 ? R : 1); ++k) u[k] = 0.0f;
+    int i = 0, j = 0;
+
+    if constexpr (C::kProj) {
+      for (int c = 0; c < nch; ++c) {
+        const int slot = i & 1;
+        mbar_wait(&xs_full[slot], (i >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
+        const uint8_t* s = smem + slot * C::SLOT;
+        rotate_row(s, reinterpret_cast<const float*>(s + C::X_BYTES + C::V_BYTES), t, p.b, p.hscale, v);
+        mbar_arrive(&xs_free[slot]);
+        mbar_wait(xt_free, (c & 1) ^ 1u, p.err, DEVERR_EPILOGUE_WAIT);
+        uint8_t* xt = smem + C::OFF_XT;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            uint4 hi, lo;
+            split8(v + kb * 64 + q * 8, hi, lo);
+            put16(xt + kb * 16384, t, q, 128, hi);
+            put16(xt + (2 + kb) * 16384, t, q, 128, lo);
+          }
+        fence_proxy_async();
+        mbar_arrive(xt_full);
+        ++i;
       }
-      if (part == 0 && threadIdx.x == 0) *p.g_out = g;
+      // c of this CTA's K range -> shared memory -> sum over the cluster
+      mbar_wait(u_full, 0, p.err, DEVERR_EPILOGUE_WAIT);
+      __syncwarp();
+      tc_fence_after();
+      {
+        uint32_t r32[32];
+        tmem_ld_32x32b_x32(u_tmem + lane_base, r32);
+        tmem_ld_wait();
+        float* up = reinterpret_cast<float*>(smem + C::OFF_XT) + t * C::UP_STRIDE;
+#pragma unroll
+        for (int k = 0; k < R; k += 4)
+          *reinterpret_cast<float4*>(up + k) = make_float4(__uint_as_float(r32[k]), __uint_as_float(r32[k + 1]),
+                                                           __uint_as_float(r32[k + 2]), __uint_as_float(r32[k + 3]));
+      }
+      cluster_arrive();
+      cluster_wait();
+      cg::cluster_group cluster = cg::this_cluster();
+      const int nranks = static_cast<int>(cluster.num_blocks());
+      for (int rk = 0; rk < nranks; ++rk) {
+        const float* rp = cluster.map_shared_rank(reinterpret_cast<float*>(smem + C::OFF_XT), rk) + t * C::UP_STRIDE;
+#pragma unroll
+        for (int k = 0; k < R; k += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(rp + k);
+          u[k] = __fadd_rn(u[k], a.x);
+          u[k + 1] = __fadd_rn(u[k + 1], a.y);
+          u[k + 2] = __fadd_rn(u[k + 2], a.z);
+          u[k + 3] = __fadd_rn(u[k + 3], a.w);
+        }
+      }
+      if (MODE == 1 && part == 0 && valid) {
+        float4* o = reinterpret_cast<float4*>(p.u_glob + static_cast<size_t>(row) * R);
+#pragma unroll
+        for (int k = 0; k < R / 4; ++k) o[k] = make_float4(u[4 * k], u[4 * k + 1], u[4 * k + 2], u[4 * k + 3]);
+      }
+    }
+    if constexpr (MODE == 2 && R > 0) {
+      if (valid) {
+        const float4* src = reinterpret_cast<const float4*>(p.u_glob + static_cast<size_t>(row) * R);
+#pragma unroll
+        for (int k = 0; k < R / 4; ++k) {
+          const float4 a = src[k];
+          u[4 * k] = a.x; u[4 * k + 1] = a.y; u[4 * k + 2] = a.z; u[4 * k + 3] = a.w;
+        }
+        if (part == 0) write_branch<R>(p, u, row, global_scale_from_amax(__uint_as_float(*p.amax_glob)));
+      }
+    }
+    if constexpr (MODE == 0 && R > 0) {
+      // park the cluster-summed c in the (now idle) T~ area until g is known
+      float* uf = reinterpret_cast<float*>(smem + C::OFF_XT + 32768) + t * C::UP_STRIDE;
+#pragma unroll
+      for (int k = 0; k < R; k += 4) *reinterpret_cast<float4*>(uf + k) = make_float4(u[k], u[k + 1], u[k + 2], u[k + 3]);
+    }
+    if constexpr (C::kMMA) {
+      uint8_t* ua = smem + C::OFF_UA;
+#pragma unroll
+      for (int q = 0; q < R / 8; ++q) {
+        uint4 hi, lo;
+        split8(u + q * 8, hi, lo);
+        put16(ua, t, q, 2 * R, hi);
+        put16(ua + 256 * R, t, q, 2 * R, lo);
+      }
+      fence_proxy_async();
+      mbar_arrive(ua_full);
+    }
+
+    // Z sweeps: Z = T~ - c V^T per chunk, then amax and / or quantisation.
+    auto z_chunk = [&](int c) {
+      const int slot = i & 1;
+      mbar_wait(&xs_full[slot], (i >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      const uint8_t* s = smem + slot * C::SLOT;
+      rotate_row(s, reinterpret_cast<const float*>(s + C::X_BYTES + C::V_BYTES), t, p.b, p.hscale, v);
+      mbar_arrive(&xs_free[slot]);
+      if constexpr (C::kMMA) {
+        mbar_wait(d2_full, j & 1, p.err, DEVERR_EPILOGUE_WAIT);
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t r32[32];
+          tmem_ld_32x32b_x32(d2_tmem + lane_base + q * 32, r32);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[q * 32 + k] = __fsub_rn(v[q * 32 + k], __uint_as_float(r32[k]));
+        }
+        tc_fence_before();
+        mbar_arrive(d2_free);
+        ++j;
+      }
+      ++i;
+    };
+    float g = 1.0f;
+    if constexpr (MODE == 2) g = global_scale_from_amax(__uint_as_float(*p.amax_glob));
+    float amax = 0.0f;
+    for (int c = 0; c < nch; ++c) {
+      z_chunk(c);
+      if constexpr (MODE == 2) {
+        if (valid) quantise_row(p, v, row, col0 + c * kChunk, g);
+      } else {
+#pragma unroll
+        for (int k = 0; k < kChunk; ++k) amax = fmaxf(amax, fabsf(v[k]));
+      }
+    }
+    if constexpr (MODE != 2) {
+      const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+      if (lane == 0) red[warp] = __uint_as_float(wmax);
+      named_bar(1, kRows);
+      const float cmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      if constexpr (MODE == 1) {
+        if (t == 0) atomicMax(p.amax_glob, __float_as_uint(cmax));
+      } else {
+        if (t == 0) red[4] = cmax;
+      }
+    }
+    if constexpr (MODE == 0) {
+      // red[4] is published by the cluster barrier B.
+      cluster_arrive();
+      cluster_wait();
+      cg::cluster_group cluster = cg::this_cluster();
+      const int nranks = static_cast<int>(cluster.num_blocks());
+      float A = 0.0f;
+      for (int rk = 0; rk < nranks; ++rk) A = fmaxf(A, cluster.map_shared_rank(red, rk)[4]);
+      g = global_scale_from_amax(A);
+      if constexpr (R > 0) {
+        if (part == 0 && valid) {
+          const float* uf = reinterpret_cast<const float*>(smem + C::OFF_XT + 32768) + t * C::UP_STRIDE;
+#pragma unroll
+          for (int k = 0; k < R; ++k) u[k] = uf[k];
+          write_branch<R>(p, u, row, g);
+        }
+      }
+      if (part == 0 && t == 0 && blockIdx.y == 0) *p.g_out = g;
+      for (int c = 0; c < nch; ++c) {
+        z_chunk(c);
+        if (valid) quantise_row(p, v, row, col0 + c * kChunk, g);
+      }
+    }
+    if constexpr (MODE == 2) {
+      if (part == 0 && t == 0 && blockIdx.y == 0) *p.g_out = g;
+    }
+    if constexpr (C::kC) {
+      cluster_arrive();
       cluster_wait();
     }
   }
-}
-
-// --- standalone quantiser (tests and tools) -------------------------------
-__global__ void amax_kernel(const float* __restrict__ T, size_t n, uint32_t* amax) {
-  float m = 0.0f;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    m = fmaxf(m, fabsf(T[i]));
-  const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
-  if ((threadIdx.x & 31) == 0) atomicMax(amax, w);
-}
-
-__global__ void quantize_blocks_kernel(const float* __restrict__ T, int rows, int K, uint8_t* codes, uint8_t* sf,
-                                       const uint32_t* amax, float* g_out) {
-  const size_t nblk = static_cast<size_t>(rows) * (K / 16);
-  const float g = global_scale_from_amax(__uint_as_float(*amax));
-  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-  for (size_t bi = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; bi < nblk;
-       bi += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int row = static_cast<int>(bi / (K / 16));
-    const int kb = static_cast<int>(bi % (K / 16));
-    float v[16];
-    const float4* src = reinterpret_cast<const float4*>(T + static_cast<size_t>(row) * K + kb * 16);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 t = src[j];
-      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (C::kMMA) {
+    if (warp == 5) {
+      __syncwarp();
+      tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    uint32_t c2[2];
-    const uint32_t S = quant_block16(v, g, c2);
-    *reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2) + kb * 8) = make_uint2(c2[0], c2[1]);
-    sf[sf_offset(row, kb, K)] = static_cast<uint8_t>(S);
   }
-}
-
-// --- prepare helpers -------------------------------------------------------
-__global__ void recip_kernel(const float* __restrict__ s, float* __restrict__ inv_s, int K, uint32_t* err) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= K) return;
-  const float v = s[i];
-  if (!(v > 0.0f) || !isfinite(v)) atomicOr(err, 1u);
-  inv_s[i] = __frcp_rn(v);
-}
-
-__global__ void split_v_kernel(const float* __restrict__ V, int K, int r, uint16_t* v_hi, uint16_t* v_lo,
-                               uint16_t* vt_hi, uint16_t* vt_lo) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= K * r) return;
-  const int k = i / r, j = i % r;
-  uint16_t hi, lo;
-  split_bf16(V[i], hi, lo);
-  v_hi[i] = hi;
-  v_lo[i] = lo;
-  vt_hi[static_cast<size_t>(j) * K + k] = hi;
-  vt_lo[static_cast<size_t>(j) * K + k] = lo;
 }
 
 template <int R, int MODE>
-cudaError_t launch_one(const PrologueParams& p, int cluster, cudaStream_t st) {
-  const int groups = (p.rows + kGroupRows - 1) / kGroupRows;
-  const int parts = p.K / kChunk / p.chunks;
-  const size_t smem = prologue_smem_bytes(R, static_cast<PrologueMode>(MODE), p.chunks);
+cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p, int parts, cudaStream_t st) {
+  using C = PCfg<R, MODE>;
   auto kern = prologue_kernel<R, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  static const cudaError_t smem_attr =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (smem_attr != cudaSuccess) return smem_attr;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(parts, groups, 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(parts, (p.rows + kRows - 1) / kRows, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  int nattr = 0;
-  if (MODE != 2) {
+  cfg.numAttrs = 0;
+  if (C::kC) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.x = parts;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    nattr = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
   }
-  cfg.attrs = attr;
-  cfg.numAttrs = nattr;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, maps, p);
 }
 
 template <int MODE>
-cudaError_t launch_mode(const PrologueParams& p, int r, int cluster, cudaStream_t st) {
+cudaError_t launch_mode(const ProMaps& maps, const PrologueParams& p, int r, int parts, cudaStream_t st) {
   switch (r) {
-    case 0: return launch_one<0, MODE>(p, cluster, st);
-    case 16: return launch_one<16, MODE>(p, cluster, st);
-    case 32: return launch_one<32, MODE>(p, cluster, st);
+    case 0: return launch_one<0, MODE>(maps, p, parts, st);
+    case 16: return launch_one<16, MODE>(maps, p, parts, st);
+    case 32: return launch_one<32, MODE>(maps, p, parts, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-size_t prologue_smem_bytes(int r, PrologueMode mode, int chunks) {
-  const int ncols = (mode == PrologueMode::Fused ? chunks * kChunk : kChunk);
-  return static_cast<size_t>(kGroupRows) * (ncols + kPad) * 4 + static_cast<size_t>(kGroupRows) * (r > 0 ? r : 4) * 4 +
-         64;
-}
-
-cudaError_t launch_prologue(const PrologueParams& p, int r, PrologueMode mode, int cluster, cudaStream_t st) {
+cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode, int parts,
+                            cudaStream_t st) {
   switch (mode) {
-    case PrologueMode::Fused: return launch_mode<0>(p, r, cluster, st);
-    case PrologueMode::Stats: return launch_mode<1>(p, r, cluster, st);
-    case PrologueMode::Quantise: return launch_mode<2>(p, r, cluster, st);
+    case PrologueMode::Fused: return launch_mode<0>(maps, p, r, parts, st);
+    case PrologueMode::Stats: return launch_mode<1>(maps, p, r, parts, st);
+    case PrologueMode::Quantise: return launch_mode<2>(maps, p, r, parts, st);
   }
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st) {
-  recip_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, uint16_t* vt_hi,
-                           uint16_t* vt_lo, cudaStream_t st) {
-  const int n = K * r;
-  split_v_kernel<<<(n + 255) / 256, 256, 0, st>>>(V, K, r, v_hi, v_lo, vt_hi, vt_lo);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_quantize_fp32(const float* T, int rows, int K, uint8_t* codes, uint8_t* sf, float* g_out,
-                                 uint32_t* amax_scratch, cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(amax_scratch, 0, sizeof(uint32_t), st);
-  if (e != cudaSuccess) return e;
-  const size_t n = static_cast<size_t>(rows) * K;
-  const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 8));
-  amax_kernel<<<blocks, 256, 0, st>>>(T, n, amax_scratch);
-  const size_t nblk = static_cast<size_t>(rows) * (K / 16);
-  const int qblocks = static_cast<int>(std::min<size_t>((nblk + 255) / 256, 148 * 8));
-  quantize_blocks_kernel<<<qblocks, 256, 0, st>>>(T, rows, K, codes, sf, amax_scratch, g_out);
-  return cudaGetLastError();
 }
 
 }  // namespace qwam

@@ -143,6 +143,12 @@ qwam_status qwam_quantize_fp32(const float* T, int rows, int K, void* codes, voi
 qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales,
                           int M, int N, int K, float alpha, float* out_f32, void* stream);
 
+/* How qwam_linear runs for M rows of this layer (host outputs, each may be
+ * NULL): kernels = kernel launches per call, fused = 1 when the prologue is the
+ * single-launch (cluster-wide amax) form, splits = K splits of the GEMM,
+ * bn = GEMM tile width. */
+qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* splits, int* bn);
+
 /* Synchronise the current device, then return (and clear) the device error
  * word set by bounded waits: *code == 0 means none expired.  Returns
  * QWAM_ERR_TIMEOUT when *code != 0. */
