@@ -237,6 +237,23 @@ def per_unit(value_units, seconds, unit):
     return value_units / seconds / 1e12
 
 
+def replica_instance_seed(rank, i):
+    """Layer-instance index of instance i on a replica rank: every rank draws
+    its own weights and activations (no two ranks share an instance)."""
+    return rank * 100003 + i
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's
+    time).  dist is torch.distributed when the job has more than one rank."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_reference(args, wl, shape):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -333,7 +350,7 @@ def main():
     P = args.instances or max(1, min(256, math.ceil(1.5 * L2_BYTES / per_inst)))
     handles, xs, ys = [], [], []
     for i in range(P):
-        c = probe if i == 0 and rank == 0 else wl["make"](rank * 100003 + i, args.seed)
+        c = probe if i == 0 and rank == 0 else wl["make"](replica_instance_seed(rank, i), args.seed)
         x = torch.from_numpy(c.x).to(dev).to(torch.bfloat16)
         W = torch.from_numpy(c.W).to(dev).to(torch.bfloat16)
         s = torch.from_numpy(c.s).to(dev)
@@ -444,10 +461,7 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = t.tolist()
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist if world > 1 else None, dev)
 
     unit = wl["unit"]
     lb, lf = layer_bytes(M, K, N, r), layer_flops(M, K, N, r)
