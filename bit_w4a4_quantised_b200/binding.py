@@ -21,6 +21,7 @@ SIGNATURES = {
     "qwam_prepare_weight": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, ctypes.POINTER(_P)]),
     "qwam_destroy": (_I, [_P]),
     "qwam_linear": (_I, [_P, _I, _P, _P, _P]),
+    "qwam_linear_noalloc": (_I, [_P, _I, _P, _P, _P]),
     "qwam_prologue": (_I, [_P, _I, _P, _P]),
     "qwam_gemm": (_I, [_I, _P, _P, _P]),
     "qwam_handle_info": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
@@ -165,6 +166,18 @@ def linear(x, h: Handle, y=None, stream=None):
         y = torch.empty((M, h.N), dtype=torch.bfloat16, device=x.device)
     _need(y, torch.bfloat16, (M, h.N), "y")
     _check(load().qwam_linear(_ptr(x), M, h.raw, _ptr(y), _stream(stream)))
+    return y
+
+
+def linear_noalloc(x, h: Handle, y, stream=None):
+    """qwam_linear_noalloc: the layer with all scratch in the library's fixed
+    static array (M <= 128, K <= 16384).  y (bf16 [M, N]) must be given, so the
+    call itself allocates nothing."""
+    import torch
+    M = x.shape[0]
+    _need(x, torch.bfloat16, (M, h.K), "x")
+    _need(y, torch.bfloat16, (M, h.N), "y")
+    _check(load().qwam_linear_noalloc(_ptr(x), M, h.raw, _ptr(y), _stream(stream)))
     return y
 
 

@@ -456,6 +456,125 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
 
 }  // namespace
 
+// ---- allocation-free variant of the layer call -----------------------------
+// Some callers must not allocate device memory once they are running: a
+// fixed-rate control loop (a cudaMalloc can synchronise the whole device and
+// stall for milliseconds) and processes whose device memory is budgeted at
+// start-up.  qwam_linear_noalloc serves them from this fixed scratch area,
+// compiled into the library, instead of the growable per-device workspace.
+// It holds the same layout as that workspace (scalars and tile tickets, then
+// activation codes, scales, u, u' and split-K partials) for up to 128 rows
+// and K <= 16384; for such calls the layout needs at most 11 MB.
+constexpr int kStaticMaxRows = 128;
+constexpr int kStaticMaxK = 16384;
+constexpr size_t kStaticBytes = size_t(12) << 20;
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticBytes];
+
+namespace {
+
+std::mutex g_static_mu;
+uint8_t* g_static_base[kMaxDevices];  // this device's address of g_static_scratch, once set up
+
+// Set-up, once per device, with that device current: look up the device
+// address of the scratch and clear its header (activation amax, g_x, the
+// error word and the split-K tile tickets must start at zero; the GEMM's last
+// split puts each ticket back to zero, so later calls find them cleared).
+qwam_status static_scratch(int dev, uint8_t** out) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_base[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();
+      return fail(QWAM_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    }
+    QW_CUDA(cudaMemset(p, 0, kHeaderBytes));
+    QW_CUDA(cudaDeviceSynchronize());
+    g_static_base[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_static_base[dev];
+  return QWAM_OK;
+}
+
+// The same two launches as qwam_linear (fused prologue, then the GEMM with
+// the same plan), with every workspace pointer inside the static scratch.
+qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cudaStream_t st) {
+  if (M > kStaticMaxRows)
+    return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes at most %d rows, got M=%d", kStaticMaxRows, M);
+  if (h->K > kStaticMaxK)
+    return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes K <= %d, this layer has K=%d", kStaticMaxK, h->K);
+  const Plan pl = plan_gemm(M, h->N, h->K);
+  const Layout lay = layout_for(M, h->K, h->N, h->r, pl.splits);
+  if (lay.total > kStaticBytes)
+    return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc needs %zu bytes of scratch, the static scratch holds %zu",
+                lay.total, kStaticBytes);
+  const int tiles = ((M + 127) / 128) * ((h->N + pl.bn - 1) / pl.bn);
+  if (pl.splits > 1 && tiles > kMaxTiles) return fail(QWAM_ERR_SHAPE, "too many output tiles for split-K");
+  uint8_t* base = nullptr;
+  QW_TRY(static_scratch(h->dev, &base));
+  uint32_t* amax = reinterpret_cast<uint32_t*>(base);
+  float* g_x = reinterpret_cast<float*>(base + 4);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base + 8);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(base + 256);
+
+  PrologueParams prm{};
+  prm.chan = h->inv_s;
+  prm.rows = M;
+  prm.K = h->K;
+  prm.b = h->b;
+  prm.hscale = 1.0f / std::sqrt(static_cast<float>(h->b));
+  prm.u_glob = reinterpret_cast<float*>(base + lay.u);
+  prm.codes = base + lay.codes;
+  prm.sf = base + lay.sf;
+  prm.branch = reinterpret_cast<uint16_t*>(base + lay.ub);
+  prm.branch_mode = 1;
+  prm.g_other = h->g_w;
+  prm.g_out = g_x;
+  prm.err = err;
+  QW_TRY(run_rows(x, prm, h->r, h->vmaps, true, amax, st));
+
+  GemmMaps maps{};
+  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, base + lay.codes, h->K / 2, M, h->K / 2, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_64B));
+  maps.b = pl.bn == 256 ? h->map_b256 : h->map_b128;
+  QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K));
+  maps.sfb = h->map_sfb;
+  if (h->r > 0) {
+    QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base + lay.ub, h->r, M, h->r * 2, h->r, 128,
+                    branch_swizzle(h->r)));
+    maps.l = pl.bn == 256 ? h->map_l256 : h->map_l128;
+  } else {
+    maps.u = maps.a;
+    maps.l = maps.b;
+  }
+  if (pl.splits == 1)
+    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B));
+  else
+    maps.y = maps.a;
+  GemmParams p{};
+  p.M = M; p.N = h->N; p.K = h->K;
+  p.k_stages = pl.k_stages;
+  p.stages_per_split = pl.stages_per_split;
+  p.splits = pl.splits;
+  p.sfa = base + lay.sf;
+  p.sfb = h->sf;
+  p.g_a_ptr = g_x;
+  p.g_b = h->g_w;
+  p.has_branch = h->r > 0;
+  p.branch_k = h->r;
+  p.bias = h->bias;
+  p.y = y;
+  p.partial = reinterpret_cast<float*>(base + lay.partial);
+  p.counters = counters;
+  p.err = err;
+  QW_CUDA(launch_gemm(maps, p, pl.bn, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
+  return QWAM_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 qwam_status qwam_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
@@ -503,6 +622,15 @@ qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, 
   if (y_bf16 == x_bf16) return fail(QWAM_ERR_INVALID_ARG, "y must not alias x");
   QW_TRY(prologue_impl(x_bf16, M, h, nullptr, nullptr, as_stream(stream), nullptr, nullptr));
   return gemm_impl(M, h, y_bf16, as_stream(stream));
+}
+
+qwam_status qwam_linear_noalloc(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream) {
+  QW_TRY(check_linear_args(x_bf16, M, h));
+  if (M == 0) return QWAM_OK;
+  if (!y_bf16) return fail(QWAM_ERR_INVALID_ARG, "y is NULL");
+  if (!aligned16(y_bf16)) return fail(QWAM_ERR_ALIGN, "y must be 16-byte aligned");
+  if (y_bf16 == x_bf16) return fail(QWAM_ERR_INVALID_ARG, "y must not alias x");
+  return linear_noalloc_impl(x_bf16, M, h, y_bf16, as_stream(stream));
 }
 
 qwam_status qwam_handle_info(qwam_handle h, int* N, int* K, int* r, int* b, float* g_w) {
@@ -615,11 +743,25 @@ qwam_status qwam_device_error(uint32_t* code) {
   QW_CUDA(cudaGetDevice(&dev));
   QW_CUDA(cudaDeviceSynchronize());
   if (dev < 0 || dev >= kMaxDevices) return QWAM_OK;
+  uint8_t* sbase = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    sbase = g_static_base[dev];
+  }
+  if (sbase) {  // the error word of qwam_linear_noalloc's static scratch
+    uint32_t c = 0;
+    QW_CUDA(cudaMemcpy(&c, sbase + 8, 4, cudaMemcpyDeviceToHost));
+    QW_CUDA(cudaMemset(sbase + 8, 0, 4));
+    *code |= c;
+  }
   std::lock_guard<std::mutex> lock(g_arena_mu);
   const Arena& a = g_arena[dev];
-  if (!a.base) return QWAM_OK;
-  QW_CUDA(cudaMemcpy(code, arena_err(a), 4, cudaMemcpyDeviceToHost));
-  QW_CUDA(cudaMemset(arena_err(a), 0, 4));
+  if (a.base) {
+    uint32_t c = 0;
+    QW_CUDA(cudaMemcpy(&c, arena_err(a), 4, cudaMemcpyDeviceToHost));
+    QW_CUDA(cudaMemset(arena_err(a), 0, 4));
+    *code |= c;
+  }
   if (*code) return fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired (flags 0x%x)", *code);
   return QWAM_OK;
 }
