@@ -177,10 +177,14 @@ qwam_status arena_get(int dev, size_t need, Arena** out) {
   return QWAM_OK;
 }
 
-int cluster_parts(int K) {
+// CTAs along K per 128-row tile of the prologue: the largest divisor of the
+// chunk count (K / 128) that is at most 8 (one portable cluster) and keeps the
+// grid within one wave of the SMs (at least one part).
+int cluster_parts(int K, int rows) {
   const int chunks = K / 128;
+  const int tiles = (rows + 127) / 128;
   for (int c = std::min(8, chunks); c >= 1; --c)
-    if (chunks % c == 0) return c;
+    if (chunks % c == 0 && (c == 1 || tiles * c <= kSMs)) return c;
   return 1;
 }
 
@@ -192,20 +196,21 @@ struct qwam_layer {
   uint8_t* codes;
   uint8_t* sf;
   uint16_t* L;
-  uint16_t *v_hi, *v_lo, *vt_hi, *vt_lo;
+  uint16_t *v_hi, *v_lo;    // V [K, r] bf16 hi/lo
+  uint16_t *px_hi, *px_lo;  // P^T = (diag(1/s) H V)^T [r, K] bf16 hi/lo
   float* inv_s;
   uint16_t* bias;
   float g_w;
   size_t sf_bytes;
   CUtensorMap map_b128, map_b256, map_l128, map_l256, map_sfb;
-  ProMaps vmaps;  // V^T and V (hi/lo) tensor maps for the prologue; x is per call
+  ProMaps vmaps;  // P^T and V (hi/lo) tensor maps for the prologue; x is per call
 };
 
 namespace {
 
 void free_layer(qwam_layer* h) {
   if (!h) return;
-  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->vt_hi, h->vt_lo, h->inv_s, h->bias};
+  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->px_hi, h->px_lo, h->inv_s, h->bias};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   h->magic = 0;
@@ -247,20 +252,20 @@ bool use_fused(int rows) { return rows <= 128; }
 qwam_status run_rows(const void* T, PrologueParams prm, int r, const ProMaps& vmaps, bool allow_fused,
                      uint32_t* amax, cudaStream_t st) {
   const int K = prm.K;
-  const int parts = cluster_parts(K);
   ProMaps maps = vmaps;
   QW_TRY(make_map(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, K, prm.rows, static_cast<uint64_t>(K) * 2, 64, 128,
                   CU_TENSOR_MAP_SWIZZLE_128B));
-  if (r == 0) maps.vt_hi = maps.vt_lo = maps.v_hi = maps.v_lo = maps.x;
-  prm.chunks = K / 128 / parts;
+  if (r == 0) maps.p_hi = maps.p_lo = maps.v_hi = maps.v_lo = maps.x;
   prm.amax_glob = amax;
+  prm.parts = cluster_parts(K, prm.rows);
+  prm.chunks = K / 128 / prm.parts;
   if (allow_fused && use_fused(prm.rows)) {
-    QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Fused, parts, st));
+    QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Fused, st));
     return QWAM_OK;
   }
   QW_CUDA(cudaMemsetAsync(amax, 0, sizeof(uint32_t), st));
-  QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Stats, parts, st));
-  QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Quantise, parts, st));
+  QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Stats, st));
+  QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Quantise, st));
   return QWAM_OK;
 }
 
@@ -285,9 +290,12 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   h->sf_bytes = round_up(static_cast<size_t>(N), 256) * K / 16;
   float* u_tmp = nullptr;
   uint32_t* scratch = nullptr;  // [0] amax, [1] err, [2] g_w (fp32)
+  uint16_t *pw_hi = nullptr, *pw_lo = nullptr;  // P^T of the weight side, diag(s) H V
   auto cleanup = [&](qwam_status s) {
     if (u_tmp) cudaFree(u_tmp);
     if (scratch) cudaFree(scratch);
+    if (pw_hi) cudaFree(pw_hi);
+    if (pw_lo) cudaFree(pw_lo);
     free_layer(h);
     return s;
   };
@@ -296,7 +304,8 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   if ((s_ = dmalloc(&h->codes, static_cast<size_t>(N) * K / 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->sf, h->sf_bytes)) != QWAM_OK || (s_ = dmalloc(&h->L, static_cast<size_t>(N) * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->v_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->v_lo, K * rr * 2)) != QWAM_OK ||
-      (s_ = dmalloc(&h->vt_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->vt_lo, K * rr * 2)) != QWAM_OK ||
+      (s_ = dmalloc(&h->px_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->px_lo, K * rr * 2)) != QWAM_OK ||
+      (s_ = dmalloc(&pw_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&pw_lo, K * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->inv_s, static_cast<size_t>(K) * 4)) != QWAM_OK ||
       (s_ = dmalloc(&u_tmp, static_cast<size_t>(N) * rr * 4)) != QWAM_OK || (s_ = dmalloc(&scratch, 64)) != QWAM_OK)
     return cleanup(s_);
@@ -312,18 +321,23 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   QW_CUDA_CLEAN(cudaMemsetAsync(scratch, 0, 64, st));
   if (bias) QW_CUDA_CLEAN(cudaMemcpyAsync(h->bias, bias, static_cast<size_t>(N) * 2, cudaMemcpyDeviceToDevice, st));
   QW_CUDA_CLEAN(launch_recip(s, h->inv_s, K, scratch + 1, st));
-  if (r > 0) QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, h->vt_hi, h->vt_lo, st));
-
+  ProMaps wmaps{};  // the weight pass uses P of the weight side
   if (r > 0) {
-    if ((s_ = make_map(&h->vmaps.vt_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->vt_hi, K, r, static_cast<uint64_t>(K) * 2,
-                       64, r, CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK ||
-        (s_ = make_map(&h->vmaps.vt_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->vt_lo, K, r, static_cast<uint64_t>(K) * 2,
-                       64, r, CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK ||
+    QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, st));
+    QW_CUDA_CLEAN(launch_make_proj(V, s, K, r, b, pw_hi, pw_lo, st));
+    QW_CUDA_CLEAN(launch_make_proj(V, h->inv_s, K, r, b, h->px_hi, h->px_lo, st));
+    auto pmap = [&](CUtensorMap* m, const uint16_t* base) {
+      return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, K, r, static_cast<uint64_t>(K) * 2, 64, r,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    };
+    if ((s_ = pmap(&h->vmaps.p_hi, h->px_hi)) != QWAM_OK || (s_ = pmap(&h->vmaps.p_lo, h->px_lo)) != QWAM_OK ||
         (s_ = make_map(&h->vmaps.v_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_hi, r, K, r * 2, r, 128,
                        branch_swizzle(r))) != QWAM_OK ||
         (s_ = make_map(&h->vmaps.v_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_lo, r, K, r * 2, r, 128,
                        branch_swizzle(r))) != QWAM_OK)
       return cleanup(s_);
+    wmaps = h->vmaps;
+    if ((s_ = pmap(&wmaps.p_hi, pw_hi)) != QWAM_OK || (s_ = pmap(&wmaps.p_lo, pw_lo)) != QWAM_OK) return cleanup(s_);
   }
   PrologueParams prm{};
   prm.chan = s;
@@ -340,7 +354,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   prm.g_out = reinterpret_cast<float*>(scratch + 2);
   prm.z_out = wd_out;
   prm.err = scratch + 3;
-  if ((s_ = run_rows(W, prm, r, h->vmaps, false, scratch, st)) != QWAM_OK) return cleanup(s_);
+  if ((s_ = run_rows(W, prm, r, wmaps, false, scratch, st)) != QWAM_OK) return cleanup(s_);
   uint32_t host_scr[4] = {0, 0, 0, 0};
   QW_CUDA_CLEAN(cudaMemcpyAsync(host_scr, scratch, 16, cudaMemcpyDeviceToHost, st));
   QW_CUDA_CLEAN(cudaStreamSynchronize(st));
@@ -366,6 +380,8 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   }
   cudaFree(u_tmp);
   cudaFree(scratch);
+  cudaFree(pw_hi);
+  cudaFree(pw_lo);
 #undef QW_CUDA_CLEAN
   *out = h;
   return QWAM_OK;

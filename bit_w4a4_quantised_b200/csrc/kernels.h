@@ -9,14 +9,15 @@
 namespace qwam {
 
 // One "rows" job of the activation prologue / weight prepare:
-//   T~ = (T * chan) H,  c = T~ V,  Z = T~ - c V^T,  quantise(Z),
+//   T~ = (T * chan) H,  c = T~ V = T P,  Z = T~ - c V^T,  quantise(Z),
 // with T = x, chan = 1/s on the activation side and T = W, chan = s on the
-// weight side.  T and V reach the kernel through TMA tensor maps.
+// weight side, and P = diag(chan) H V precomputed once per layer.  T, P and V
+// reach the kernel through TMA tensor maps.
 struct ProMaps {
-  CUtensorMap x;      // T bf16 [rows, K], box 64 x 128 rows, 128B swizzle
-  CUtensorMap vt_hi;  // V^T bf16 [r, K], box 64 x r, 128B swizzle
-  CUtensorMap vt_lo;
-  CUtensorMap v_hi;   // V bf16 [K, r], box r x 128 rows, 2r-byte swizzle
+  CUtensorMap x;     // T bf16 [rows, K], box 64 x 128 rows, 128B swizzle
+  CUtensorMap p_hi;  // P^T bf16 [r, K] (hi/lo split of fp32 P), box 64 x r, 128B swizzle
+  CUtensorMap p_lo;
+  CUtensorMap v_hi;  // V bf16 [K, r] (hi/lo split), box r x 128 rows, 2r-byte swizzle
   CUtensorMap v_lo;
 };
 
@@ -26,6 +27,7 @@ struct PrologueParams {
   int K;
   int b;                  // Hadamard block (power of two, <= 128)
   int chunks;             // 128-column chunks per CTA
+  int parts;              // CTAs along K per row tile (one cluster when they exchange)
   float hscale;           // fp32(1 / sqrt(b))
   float* u_glob;          // fp32 [rows, r]: written by Stats, read by Quantise
   uint32_t* amax_glob;    // fp32 bits of max|Z|: atomicMax'd by Stats
@@ -45,12 +47,14 @@ enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2 };
 // Grid: parts x ceil(rows / 128) CTAs; Fused and Stats (r > 0) launch the
 // parts of a row tile as one cluster.  Fused requires rows <= 128; Stats
 // requires *amax_glob == 0.
-cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode, int parts,
+cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode,
                             cudaStream_t st);
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st);
-cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, uint16_t* vt_hi,
-                           uint16_t* vt_lo, cudaStream_t st);
+cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, cudaStream_t st);
+// P^T = (diag(chan) H V)^T split into bf16 hi/lo, [r, K] each; H block size b.
+cudaError_t launch_make_proj(const float* V, const float* chan, int K, int r, int b, uint16_t* p_hi, uint16_t* p_lo,
+                             cudaStream_t st);
 cudaError_t launch_quantize_fp32(const float* T, int rows, int K, uint8_t* codes, uint8_t* sf, float* g_out,
                                  uint32_t* amax_scratch, cudaStream_t st);
 

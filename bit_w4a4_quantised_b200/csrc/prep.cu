@@ -1,7 +1,9 @@
 // Kernels outside the per-call hot path: the standalone NVFP4 quantiser (used by
 // tests and tools on arbitrary fp32 tensors) and the prepare-time helpers that
-// derive 1/s and the bf16 hi/lo split of V stored in a layer handle.
+// derive 1/s, the bf16 hi/lo split of V and the projection matrix
+// P = diag(chan) H V stored in a layer handle.
 #include <algorithm>
+#include <cmath>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -52,17 +54,38 @@ __global__ void recip_kernel(const float* __restrict__ s, float* __restrict__ in
   inv_s[i] = __frcp_rn(v);
 }
 
-__global__ void split_v_kernel(const float* __restrict__ V, int K, int r, uint16_t* v_hi, uint16_t* v_lo,
-                               uint16_t* vt_hi, uint16_t* vt_lo) {
+__global__ void split_v_kernel(const float* __restrict__ V, int K, int r, uint16_t* v_hi, uint16_t* v_lo) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= K * r) return;
-  const int k = i / r, j = i % r;
   uint16_t hi, lo;
   split_bf16(V[i], hi, lo);
   v_hi[i] = hi;
   v_lo[i] = lo;
-  vt_hi[static_cast<size_t>(j) * K + k] = hi;
-  vt_lo[static_cast<size_t>(j) * K + k] = lo;
+}
+
+// x~ V = ((x * chan) H) V = x (diag(chan) H V): the rank-r coordinates come
+// straight from T with P = diag(chan) H V.  One CTA = 128 consecutive k of one
+// column j: Sylvester FWHT of V[:, j] inside each b-block (butterflies
+// (lo + hi, lo - hi)), times 1/sqrt(b), times chan[k], split to bf16 hi/lo and
+// stored transposed ([r, K], K contiguous: the K-major B operand of the MMA).
+__global__ void make_proj_kernel(const float* __restrict__ V, const float* __restrict__ chan, int K, int r, int b,
+                                 float hscale, uint16_t* p_hi, uint16_t* p_lo) {
+  __shared__ float buf[128];
+  const int t = threadIdx.x, j = blockIdx.y;
+  const int k = blockIdx.x * 128 + t;
+  buf[t] = V[static_cast<size_t>(k) * r + j];
+  __syncthreads();
+  for (int h = 1; h < b; h <<= 1) {
+    const float a = buf[t], c = buf[t ^ h];
+    __syncthreads();
+    buf[t] = (t & h) ? __fsub_rn(c, a) : __fadd_rn(a, c);
+    __syncthreads();
+  }
+  const float v = __fmul_rn(__fmul_rn(buf[t], hscale), chan[k]);
+  uint16_t hi, lo;
+  split_bf16(v, hi, lo);
+  p_hi[static_cast<size_t>(j) * K + k] = hi;
+  p_lo[static_cast<size_t>(j) * K + k] = lo;
 }
 
 }  // namespace
@@ -72,10 +95,17 @@ cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cud
   return cudaGetLastError();
 }
 
-cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, uint16_t* vt_hi,
-                           uint16_t* vt_lo, cudaStream_t st) {
+cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, cudaStream_t st) {
   const int n = K * r;
-  split_v_kernel<<<(n + 255) / 256, 256, 0, st>>>(V, K, r, v_hi, v_lo, vt_hi, vt_lo);
+  split_v_kernel<<<(n + 255) / 256, 256, 0, st>>>(V, K, r, v_hi, v_lo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_make_proj(const float* V, const float* chan, int K, int r, int b, uint16_t* p_hi, uint16_t* p_lo,
+                             cudaStream_t st) {
+  if (K % 128 || b < 1 || b > 128 || (b & (b - 1)) || r < 1) return cudaErrorInvalidValue;
+  const float hscale = 1.0f / std::sqrt(static_cast<float>(b));
+  make_proj_kernel<<<dim3(K / 128, r), 128, 0, st>>>(V, chan, K, r, b, hscale, p_hi, p_lo);
   return cudaGetLastError();
 }
 
