@@ -177,14 +177,14 @@ qwam_status arena_get(int dev, size_t need, Arena** out) {
   return QWAM_OK;
 }
 
-// CTAs along K per 128-row tile of the prologue: the largest divisor of the
-// chunk count (K / 128) that is at most 8 (one portable cluster) and keeps the
-// grid within one wave of the SMs (at least one part).
+// CTAs along K per 128-row tile of the prologue: the largest power of two
+// that divides the chunk count (K / 128), is at most 8 (one portable cluster)
+// and keeps the grid within one wave of the SMs (at least one part).
 int cluster_parts(int K, int rows) {
   const int chunks = K / 128;
   const int tiles = (rows + 127) / 128;
-  for (int c = std::min(8, chunks); c >= 1; --c)
-    if (chunks % c == 0 && (c == 1 || tiles * c <= kSMs)) return c;
+  for (int c = 8; c > 1; c >>= 1)
+    if (chunks % c == 0 && tiles * c <= kSMs) return c;
   return 1;
 }
 

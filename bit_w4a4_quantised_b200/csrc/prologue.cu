@@ -67,7 +67,7 @@ struct PCfg {
   static constexpr bool kSmall = W == 32;
   static constexpr int UC = R > 0 ? R / 2 : 1;        // c columns per row thread (two per row)
   static constexpr int X_BYTES = kRows * kChunk * 2;  // two 64-column SW128 boxes
-  static constexpr int P_BYTES = 512 * R;             // P^T hi/lo: 4 boxes of R rows x 128 B
+  static constexpr int P_BYTES = 512 * R;             // P^T: [kb][hi, lo] boxes of R rows x 128 B
   static constexpr int V_BYTES = 512 * R;             // V hi/lo: 2 boxes of 128 rows x 2R B
   static constexpr int CH_BYTES = kChunk * 4;
   static constexpr int OFF_P = X_BYTES;
@@ -76,13 +76,18 @@ struct PCfg {
   static constexpr int SLOT = (OFF_CH + CH_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_UA = 2 * SLOT;             // c hi/lo: A operand of the deflation
   static constexpr int UA_BYTES = 512 * R;
-  static constexpr int UP_STRIDE = R + 4;             // fp32 partial c rows, read by the cluster
-  static constexpr int OFF_UP = OFF_UA + UA_BYTES;
-  static constexpr int UP_BYTES = kProj ? kRows * UP_STRIDE * 4 : 0;
-  static constexpr int OFF_BAR = OFF_UP + UP_BYTES;
-  static constexpr int OFF_RED = OFF_BAR + 128;       // warp maxima [8], CTA max at [8]
-  static constexpr int SMEM = OFF_RED + 64 + 1024;
-  static constexpr uint32_t TMEM_COLS = 256;          // D2 [0, 128), c [128, 128 + R)
+  // Cluster sum of c, reduce-scatter then all-gather, both pushed with remote
+  // stores: RS[rank][row in slice][R] receives the partials of this CTA's row
+  // slice from every rank; UG[row][R + 4] receives the summed rows.
+  static constexpr int OFF_RS = OFF_UA + UA_BYTES;
+  static constexpr int RS_BYTES = kProj ? kRows * R * 4 : 0;
+  static constexpr int UG_STRIDE = R + 4;
+  static constexpr int OFF_UG = OFF_RS + RS_BYTES;
+  static constexpr int UG_BYTES = kProj ? kRows * UG_STRIDE * 4 : 0;
+  static constexpr int OFF_BAR = OFF_UG + UG_BYTES;
+  static constexpr int OFF_RED = OFF_BAR + 128;       // warp maxima [0, 8), CTA maxima by rank [8, 16)
+  static constexpr int SMEM = OFF_RED + 128 + 1024;
+  static constexpr uint32_t TMEM_COLS = 256;          // D2 [0, 128), T P^T hi | lo [128, 128 + 2R)
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(!kSmall || MODE == 0, "the small layout is a Fused-only form");
 };
@@ -311,6 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C::kMMA ? *tmem_slot : 0u;
+  // Cluster barriers, in order: A0 (every CTA of the cluster is running, so its
+  // shared memory may take remote stores), A1 / A2 (partial c scattered / summed
+  // c gathered), B (CTA amax published; Fused), C (no more remote access: exit).
+  if constexpr (C::kCluster) cluster_arrive();  // A0
   const uint32_t d2_tmem = tmem;
   const uint32_t u_tmem = tmem + 128;
 
@@ -324,7 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&maps.v_hi); tma_prefetch_desc(&maps.v_lo);
       }
     }
-    if constexpr (C::kNeedA) cluster_arrive();
     int last = -1;
     bool ok = true;
     auto issue = [&](int i) {
@@ -350,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = &maps.x; dst = s + lane * 16384; x = col + 64 * lane; y = m0;
       } else if (R > 0 && lane < 6 && (kind & LD_P)) {
         const int pp = (lane - 2) >> 1, kb = (lane - 2) & 1;
-        m = pp ? &maps.p_lo : &maps.p_hi; dst = s + C::OFF_P + (pp * 2 + kb) * R * 128; x = col + kb * 64; y = 0;
+        m = pp ? &maps.p_lo : &maps.p_hi; dst = s + C::OFF_P + (kb * 2 + pp) * R * 128; x = col + kb * 64; y = 0;
       } else if (R > 0 && lane >= 6 && lane < 8 && (kind & LD_V)) {
         const int pp = lane - 6;
         m = pp ? &maps.v_lo : &maps.v_hi; dst = s + C::OFF_V + pp * 256 * R; x = 0; y = col;
@@ -359,19 +367,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && (kind & LD_CH)) bulk_load(s + C::OFF_CH, p.chan + col, C::CH_BYTES, &full[slot]);
       last = i;
     };
-    // loads before the amax exchange, then (Fused, several chunks) the second sweep
-    const int first_part = sch.total - (sch.zsweeps == 2 ? nch : 0);
-    for (int i = 0; i < first_part; ++i) issue(i);
-    __syncwarp();
-    if constexpr (C::kNeedA) cluster_wait();
-    if constexpr (C::kNeedB) cluster_arrive();
-    for (int i = first_part; i < sch.total; ++i) issue(i);
+    // The producers pass each cluster barrier before any load whose ring slot
+    // the rows free only after that barrier (a slot is reused two loads later),
+    // so no wait here depends on a barrier this warp has not reached.
+    const int zs1 = sch.nproj, zs2 = sch.nproj + nch;
+    bool didA = !C::kNeedA, didB = !C::kNeedB;
+    auto pass_a = [&]() {
+      if (!didA) {
+        __syncwarp();
+        cluster_wait();    // A0
+        cluster_arrive();  // A1
+        cluster_wait();
+        cluster_arrive();  // A2
+        didA = true;
+      }
+    };
+    auto pass_b = [&]() {
+      if (!didB) {
+        pass_a();
+        __syncwarp();
+        cluster_wait();    // A2, or A0 without the exchange of c
+        cluster_arrive();  // B
+        didB = true;
+      }
+    };
+    for (int i = 0; i < sch.total; ++i) {
+      if (i == zs1 + 2) pass_a();
+      if (sch.zsweeps == 2 && i == zs2 + 2) pass_b();
+      issue(i);
+    }
+    pass_a();
+    pass_b();
     __syncwarp();
     if (lane == 0 && last >= 0) mbar_wait(&full[last & 1], (last >> 1) & 1, p.err, DEVERR_DRAIN_WAIT);
     __syncwarp();
-    if constexpr (C::kNeedB) cluster_wait();
     if constexpr (C::kCluster) {
-      cluster_arrive();
+      cluster_wait();  // the last barrier arrived at (B, else A2)
+      cluster_arrive();  // C
       cluster_wait();
     }
   } else if (warp == kMmaWarp) {
@@ -389,15 +421,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t xs = smem_u32(smem + slot * C::SLOT);
             const uint32_t ps = xs + C::OFF_P;
+            // B = [P^T hi; P^T lo] (2R rows): columns [0, R) of the result
+            // accumulate T P_hi, columns [R, 2R) accumulate T P_lo
 #pragma unroll
             for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const uint64_t a = smem_desc(xs + kb * 16384 + k * 32, 16, 1024, 2);
-                const uint64_t bh = smem_desc(ps + kb * R * 128 + k * 32, 16, 1024, 2);
-                const uint64_t bl = smem_desc(ps + (2 + kb) * R * 128 + k * 32, 16, 1024, 2);
-                mma_bf16(u_tmem, a, bl, idesc_bf16(128, R), acc);
-                mma_bf16(u_tmem, a, bh, idesc_bf16(128, R), 1u);
+                const uint64_t b = smem_desc(ps + kb * 2 * R * 128 + k * 32, 16, 1024, 2);
+                mma_bf16(u_tmem, a, b, idesc_bf16(128, 2 * R), acc);
                 acc = 1u;
               }
             if (!sch.merged) {
@@ -409,7 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      if constexpr (C::kNeedA) cluster_arrive();
+      if constexpr (C::kNeedA) {
+        cluster_wait();    // A0
+        cluster_arrive();  // A1
+        cluster_wait();
+        cluster_arrive();  // A2
+      }
       // deflation of one chunk: D2[128 x 128] = c (hi/lo) . V_chunk^T (hi/lo)
       const uint32_t sbo_u = 8u * 2u * R;
       const uint32_t swz_u = umma_swizzle_code(2 * R);
@@ -441,22 +478,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; ok && c < nch; ++c) ok = deflate();
       }
       __syncwarp();
-      if constexpr (C::kNeedA) cluster_wait();
-      if constexpr (C::kNeedB) cluster_arrive();
+      if constexpr (C::kNeedB) {
+        cluster_wait();    // A2
+        cluster_arrive();  // B
+      }
       if (sch.zsweeps == 2) {
         if (lane == 0)
           for (int c = 0; ok && c < nch; ++c) ok = deflate();
         __syncwarp();
       }
-      if constexpr (C::kNeedB) cluster_wait();
     } else {
       if constexpr (C::kNeedB) {
-        cluster_arrive();
-        cluster_wait();
+        cluster_wait();    // A0
+        cluster_arrive();  // B
       }
     }
     if constexpr (C::kCluster) {
-      cluster_arrive();
+      cluster_wait();    // the last barrier arrived at (B, else A2)
+      cluster_arrive();  // C
       cluster_wait();
     }
   } else {
@@ -490,59 +529,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if constexpr (C::kProj) {
-      // partial c of this CTA's K range: TMEM -> shared memory -> cluster sum
+      // Partial c of this CTA's K range (T P_hi + T P_lo, from TMEM), summed
+      // over the cluster: reduce-scatter by row slice, then all-gather, both by
+      // remote stores (remote loads would cost a round trip each).
       mbar_wait(u_full, 0, p.err, DEVERR_EPILOGUE_WAIT);
       __syncwarp();
       tc_fence_after();
-      float* up = reinterpret_cast<float*>(smem + C::OFF_UP) + urow * C::UP_STRIDE + uc0;
+      const int SL = (C::kSmall ? 32 : kRows) / p.parts;  // rows per owner
+      const uint32_t my_rank = cluster_rank();
+      float* rs = reinterpret_cast<float*>(smem + C::OFF_RS);
+      float* ug = reinterpret_cast<float*>(smem + C::OFF_UG);
+      cluster_wait();  // A0
       if (uact) {
+        float pu[C::UC];
         if constexpr (C::UC == 16) {
-          uint32_t r16[16];
-          tmem_ld_32x32b_x16(u_tmem + lane_base + uc0, r16);
+          uint32_t a16[16], b16[16];
+          tmem_ld_32x32b_x16(u_tmem + lane_base + uc0, a16);
+          tmem_ld_32x32b_x16(u_tmem + lane_base + R + uc0, b16);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 16; k += 4)
-            *reinterpret_cast<float4*>(up + k) = make_float4(__uint_as_float(r16[k]), __uint_as_float(r16[k + 1]),
-                                                             __uint_as_float(r16[k + 2]), __uint_as_float(r16[k + 3]));
+          for (int k = 0; k < 16; ++k) pu[k] = __fadd_rn(__uint_as_float(a16[k]), __uint_as_float(b16[k]));
         } else {
-          uint32_t r8[8];
-          tmem_ld_32x32b_x8(u_tmem + lane_base + uc0, r8);
+          uint32_t a8[8], b8[8];
+          tmem_ld_32x32b_x8(u_tmem + lane_base + uc0, a8);
+          tmem_ld_32x32b_x8(u_tmem + lane_base + R + uc0, b8);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 8; k += 4)
-            *reinterpret_cast<float4*>(up + k) = make_float4(__uint_as_float(r8[k]), __uint_as_float(r8[k + 1]),
-                                                             __uint_as_float(r8[k + 2]), __uint_as_float(r8[k + 3]));
+          for (int k = 0; k < 8; ++k) pu[k] = __fadd_rn(__uint_as_float(a8[k]), __uint_as_float(b8[k]));
         }
+        const uint32_t dst = dsmem_addr(smem_u32(rs + (static_cast<int>(my_rank) * SL + urow % SL) * R + uc0),
+                                        static_cast<uint32_t>(urow / SL));
+#pragma unroll
+        for (int k = 0; k < C::UC / 4; ++k)
+          dsmem_st_f4(dst + 16u * k, make_float4(pu[4 * k], pu[4 * k + 1], pu[4 * k + 2], pu[4 * k + 3]));
       }
-      cluster_arrive();
+      cluster_arrive();  // A1
+      cluster_wait();
+      for (int it = threadIdx.x; it < SL * (R / 4); it += kRowThreads) {
+        const int srow = it / (R / 4), c4 = it % (R / 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int rk = 0; rk < p.parts; ++rk) {  // rank order: deterministic
+          const float4 v = *reinterpret_cast<const float4*>(rs + (rk * SL + srow) * R + 4 * c4);
+          acc.x = __fadd_rn(acc.x, v.x);
+          acc.y = __fadd_rn(acc.y, v.y);
+          acc.z = __fadd_rn(acc.z, v.z);
+          acc.w = __fadd_rn(acc.w, v.w);
+        }
+        const uint32_t src = smem_u32(ug + (static_cast<int>(my_rank) * SL + srow) * C::UG_STRIDE + 4 * c4);
+        for (int rk = 0; rk < p.parts; ++rk) dsmem_st_f4(dsmem_addr(src, static_cast<uint32_t>(rk)), acc);
+      }
+      cluster_arrive();  // A2
       cluster_wait();
       if (uact) {
-        // every load is issued before the sums, which run in rank order
-        const uint32_t my = smem_u32(up);
+        const float* g = ug + urow * C::UG_STRIDE + uc0;
 #pragma unroll
-        for (int h2 = 0; h2 < C::UC / 4; h2 += 2) {
-          float4 vals[kMaxParts][2];
-#pragma unroll
-          for (int rk = 0; rk < kMaxParts; ++rk) {
-            if (rk < p.parts) {
-              const uint32_t a = dsmem_addr(my, static_cast<uint32_t>(rk));
-              vals[rk][0] = dsmem_ld_f4(a + 16u * h2);
-              vals[rk][1] = dsmem_ld_f4(a + 16u * (h2 + 1));
-            }
-          }
-#pragma unroll
-          for (int rk = 0; rk < kMaxParts; ++rk) {
-            if (rk < p.parts) {
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                float* d = u + 4 * (h2 + e);
-                d[0] = __fadd_rn(d[0], vals[rk][e].x);
-                d[1] = __fadd_rn(d[1], vals[rk][e].y);
-                d[2] = __fadd_rn(d[2], vals[rk][e].z);
-                d[3] = __fadd_rn(d[3], vals[rk][e].w);
-              }
-            }
-          }
+        for (int k = 0; k < C::UC; k += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(g + k);
+          u[k] = v.x; u[k + 1] = v.y; u[k + 2] = v.z; u[k + 3] = v.w;
         }
       }
       if (MODE == 1 && part == 0 && uvalid) {
@@ -628,29 +671,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < W; ++k) amax = fmaxf(amax, fabsf(z[k]));
       }
     }
+    if constexpr (MODE == 0 && !C::kNeedA) cluster_wait();  // A0, before the remote stores below
     if constexpr (MODE != 2) {
       const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
       if (lane == 0) red[warp] = __uint_as_float(wmax);
       named_bar(1, kRowThreads);
-      if (threadIdx.x == 0) {
+      if (threadIdx.x < 32) {
         float cmax = red[0];
 #pragma unroll
         for (int w = 1; w < kRowWarps; ++w) cmax = fmaxf(cmax, red[w]);
-        if constexpr (MODE == 1)
-          atomicMax(p.amax_glob, __float_as_uint(cmax));
-        else
-          red[kRowWarps] = cmax;
+        if constexpr (MODE == 1) {
+          if (threadIdx.x == 0) atomicMax(p.amax_glob, __float_as_uint(cmax));
+        } else if (threadIdx.x < p.parts) {
+          // push this CTA's maximum into slot [8 + rank] of every rank
+          const uint32_t slot = smem_u32(red + kRowWarps + cluster_rank());
+          dsmem_st_f32(dsmem_addr(slot, static_cast<uint32_t>(threadIdx.x)), cmax);
+        }
       }
     }
     if constexpr (MODE == 0) {
-      // red[8] of every CTA is published by cluster barrier B
-      cluster_arrive();
+      cluster_arrive();  // B
       cluster_wait();
-      const uint32_t my = smem_u32(red + kRowWarps);
       float A = 0.0f;
-#pragma unroll
-      for (int rk = 0; rk < kMaxParts; ++rk)
-        if (rk < p.parts) A = fmaxf(A, dsmem_ld_f32(dsmem_addr(my, static_cast<uint32_t>(rk))));
+      for (int rk = 0; rk < p.parts; ++rk) A = fmaxf(A, red[kRowWarps + rk]);
       g = global_scale_from_amax(A);
       if constexpr (R > 0) {
         if (part == 0 && uvalid) write_branch<C::UC>(p, u, R, urow_g, uc0, g);
@@ -690,7 +733,7 @@ cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p, cudaStream_
   static const cudaError_t smem_attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (smem_attr != cudaSuccess) return smem_attr;
-  if (p.parts < 1 || p.parts > kMaxParts) return cudaErrorInvalidValue;
+  if (p.parts < 1 || p.parts > kMaxParts || (p.parts & (p.parts - 1))) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.parts, (p.rows + kRows - 1) / kRows, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
