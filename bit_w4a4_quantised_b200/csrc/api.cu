@@ -20,8 +20,7 @@ namespace {
 
 constexpr uint32_t kMagic = 0x514d5731u;
 constexpr int kMaxDevices = 64;
-constexpr size_t kHeaderBytes = 256 + 65536;  // scalars, then split-K tile tickets
-constexpr int kMaxTiles = 16384;
+constexpr size_t kHeaderBytes = 256;  // scalars: activation amax, g_x, device error word
 constexpr int kSMs = 148;
 
 thread_local std::string g_err;
@@ -101,19 +100,24 @@ CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZL
 
 // ---- GEMM launch plan ------------------------------------------------------
 struct Plan {
-  int bn, k_stages, splits, stages_per_split;
+  int bn, k_stages, splits;
 };
 
+// Split-K when the output tiles leave SMs idle: the largest power of two <= 8
+// (one portable cluster per tile) with splits <= K / 128 and tiles * splits
+// within one wave of the SMs.
 Plan plan_gemm(int M, int N, int K) {
   Plan p{};
   p.k_stages = (K + 127) / 128;
   const int tiles_m = (M + 127) / 128;
   p.bn = (M <= 128 || N < 256) ? 128 : 256;
   const int tiles = tiles_m * ((N + p.bn - 1) / p.bn);
-  int splits = 1;
-  if (tiles < kSMs) splits = std::min(p.k_stages, std::max(1, kSMs / tiles));
-  p.stages_per_split = (p.k_stages + splits - 1) / splits;
-  p.splits = (p.k_stages + p.stages_per_split - 1) / p.stages_per_split;
+  p.splits = 1;
+  for (int c = 8; c >= 2; c >>= 1)
+    if (c <= p.k_stages && tiles * c <= kSMs) {
+      p.splits = c;
+      break;
+    }
   return p;
 }
 
@@ -126,10 +130,10 @@ std::mutex g_arena_mu;
 Arena g_arena[kMaxDevices];
 
 struct Layout {
-  size_t codes, sf, u, ub, partial, total;
+  size_t codes, sf, u, ub, total;
 };
 
-Layout layout_for(int M, int K, int N, int r, int splits) {
+Layout layout_for(int M, int K, int r) {
   Layout L{};
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
@@ -143,7 +147,6 @@ Layout layout_for(int M, int K, int N, int r, int splits) {
   L.sf = take(Mp * K / 16);
   L.u = take(static_cast<size_t>(M) * rr * 4);
   L.ub = take(Mp * rr * 2);
-  L.partial = take(splits > 1 ? static_cast<size_t>(splits) * M * N * 4 : 0);
   L.total = off;
   return L;
 }
@@ -151,7 +154,6 @@ Layout layout_for(int M, int K, int N, int r, int splits) {
 uint32_t* arena_amax(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base); }
 float* arena_gx(const Arena& a) { return reinterpret_cast<float*>(a.base + 4); }
 uint32_t* arena_err(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base + 8); }
-uint32_t* arena_counters(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base + 256); }
 
 qwam_status arena_get(int dev, size_t need, Arena** out) {
   std::lock_guard<std::mutex> lock(g_arena_mu);
@@ -399,7 +401,7 @@ qwam_status check_linear_args(const void* x, int M, qwam_handle h) {
 qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, float* u_out, cudaStream_t st,
                           Arena** arena_out, Layout* lay_out) {
   const Plan pl = plan_gemm(M, h->N, h->K);
-  const Layout lay = layout_for(M, h->K, h->N, h->r, pl.splits);
+  const Layout lay = layout_for(M, h->K, h->r);
   Arena* a = nullptr;
   QW_TRY(arena_get(h->dev, lay.total, &a));
   PrologueParams prm{};
@@ -426,11 +428,9 @@ qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, flo
 
 qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   const Plan pl = plan_gemm(M, h->N, h->K);
-  const Layout lay = layout_for(M, h->K, h->N, h->r, pl.splits);
+  const Layout lay = layout_for(M, h->K, h->r);
   Arena* a = nullptr;
   QW_TRY(arena_get(h->dev, lay.total, &a));
-  const int tiles = ((M + 127) / 128) * ((h->N + pl.bn - 1) / pl.bn);
-  if (pl.splits > 1 && tiles > kMaxTiles) return fail(QWAM_ERR_SHAPE, "too many output tiles for split-K");
   GemmMaps maps{};
   QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->base + lay.codes, h->K / 2, M, h->K / 2, 64, 128,
                   CU_TENSOR_MAP_SWIZZLE_64B));
@@ -453,7 +453,6 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   GemmParams p{};
   p.M = M; p.N = h->N; p.K = h->K;
   p.k_stages = pl.k_stages;
-  p.stages_per_split = pl.stages_per_split;
   p.splits = pl.splits;
   p.sfa = a->base + lay.sf;
   p.sfb = h->sf;
@@ -463,8 +462,6 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   p.branch_k = h->r;
   p.bias = h->bias;
   p.y = y;
-  p.partial = reinterpret_cast<float*>(a->base + lay.partial);
-  p.counters = arena_counters(*a);
   p.err = arena_err(*a);
   QW_CUDA(launch_gemm(maps, p, pl.bn, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
   return QWAM_OK;
@@ -478,12 +475,12 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
 // stall for milliseconds) and processes whose device memory is budgeted at
 // start-up.  qwam_linear_noalloc serves them from this fixed scratch area,
 // compiled into the library, instead of the growable per-device workspace.
-// It holds the same layout as that workspace (scalars and tile tickets, then
-// activation codes, scales, u, u' and split-K partials) for up to 128 rows
-// and K <= 16384; for such calls the layout needs at most 11 MB.
+// It holds the same layout as that workspace (scalars, then activation codes,
+// scales, u and u') for up to 128 rows and K <= 16384; for such calls the
+// layout needs at most 1.2 MB.
 constexpr int kStaticMaxRows = 128;
 constexpr int kStaticMaxK = 16384;
-constexpr size_t kStaticBytes = size_t(12) << 20;
+constexpr size_t kStaticBytes = size_t(2) << 20;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticBytes];
 
@@ -493,9 +490,8 @@ std::mutex g_static_mu;
 uint8_t* g_static_base[kMaxDevices];  // this device's address of g_static_scratch, once set up
 
 // Set-up, once per device, with that device current: look up the device
-// address of the scratch and clear its header (activation amax, g_x, the
-// error word and the split-K tile tickets must start at zero; the GEMM's last
-// split puts each ticket back to zero, so later calls find them cleared).
+// address of the scratch and clear its header (the device error word must
+// start at zero; the other scalars are written before they are read).
 qwam_status static_scratch(int dev, uint8_t** out) {
   std::lock_guard<std::mutex> lock(g_static_mu);
   if (!g_static_base[dev]) {
@@ -521,18 +517,15 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   if (h->K > kStaticMaxK)
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes K <= %d, this layer has K=%d", kStaticMaxK, h->K);
   const Plan pl = plan_gemm(M, h->N, h->K);
-  const Layout lay = layout_for(M, h->K, h->N, h->r, pl.splits);
+  const Layout lay = layout_for(M, h->K, h->r);
   if (lay.total > kStaticBytes)
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc needs %zu bytes of scratch, the static scratch holds %zu",
                 lay.total, kStaticBytes);
-  const int tiles = ((M + 127) / 128) * ((h->N + pl.bn - 1) / pl.bn);
-  if (pl.splits > 1 && tiles > kMaxTiles) return fail(QWAM_ERR_SHAPE, "too many output tiles for split-K");
   uint8_t* base = nullptr;
   QW_TRY(static_scratch(h->dev, &base));
   uint32_t* amax = reinterpret_cast<uint32_t*>(base);
   float* g_x = reinterpret_cast<float*>(base + 4);
   uint32_t* err = reinterpret_cast<uint32_t*>(base + 8);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(base + 256);
 
   PrologueParams prm{};
   prm.chan = h->inv_s;
@@ -572,7 +565,6 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   GemmParams p{};
   p.M = M; p.N = h->N; p.K = h->K;
   p.k_stages = pl.k_stages;
-  p.stages_per_split = pl.stages_per_split;
   p.splits = pl.splits;
   p.sfa = base + lay.sf;
   p.sfb = h->sf;
@@ -582,8 +574,6 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   p.branch_k = h->r;
   p.bias = h->bias;
   p.y = y;
-  p.partial = reinterpret_cast<float*>(base + lay.partial);
-  p.counters = counters;
   p.err = err;
   QW_CUDA(launch_gemm(maps, p, pl.bn, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
   return QWAM_OK;
@@ -726,7 +716,6 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   GemmParams p{};
   p.M = M; p.N = N; p.K = K;
   p.k_stages = (K + 127) / 128;
-  p.stages_per_split = p.k_stages;
   p.splits = 1;
   p.sfa = static_cast<const uint8_t*>(a_scales);
   p.sfb = static_cast<const uint8_t*>(b_scales);
@@ -734,7 +723,6 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   p.g_a = alpha;
   p.g_b = 1.0f;
   p.out_f32 = out_f32;
-  p.counters = arena_counters(*a);
   p.err = arena_err(*a);
   QW_CUDA(launch_gemm(maps, p, bn, GemmEpilogue::RawF32, as_stream(stream)));
   return QWAM_OK;

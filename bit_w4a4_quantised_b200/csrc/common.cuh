@@ -59,6 +59,35 @@ __device__ __forceinline__ uint32_t pack2(uint16_t lo_col, uint16_t hi_col) {
   return static_cast<uint32_t>(lo_col) | (static_cast<uint32_t>(hi_col) << 16);
 }
 
+// Packed pairs of fp32 (sm_100 f32x2): each lane of the pair is one correctly
+// rounded fp32 operation, bit-identical to the scalar __fadd_rn / __fsub_rn /
+// __fmul_rn, at twice the rate per instruction.
+__device__ __forceinline__ uint64_t f2_bits(float2 v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_from(uint64_t b) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(b));
+  return v;
+}
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
@@ -142,6 +171,15 @@ __device__ __forceinline__ void bulk_wait() {
 }
 // Generic-proxy shared-memory writes -> visible to TMA / tensor-core reads.
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream still runs;
+// griddep_wait() blocks until that kernel has completed and its memory writes
+// are visible.  griddep_launch_dependents() lets the next such kernel start.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 // Barrier over the first `count` threads of the CTA (id 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -28,9 +28,12 @@
 //                   accumulator to registers, release it to the next tile, add
 //                   bias, round to bf16, stage through 128B-swizzled smem and
 //                   store with TMA (ragged M / N are clipped by the tensor map).
-// Split-K (small M): fp32 partials; the last split of a tile (atomic ticket)
-// sums them in split order and writes y.  Every mbarrier wait is bounded.  No
-// TMA multicast.
+// Split-K (small M): the splits of an output tile form one cluster (split
+// fastest in the grid, one work item per CTA).  Once every split's MMAs are
+// done, each pushes its fp32 accumulator rows to the CTA that owns them (a
+// 128 / splits row slice) through distributed shared memory, into the owner's
+// now idle operand ring; the owner sums the splits in order and writes y.
+// Every mbarrier wait is bounded.  No TMA multicast.
 #include <algorithm>
 
 #include "common.cuh"
@@ -77,9 +80,9 @@ struct Cfg {
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(kBM * BN * 4 <= STAGES * (A_BYTES + B_BYTES), "split-K receive area fits in the operand ring");
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return pack2(bf16_bits_rn(a), bf16_bits_rn(b));
@@ -89,11 +92,12 @@ struct TileCoord {
   int m0, n0, split;
 };
 
-// Tiles run M-fastest so consecutive CTAs reuse the same weight tile from L2.
-__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bn) {
-  const int mt = t % tiles_m;
-  const int rest = t / tiles_m;
-  return {mt * kBM, (rest % tiles_n) * bn, rest / tiles_n};
+// Tiles run M-fastest so consecutive CTAs reuse the same weight tile from L2;
+// with split-K the split index is fastest (a tile's splits are one cluster).
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bn, int splits) {
+  const int sp = t % splits;
+  const int rest = t / splits;
+  return {(rest % tiles_m) * kBM, (rest / tiles_m % tiles_n) * bn, sp};
 }
 
 template <int BN, int EPI>
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   uint64_t* acc_full = branch_empty + 1;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  uint32_t* last_flag = tmem_slot + 1;
+  constexpr bool kClusterK = EPI == static_cast<int>(GemmEpilogue::SplitK);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (p.M + kBM - 1) / kBM;
@@ -141,12 +145,15 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Split-K cluster barriers: A0 (every split CTA runs), R (every split's MMAs
+  // are done, so its operand ring may take remote stores), P (all rows pushed).
+  if constexpr (kClusterK) cluster_arrive();  // A0
 
-  // stage range [s_begin, s_begin + n_st) of a split
+  // stage range [s_begin, s_begin + n_st) of a split: balanced, every split of
+  // a tile gets at least one stage when splits <= k_stages
   auto stage_range = [&](int split, int& s_begin, int& n_st) {
-    s_begin = split * p.stages_per_split;
-    const int s_end = min(s_begin + p.stages_per_split, p.k_stages);
-    n_st = max(0, s_end - s_begin);
+    s_begin = split * p.k_stages / p.splits;
+    n_st = (split + 1) * p.k_stages / p.splits - s_begin;
   };
 
   if (warp < C::MMA_WARP) {
@@ -165,8 +172,9 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     int g = 0;  // global stage counter of this CTA
     int last = -1, nbranch = 0;
     bool ok = true;
+    bool dep_done = false;  // griddep_wait() done: A, its scales and U may be read
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN);
+      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
       int s_begin, n_st;
       stage_range(tc.split, s_begin, n_st);
       if (p.has_branch && tc.split == 0 && st == C::STAGES - 1) {
@@ -178,8 +186,13 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         }
         bok = __shfl_sync(0xffffffffu, bok, 0);
         if (!bok) break;
-        if (lane < 2)
-          tma_load_2d(smem + (lane ? C::OFF_L : C::OFF_U), lane ? &tmL : &tmU, branch_full, 0, lane ? tc.n0 : tc.m0);
+        // L (weights) may load before the activation producer has finished; U not
+        if (lane == 1) tma_load_2d(smem + C::OFF_L, &tmL, branch_full, 0, tc.n0);
+        if (!dep_done) {
+          griddep_wait();
+          dep_done = true;
+        }
+        if (lane == 0) tma_load_2d(smem + C::OFF_U, &tmU, branch_full, 0, tc.m0);
         ++nbranch;
       }
       for (int i = 0; i < n_st; ++i, ++g) {
@@ -195,8 +208,11 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         const int s = s_begin + i;
         if (lane == 0) mbar_arrive_expect_tx(&full[st], C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
         __syncwarp();
-        // one converged instruction: A, B, A scales, B scales (1 + BN/128 blocks of 1 KB)
-        if (lane < 3 + BN / 128) {
+        // one converged instruction: A, B, A scales, B scales (1 + BN/128 blocks of 1 KB).
+        // This warp's first stage issues the weight boxes, then waits for the
+        // kernel that writes A before issuing A and its scales.
+        const bool split_issue = !dep_done;
+        if (lane < 3 + BN / 128 && !(split_issue && (lane == 0 || lane == 2))) {
           const CUtensorMap* m;
           uint8_t* dst;
           int x, y;
@@ -214,6 +230,15 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
           }
           tma_load_2d(dst, m, &full[st], x, y);
         }
+        if (split_issue) {
+          griddep_wait();
+          dep_done = true;
+          if (lane == 0)
+            tma_load_2d(smem + C::OFF_A + st * C::A_BYTES, &tmA, &full[st], s * kStageBytes, tc.m0);
+          else if (lane == 2)
+            tma_load_2d(smem + C::OFF_SFA + st * C::SFA_BYTES, &tmSA, &full[st], 0,
+                        2 * ((tc.m0 / 128) * k64_total + kK64 * s));
+        }
         last = g;
       }
     }
@@ -223,6 +248,13 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       if (nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
     }
     __syncwarp();
+    if constexpr (kClusterK) {
+      cluster_wait();    // A0
+      cluster_arrive();  // R
+      cluster_wait();
+      cluster_arrive();  // P
+      cluster_wait();
+    }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -234,7 +266,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       int g = 0, tl = 0, nbranch = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tl) {
-        const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN);
+        const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
         int s_begin, n_st;
         stage_range(tc.split, s_begin, n_st);
         // the epilogue must have drained the previous tile's accumulator
@@ -277,6 +309,13 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       }
     }
     __syncwarp();
+    if constexpr (kClusterK) {
+      cluster_wait();    // A0
+      cluster_arrive();  // R
+      cluster_wait();
+      cluster_arrive();  // P
+      cluster_wait();
+    }
   } else {
     // ------------------------------------------------ epilogue
     const int ew = warp - C::EPI_WARP0;  // 0..7
@@ -284,13 +323,14 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     const int half = ew >> 2;            // column half [half*BN/2, (half+1)*BN/2)
     const int et = threadIdx.x - 32 * C::EPI_WARP0;
     constexpr int HC = BN / 2;           // columns per thread
+    griddep_wait();  // g_a is written by the kernel before this one
     const float gs = __fmul_rn(p.g_a_ptr ? *p.g_a_ptr : p.g_a, p.g_b);
     const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
     uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
     int tl = 0, g = 0;
     bool sf_ok = true;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
-      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN);
+      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
       // Scale blocks of this tile's stages: smem -> TMEM.  A warp's tcgen05.cp
       // instructions run one after another (~115 cycles each), so the 4 * NSF
       // copies of a stage are spread over the eight epilogue warps, which are
@@ -376,9 +416,8 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
             }
           }
         }
-      } else {
-        // fp32 out (raw or split-K partial): direct row stores
-        const float sc = (EPI == static_cast<int>(GemmEpilogue::RawF32)) ? gs : 1.0f;
+      } else if constexpr (EPI == static_cast<int>(GemmEpilogue::RawF32)) {
+        // fp32 out: direct row stores
 #pragma unroll 1
         for (int q = 0; q < HC / 32; ++q) {
           uint32_t r[32];
@@ -386,61 +425,72 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
           tmem_ld_wait();
           const int n = c0 + q * 32;
           if (!ok || row >= p.M || n >= p.N) continue;
-          float* dst = (EPI == static_cast<int>(GemmEpilogue::RawF32))
-                           ? p.out_f32 + static_cast<size_t>(row) * p.N + n
-                           : p.partial + (static_cast<size_t>(tc.split) * p.M + row) * p.N + n;
-          float4* d4 = reinterpret_cast<float4*>(dst);
+          float4* d4 = reinterpret_cast<float4*>(p.out_f32 + static_cast<size_t>(row) * p.N + n);
           const int nv = min(32, p.N - n) / 4;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             if (k < nv)
-              d4[k] = make_float4(__fmul_rn(__uint_as_float(r[4 * k]), sc), __fmul_rn(__uint_as_float(r[4 * k + 1]), sc),
-                                  __fmul_rn(__uint_as_float(r[4 * k + 2]), sc),
-                                  __fmul_rn(__uint_as_float(r[4 * k + 3]), sc));
+              d4[k] = make_float4(__fmul_rn(__uint_as_float(r[4 * k]), gs), __fmul_rn(__uint_as_float(r[4 * k + 1]), gs),
+                                  __fmul_rn(__uint_as_float(r[4 * k + 2]), gs),
+                                  __fmul_rn(__uint_as_float(r[4 * k + 3]), gs));
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
-        if constexpr (EPI == static_cast<int>(GemmEpilogue::SplitK)) {
-          __threadfence();
-          epi_bar();
-          const int tile = tc.m0 / kBM + tiles_m * (tc.n0 / BN);
-          if (et == 0) {
-            const uint32_t prev = atomicAdd(&p.counters[tile], 1u);
-            *last_flag = (prev == static_cast<uint32_t>(p.splits - 1)) ? 1u : 0u;
+      } else {
+        // Split-K: this tile's MMAs are done (acc_full), so this CTA's operand
+        // ring is idle.  Push accumulator rows to their owner's ring, laid out
+        // [split][row in slice][BN]; the owner sums them in split order.
+        const int SLR = kBM / p.splits;  // rows per owner
+        float* ring = reinterpret_cast<float*>(smem + C::OFF_A);
+        cluster_wait();    // A0
+        cluster_arrive();  // R
+        cluster_wait();
+        const int rloc = qd * 32 + lane;
+        const uint32_t dst = dsmem_addr(smem_u32(ring + (tc.split * SLR + rloc % SLR) * BN + half * HC),
+                                        static_cast<uint32_t>(rloc / SLR));
+#pragma unroll 1
+        for (int q = 0; q < HC / 32; ++q) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + q * 32, r);
+          tmem_ld_wait();
+          if (ok && row < p.M) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              dsmem_st_f4(dst + static_cast<uint32_t>((q * 32 + 4 * k) * 4),
+                          make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                      __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3])));
           }
-          epi_bar();
-          if (*last_flag) {
-            __threadfence();
-            const int rows_v = min(kBM, p.M - tc.m0), cols_v = min(BN, p.N - tc.n0);
-            const int c4 = cols_v / 4;
-            uint16_t* y = static_cast<uint16_t*>(p.y);
-            for (int idx = et; idx < rows_v * c4; idx += 32 * kEpiWarps) {
-              const int m = tc.m0 + idx / c4, n = tc.n0 + (idx % c4) * 4;
-              float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
-              for (int sp = 0; sp < p.splits; ++sp) {
-                const float4 v =
-                    __ldcg(reinterpret_cast<const float4*>(p.partial + (static_cast<size_t>(sp) * p.M + m) * p.N + n));
-                sacc.x = __fadd_rn(sacc.x, v.x);
-                sacc.y = __fadd_rn(sacc.y, v.y);
-                sacc.z = __fadd_rn(sacc.z, v.z);
-                sacc.w = __fadd_rn(sacc.w, v.w);
-              }
-              float b4[4] = {0.f, 0.f, 0.f, 0.f};
-              if (bias) {
-                const uint2 braw = __ldg(reinterpret_cast<const uint2*>(bias + n));
-                b4[0] = __uint_as_float(braw.x << 16);
-                b4[1] = __uint_as_float(braw.x & 0xffff0000u);
-                b4[2] = __uint_as_float(braw.y << 16);
-                b4[3] = __uint_as_float(braw.y & 0xffff0000u);
-              }
-              *reinterpret_cast<uint2*>(y + static_cast<size_t>(m) * p.N + n) =
-                  make_uint2(pack_bf16x2(__fmaf_rn(sacc.x, gs, b4[0]), __fmaf_rn(sacc.y, gs, b4[1])),
-                             pack_bf16x2(__fmaf_rn(sacc.z, gs, b4[2]), __fmaf_rn(sacc.w, gs, b4[3])));
-            }
-            if (et == 0) p.counters[tile] = 0u;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        cluster_arrive();  // P
+        cluster_wait();
+        uint16_t* y = static_cast<uint16_t*>(p.y);
+        for (int it = et; it < SLR * (BN / 4); it += 32 * kEpiWarps) {
+          const int srow = it / (BN / 4), c4 = it % (BN / 4);
+          const int m = tc.m0 + tc.split * SLR + srow, n = tc.n0 + 4 * c4;
+          if (m >= p.M || n >= p.N) continue;
+          float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int sp = 0; sp < p.splits; ++sp) {
+            const float4 v = *reinterpret_cast<const float4*>(ring + (sp * SLR + srow) * BN + 4 * c4);
+            sacc.x = __fadd_rn(sacc.x, v.x);
+            sacc.y = __fadd_rn(sacc.y, v.y);
+            sacc.z = __fadd_rn(sacc.z, v.z);
+            sacc.w = __fadd_rn(sacc.w, v.w);
           }
-          epi_bar();  // the ticket flag is reused by the next tile
+          float b4[4] = {0.f, 0.f, 0.f, 0.f};
+          if (bias) {
+            const uint2 braw = __ldg(reinterpret_cast<const uint2*>(bias + n));
+            b4[0] = __uint_as_float(braw.x << 16);
+            b4[1] = __uint_as_float(braw.x & 0xffff0000u);
+            b4[2] = __uint_as_float(braw.y << 16);
+            b4[3] = __uint_as_float(braw.y & 0xffff0000u);
+          }
+          *reinterpret_cast<uint2*>(y + static_cast<size_t>(m) * p.N + n) =
+              make_uint2(pack_bf16x2(__fmaf_rn(sacc.x, gs, b4[0]), __fmaf_rn(sacc.y, gs, b4[1])),
+                         pack_bf16x2(__fmaf_rn(sacc.z, gs, b4[2]), __fmaf_rn(sacc.w, gs, b4[3])));
         }
       }
     }
@@ -469,9 +519,29 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN) * p.splits;
-  const int grid = std::min(tiles, sms);
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(m.a, m.b, m.u, m.l, m.y, m.sfa, m.sfb, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (EPI == static_cast<int>(GemmEpilogue::SplitK)) {
+    // one work item per CTA; the splits of a tile are one cluster
+    if (p.splits < 2 || p.splits > 8 || (p.splits & (p.splits - 1)) || p.splits > p.k_stages)
+      return cudaErrorInvalidValue;
+    cfg.gridDim = dim3(tiles, 1, 1);
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = p.splits;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  } else {
+    cfg.gridDim = dim3(std::min(tiles, sms), 1, 1);
+  }
+  return cudaLaunchKernelEx(&cfg, kern, m.a, m.b, m.u, m.l, m.y, m.sfa, m.sfb, p);
 }
 
 template <int BN>

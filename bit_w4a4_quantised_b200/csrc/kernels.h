@@ -63,9 +63,8 @@ enum class GemmEpilogue { Bf16 = 0, RawF32 = 1, SplitK = 2 };
 
 struct GemmParams {
   int M, N, K;
-  int k_stages;            // ceil(K / 256)
-  int stages_per_split;
-  int splits;
+  int k_stages;            // K / 128 (one stage = 128 K)
+  int splits;              // 1, or 2 / 4 / 8 (split-K cluster; splits <= k_stages)
   const uint8_t* sfa;      // tiled, rows padded to 128
   const uint8_t* sfb;      // tiled, rows padded to 256
   const float* g_a_ptr;    // device scalar (activation scale) or nullptr
@@ -76,8 +75,6 @@ struct GemmParams {
   const void* bias;        // bf16 [N] or nullptr
   void* y;                 // bf16 [M, N]
   float* out_f32;          // fp32 [M, N] (raw epilogue)
-  float* partial;          // fp32 [splits, M, N]
-  uint32_t* counters;      // one per output tile, zero between launches
   uint32_t* err;
 };
 

@@ -130,6 +130,7 @@ template <int W>
 __device__ __forceinline__ void rotate_cols(const uint8_t* xs, const float* chan, int row, int s0, int b, float hscale,
                                             float (&v)[W]) {
   constexpr int NSEG = kChunk / W;
+  float2* v2 = reinterpret_cast<float2*>(v);  // element pairs (2i, 2i + 1)
 #pragma unroll
   for (int i = 0; i < W; ++i) v[i] = 0.0f;
 #pragma unroll
@@ -142,33 +143,44 @@ __device__ __forceinline__ void rotate_cols(const uint8_t* xs, const float* chan
 #pragma unroll
     for (int g = 0; g < W / 8; ++g) {
       const uint4 w = *reinterpret_cast<const uint4*>(box + (((c16 + g) ^ (row & 7)) << 4));
-      float t[8];
-      unpack8(w, t);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
       const float4 c0 = *reinterpret_cast<const float4*>(chan + col + 8 * g);
       const float4 c1 = *reinterpret_cast<const float4*>(chan + col + 8 * g + 4);
-      const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const float2 cc[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
+                            make_float2(c1.z, c1.w)};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float a = __fmul_rn(t[e], cc[e]);
-        v[8 * g + e] = neg ? __fsub_rn(v[8 * g + e], a) : __fadd_rn(v[8 * g + e], a);
+      for (int e = 0; e < 4; ++e) {
+        const float2 t = make_float2(__uint_as_float(ws[e] << 16), __uint_as_float(ws[e] & 0xffff0000u));
+        const float2 a = f2_mul(t, cc[e]);
+        v2[4 * g + e] = neg ? f2_sub(v2[4 * g + e], a) : f2_add(v2[4 * g + e], a);
       }
     }
   }
+  // stride 1 pairs the two lanes of a float2: scalar
+  if (b > 1) {
 #pragma unroll
-  for (int hh = 1; hh < W; hh <<= 1) {
+    for (int i = 0; i < W; i += 2) {
+      const float a = v[i], c = v[i + 1];
+      v[i] = __fadd_rn(a, c);
+      v[i + 1] = __fsub_rn(a, c);
+    }
+  }
+#pragma unroll
+  for (int hh = 2; hh < W; hh <<= 1) {
     if (hh < b) {
 #pragma unroll
-      for (int i = 0; i < W; ++i) {
+      for (int i = 0; i < W; i += 2) {
         if (!(i & hh)) {
-          const float a = v[i], c = v[i + hh];
-          v[i] = __fadd_rn(a, c);
-          v[i + hh] = __fsub_rn(a, c);
+          const float2 a = v2[i / 2], c = v2[(i + hh) / 2];
+          v2[i / 2] = f2_add(a, c);
+          v2[(i + hh) / 2] = f2_sub(a, c);
         }
       }
     }
   }
+  const float2 hs = make_float2(hscale, hscale);
 #pragma unroll
-  for (int i = 0; i < W; ++i) v[i] = __fmul_rn(v[i], hscale);
+  for (int i = 0; i < W / 2; ++i) v2[i] = f2_mul(v2[i], hs);
 }
 
 // Quantise this thread's W values of row `row`, chunk columns starting at `col`.
@@ -320,6 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // shared memory may take remote stores), A1 / A2 (partial c scattered / summed
   // c gathered), B (CTA amax published; Fused), C (no more remote access: exit).
   if constexpr (C::kCluster) cluster_arrive();  // A0
+  // the GEMM that consumes this launch's output may start its weight loads now
+  griddep_launch_dependents();
   const uint32_t d2_tmem = tmem;
   const uint32_t u_tmem = tmem + 128;
 
@@ -646,8 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r32[32];
             tmem_ld_32x32b_x32(d2_tmem + lane_base + s0 * W + pc * 32, r32);
             tmem_ld_wait();
+            float2* z2 = reinterpret_cast<float2*>(z + pc * 32);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) z[pc * 32 + k] = __fsub_rn(z[pc * 32 + k], __uint_as_float(r32[k]));
+            for (int k = 0; k < 16; ++k)
+              z2[k] = f2_sub(z2[k], make_float2(__uint_as_float(r32[2 * k]), __uint_as_float(r32[2 * k + 1])));
           }
         }
         tc_fence_before();

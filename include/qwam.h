@@ -108,17 +108,16 @@ qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, 
  * is budgeted at start-up.
  *
  * Same arguments, launches and result as qwam_linear (same kernels and the
- * same GEMM plan), but all scratch lives in one fixed 12 MiB array compiled
+ * same GEMM plan), but all scratch lives in one fixed 2 MiB array compiled
  * into the library (one copy per device) instead of the growable workspace.
  * Limits: M <= 128 rows and K <= 16384 (QWAM_ERR_SHAPE beyond them, before
  * anything is launched); within them every N, r and b that qwam_linear takes.
  * The first call on a device does the set-up (looks up the array's device
- * address and clears its header, synchronising the device); make that first
- * call before any latency-critical loop.  The scalars and split-K tile
- * tickets in that header must start at zero; the kernels leave the tickets at
- * zero after every completed call.  All calls share the one array per
- * device, whatever the handle: calls that overlap in time (other streams,
- * other threads) race on it and corrupt each other's results, so order them.
+ * address and clears its header, whose error word must start at zero,
+ * synchronising the device); make that first call before any latency-critical
+ * loop.  All calls share the one array per device, whatever the handle: calls
+ * that overlap in time (other streams, other threads) race on it and corrupt
+ * each other's results, so order them.
  * Expired bounded waits are reported by qwam_device_error.
  * ------------------------------------------------------------------------- */
 qwam_status qwam_linear_noalloc(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream);
