@@ -89,28 +89,37 @@ qwam_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
 }
 
 // Scale buffer of `rows_padded` rows (multiple of 128) and K columns in the tiled
-// layout, viewed as u8 [rows_padded * K / 16 / 256, 256]: one GEMM stage (two
-// 512-byte atoms) is a 256 x 4 box.
+// layout, viewed as u8 [rows_padded * K / 16 / 256, 256]: one slot of the GEMM's
+// scale ring (eight 512-byte atoms = eight K64 steps of 128 rows) is a 256 x 16 box.
 qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, int K) {
   const uint64_t total = static_cast<uint64_t>(rows_padded) * K / 16;
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, total / 256, 256, 256, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, total / 256, 256, 256, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Packed E2M1 operand [rows, K/2] u8 as the GEMM reads it: one box per stage of
+// ks K elements (ks / 2 bytes, one swizzle atom wide) by box_rows rows.
+qwam_status make_codes_map(CUtensorMap* m, const void* base, int rows, int K, int ks, int box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, K / 2, rows, K / 2, ks / 2, box_rows,
+                  ks == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B; }
 
 // ---- GEMM launch plan ------------------------------------------------------
 struct Plan {
-  int bn, k_stages, splits;
+  int bn, ks, k_stages, splits;
 };
 
 // Split-K when the output tiles leave SMs idle: the largest power of two <= 8
-// (one portable cluster per tile) with splits <= K / 128 and tiles * splits
+// (one portable cluster per tile) with splits <= k_stages and tiles * splits
 // within one wave of the SMs.
 Plan plan_gemm(int M, int N, int K) {
   Plan p{};
-  p.k_stages = (K + 127) / 128;
+  const GemmShape sh = gemm_shape(M, N);
+  p.bn = sh.bn;
+  p.ks = sh.ks;
+  p.k_stages = (K + p.ks - 1) / p.ks;
   const int tiles_m = (M + 127) / 128;
-  p.bn = (M <= 128 || N < 256) ? 128 : 256;
   const int tiles = tiles_m * ((N + p.bn - 1) / p.bn);
   p.splits = 1;
   for (int c = 8; c >= 2; c >>= 1)
@@ -204,7 +213,7 @@ struct qwam_layer {
   uint16_t* bias;
   float g_w;
   size_t sf_bytes;
-  CUtensorMap map_b128, map_b256, map_l128, map_l256, map_sfb;
+  CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256, map_sfb;
   ProMaps vmaps;  // P^T and V (hi/lo) tensor maps for the prologue; x is per call
 };
 
@@ -364,10 +373,9 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   if (host_scr[3]) return cleanup(fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired in prepare (flags 0x%x)", host_scr[3]));
   std::memcpy(&h->g_w, &host_scr[2], 4);
 
-  if ((s_ = make_map(&h->map_b128, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 64, 128,
-                     CU_TENSOR_MAP_SWIZZLE_64B)) != QWAM_OK ||
-      (s_ = make_map(&h->map_b256, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->codes, K / 2, N, K / 2, 64, 256,
-                     CU_TENSOR_MAP_SWIZZLE_64B)) != QWAM_OK)
+  if ((s_ = make_codes_map(&h->map_b128_k128, h->codes, N, K, 128, 128)) != QWAM_OK ||
+      (s_ = make_codes_map(&h->map_b128_k256, h->codes, N, K, 256, 128)) != QWAM_OK ||
+      (s_ = make_codes_map(&h->map_b256_k256, h->codes, N, K, 256, 256)) != QWAM_OK)
     return cleanup(s_);
   if ((s_ = make_sf_map(&h->map_sfb, h->sf, round_up(static_cast<size_t>(N), 256), K)) != QWAM_OK) return cleanup(s_);
   if (r > 0) {
@@ -377,8 +385,8 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
             QWAM_OK)
       return cleanup(s_);
   } else {
-    h->map_l128 = h->map_b128;
-    h->map_l256 = h->map_b256;
+    h->map_l128 = h->map_b128_k128;
+    h->map_l256 = h->map_b256_k256;
   }
   cudaFree(u_tmp);
   cudaFree(scratch);
@@ -432,9 +440,8 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   Arena* a = nullptr;
   QW_TRY(arena_get(h->dev, lay.total, &a));
   GemmMaps maps{};
-  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->base + lay.codes, h->K / 2, M, h->K / 2, 64, 128,
-                  CU_TENSOR_MAP_SWIZZLE_64B));
-  maps.b = pl.bn == 256 ? h->map_b256 : h->map_b128;
+  QW_TRY(make_codes_map(&maps.a, a->base + lay.codes, M, h->K, pl.ks, 128));
+  maps.b = pl.bn == 256 ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
   QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K));
   maps.sfb = h->map_sfb;
   if (h->r > 0) {
@@ -463,7 +470,8 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   p.bias = h->bias;
   p.y = y;
   p.err = arena_err(*a);
-  QW_CUDA(launch_gemm(maps, p, pl.bn, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
+  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
+                      st));
   return QWAM_OK;
 }
 
@@ -544,9 +552,8 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   QW_TRY(run_rows(x, prm, h->r, h->vmaps, true, amax, st));
 
   GemmMaps maps{};
-  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, base + lay.codes, h->K / 2, M, h->K / 2, 64, 128,
-                  CU_TENSOR_MAP_SWIZZLE_64B));
-  maps.b = pl.bn == 256 ? h->map_b256 : h->map_b128;
+  QW_TRY(make_codes_map(&maps.a, base + lay.codes, M, h->K, pl.ks, 128));
+  maps.b = pl.bn == 256 ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
   QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K));
   maps.sfb = h->map_sfb;
   if (h->r > 0) {
@@ -575,7 +582,8 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   p.bias = h->bias;
   p.y = y;
   p.err = err;
-  QW_CUDA(launch_gemm(maps, p, pl.bn, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
+  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
+                      st));
   return QWAM_OK;
 }
 
@@ -704,18 +712,18 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   QW_TRY(current_device(&dev));
   Arena* a = nullptr;
   QW_TRY(arena_get(dev, kHeaderBytes, &a));
-  const int bn = N > 128 ? 256 : 128;
+  const GemmShape sh = gemm_shape(M, N);
   GemmMaps maps{};
-  QW_TRY(make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B));
-  QW_TRY(make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, K / 2, N, K / 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_64B));
+  QW_TRY(make_codes_map(&maps.a, a_codes, M, K, sh.ks, 128));
+  QW_TRY(make_codes_map(&maps.b, b_codes, N, K, sh.ks, sh.bn));
   maps.u = maps.a;
   maps.l = maps.b;
   maps.y = maps.a;
   QW_TRY(make_sf_map(&maps.sfa, a_scales, round_up(static_cast<size_t>(M), 128), K));
-  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), bn), K));
+  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), sh.bn), K));
   GemmParams p{};
   p.M = M; p.N = N; p.K = K;
-  p.k_stages = (K + 127) / 128;
+  p.k_stages = (K + sh.ks - 1) / sh.ks;
   p.splits = 1;
   p.sfa = static_cast<const uint8_t*>(a_scales);
   p.sfb = static_cast<const uint8_t*>(b_scales);
@@ -724,7 +732,7 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   p.g_b = 1.0f;
   p.out_f32 = out_f32;
   p.err = arena_err(*a);
-  QW_CUDA(launch_gemm(maps, p, bn, GemmEpilogue::RawF32, as_stream(stream)));
+  QW_CUDA(launch_gemm(maps, p, sh, GemmEpilogue::RawF32, as_stream(stream)));
   return QWAM_OK;
 }
 

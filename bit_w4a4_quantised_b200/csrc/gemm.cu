@@ -12,19 +12,21 @@
 // quantisations", section "What ASP is...": y = (x~V)(W~V)^T + NVFP4GEMM(...) +
 // bias; branch kept in bf16).
 //
-// Persistent kernel, one CTA per SM, tiles of 128 x BN (K in 128-element
-// stages, one 64B-swizzle atom of packed E2M1 per row, K64 per MMA; 6-8 stages
-// in flight to cover the ~0.7 us TMA latency).  Roles:
-//   producer warps  one per shared-memory ring slot; each stage is one
-//                   converged TMA instruction (A, B and their scale blocks on
-//                   four or five lanes).  A TMA instruction holds its warp for a
-//                   fixed ~600 cycles, so the slots have their own warps.
+// Persistent kernel, one CTA per SM, tiles of 128 x BN, K in stages of KS
+// elements (KS / 2 bytes of packed E2M1 per row: one 128B- or 64B-swizzle
+// atom), K64 per MMA.  On this part the TMA engine costs a roughly fixed time
+// per box, so the operands come in few, large boxes: one A and one B box per
+// stage, and the E4M3 scale blocks on a ring of their own, eight K64 steps
+// (4 KB per 128 rows) per box.  Roles:
+//   producer warps  one per operand ring slot (a TMA instruction holds its warp
+//                   for a fixed ~600 cycles); the first stage's weight box goes
+//                   out before the wait on the kernel that writes A.
+//   scale warp      loads the scale ring.
 //   MMA warp        owns TMEM; issues only tcgen05.mma (bf16 branch, then FP4).
 //   epilogue warps  eight, two per TMEM lane quarter (column halves).  While a
-//                   tile accumulates they copy each stage's scale blocks into the
-//                   slot's TMEM scale columns (tcgen05.cp; a warp's copies run one
-//                   after another, so eight warps share them and the copies run
-//                   beside the MMAs, not between them).  Then they drain the
+//                   tile accumulates they copy the scale blocks into a TMEM
+//                   scale ring (tcgen05.cp; a warp's copies run one after
+//                   another, so eight warps share them).  Then they drain the
 //                   accumulator to registers, release it to the next tile, add
 //                   bias, round to bf16, stage through 128B-swizzled smem and
 //                   store with TMA (ragged M / N are clipped by the tensor map).
@@ -43,46 +45,47 @@ namespace qwam {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kStageBytes = 64;   // bytes per row per stage: 128 E2M1 codes, one 64B-swizzle atom
-constexpr int kK64 = 2;           // K64 MMA steps per stage
 constexpr int kEpiWarps = 8;
+constexpr int kSFK = 8;  // K64 steps per scale-ring slot
 
-template <int BN>
+template <int BN, int KS>
 struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 6 : 8;
-  static constexpr int NSF = 1 + BN / 128;                  // scale block columns (A, B halves)
-  static constexpr int MMA_WARP = STAGES;
-  static constexpr int EPI_WARP0 = MMA_WARP + 1;
+  static constexpr int ROWB = KS / 2;                       // operand bytes per row per stage
+  static constexpr int K64 = KS / 64;                       // MMAs per stage
+  static constexpr uint32_t SWZ = ROWB == 128 ? 2u : 4u;    // UMMA layout: 128B / 64B swizzle
+  static constexpr int STAGES = KS == 256 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8);
+  static constexpr int NSFB = BN / 128;                     // 128-row scale blocks of B
+  static constexpr int SF_ATOMS = kSFK * 512;               // one 128-row scale block of a slot
+  static constexpr int SF_SLOT = SF_ATOMS * (1 + NSFB);
+  static constexpr int SF_WARP = STAGES;
+  static constexpr int MMA_WARP = STAGES + 1;
+  static constexpr int EPI_WARP0 = STAGES + 2;
   static constexpr int THREADS = 32 * (EPI_WARP0 + kEpiWarps);
-  static constexpr int A_BYTES = kBM * kStageBytes;
-  static constexpr int B_BYTES = BN * kStageBytes;
-  static constexpr int SFA_BYTES = kK64 * 512;
-  static constexpr int SFB_BYTES = (BN / 128) * kK64 * 512;
+  static constexpr int A_BYTES = kBM * ROWB;
+  static constexpr int B_BYTES = BN * ROWB;
   static constexpr int U_BYTES = kBM * 64;
   static constexpr int L_BYTES = BN * 64;
   static constexpr int STG_BYTES = 4096;                    // per epilogue warp: 32 rows x 128 B
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_U = OFF_SFB + STAGES * SFB_BYTES;
+  static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_U = OFF_SF + 2 * SF_SLOT;
   static constexpr int OFF_L = OFF_U + U_BYTES;
   static constexpr int OFF_STG = OFF_L + L_BYTES;
   static constexpr int OFF_BAR = OFF_STG + kEpiWarps * STG_BYTES;
-  static constexpr int NBAR = 3 * STAGES + 4;
+  static constexpr int NBAR = 2 * STAGES + 6 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  // TMEM columns: accumulator [0, BN), then per slot kK64 steps of scale
-  // factors: A needs 4 columns per step (128 rows), B needs BN/32.
-  static constexpr int SF_A_COLS = kK64 * 4;
-  static constexpr int SF_COLS = SF_A_COLS + kK64 * (BN / 32);
-  static constexpr int TMEM_USED = BN + STAGES * SF_COLS;
+  // TMEM columns: accumulator [0, BN), then two scale slots, each kSFK K64
+  // steps of A (4 columns) then of B (BN / 32 columns).
+  static constexpr int SF_A_COLS = kSFK * 4;
+  static constexpr int SF_COLS = SF_A_COLS + kSFK * (BN / 32);
+  static constexpr int TMEM_USED = BN + 2 * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(kBM * BN * 4 <= STAGES * (A_BYTES + B_BYTES), "split-K receive area fits in the operand ring");
 };
-
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return pack2(bf16_bits_rn(a), bf16_bits_rn(b));
@@ -100,19 +103,21 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n,
   return {(rest % tiles_m) * kBM, (rest / tiles_m % tiles_n) * bn, sp};
 }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
+template <int BN, int KS, int EPI>
+__global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmSA,
                     const __grid_constant__ CUtensorMap tmSB, const GemmParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, KS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // TMA landed
-  uint64_t* sf_ready = full + C::STAGES;                            // scale copies done
-  uint64_t* empty = sf_ready + C::STAGES;                           // MMAs done with slot
-  uint64_t* branch_full = empty + C::STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES] A/B landed
+  uint64_t* empty = full + C::STAGES;                               // [STAGES] MMAs done with the slot
+  uint64_t* sf_full = empty + C::STAGES;                            // [2] scale boxes landed
+  uint64_t* sf_ready = sf_full + 2;                                 // [2] scales copied to TMEM (smem free)
+  uint64_t* sf_tfree = sf_ready + 2;                                // [2] MMAs done with the TMEM scale slot
+  uint64_t* branch_full = sf_tfree + 2;
   uint64_t* branch_empty = branch_full + 1;
   uint64_t* acc_full = branch_empty + 1;
   uint64_t* acc_empty = acc_full + 1;
@@ -128,8 +133,12 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&sf_ready[i], kEpiWarps);
       mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sf_full[i], 1);
+      mbar_init(&sf_ready[i], kEpiWarps);
+      mbar_init(&sf_tfree[i], 1);
     }
     mbar_init(branch_full, 1);
     mbar_init(branch_empty, 1);
@@ -149,34 +158,40 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   // are done, so its operand ring may take remote stores), P (all rows pushed).
   if constexpr (kClusterK) cluster_arrive();  // A0
 
-  // stage range [s_begin, s_begin + n_st) of a split: balanced, every split of
-  // a tile gets at least one stage when splits <= k_stages
-  auto stage_range = [&](int split, int& s_begin, int& n_st) {
-    s_begin = split * p.k_stages / p.splits;
-    n_st = (split + 1) * p.k_stages / p.splits - s_begin;
+  // A split's K range: stages [s_begin, s_begin + n_st) (balanced: every split
+  // gets at least one stage when splits <= k_stages), K64 steps
+  // [k64_begin, k64_begin + n_k64), scale slots of kSFK steps.
+  struct Range {
+    int s_begin, n_st, k64_begin, n_k64, nsf;
+  };
+  auto range_of = [&](int split) {
+    Range r;
+    r.s_begin = split * p.k_stages / p.splits;
+    r.n_st = (split + 1) * p.k_stages / p.splits - r.s_begin;
+    r.k64_begin = r.s_begin * C::K64;
+    r.n_k64 = min(r.n_st * C::K64, k64_total - r.k64_begin);
+    r.nsf = (r.n_k64 + kSFK - 1) / kSFK;
+    return r;
   };
 
-  if (warp < C::MMA_WARP) {
-    // ------------------------------------------------ producers: warp st owns slot st
+  if (warp < C::STAGES) {
+    // ------------------------------------------------ operand producers: warp st owns slot st
     const int st = warp;
     if (lane == 0 && st == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      tma_prefetch_desc(&tmSA);
-      tma_prefetch_desc(&tmSB);
       if (p.has_branch) {
         tma_prefetch_desc(&tmU);
         tma_prefetch_desc(&tmL);
       }
     }
-    int g = 0;  // global stage counter of this CTA
+    int g = 0;  // stage counter of this CTA
     int last = -1, nbranch = 0;
     bool ok = true;
-    bool dep_done = false;  // griddep_wait() done: A, its scales and U may be read
+    bool dep_done = false;  // griddep_wait() done: A and U may be read
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
       const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
-      int s_begin, n_st;
-      stage_range(tc.split, s_begin, n_st);
+      const Range rg = range_of(tc.split);
       if (p.has_branch && tc.split == 0 && st == C::STAGES - 1) {
         // branch operands of this tile, once the previous tile's branch MMAs are done
         int bok = 1;
@@ -195,7 +210,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         if (lane == 0) tma_load_2d(smem + C::OFF_U, &tmU, branch_full, 0, tc.m0);
         ++nbranch;
       }
-      for (int i = 0; i < n_st; ++i, ++g) {
+      for (int i = 0; i < rg.n_st; ++i, ++g) {
         if (g % C::STAGES != st) continue;
         const uint32_t ph = (g / C::STAGES) & 1;
         int wok = 1;
@@ -205,39 +220,20 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
           ok = false;
           break;
         }
-        const int s = s_begin + i;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
+        const int x = (rg.s_begin + i) * C::ROWB;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::A_BYTES + C::B_BYTES);
         __syncwarp();
-        // one converged instruction: A, B, A scales, B scales (1 + BN/128 blocks of 1 KB).
-        // This warp's first stage issues the weight boxes, then waits for the
-        // kernel that writes A before issuing A and its scales.
-        const bool split_issue = !dep_done;
-        if (lane < 3 + BN / 128 && !(split_issue && (lane == 0 || lane == 2))) {
-          const CUtensorMap* m;
-          uint8_t* dst;
-          int x, y;
-          if (lane == 0) {
-            m = &tmA; dst = smem + C::OFF_A + st * C::A_BYTES; x = s * kStageBytes; y = tc.m0;
-          } else if (lane == 1) {
-            m = &tmB; dst = smem + C::OFF_B + st * C::B_BYTES; x = s * kStageBytes; y = tc.n0;
-          } else if (lane == 2) {
-            m = &tmSA; dst = smem + C::OFF_SFA + st * C::SFA_BYTES; x = 0;
-            y = 2 * ((tc.m0 / 128) * k64_total + kK64 * s);
-          } else {
-            const int j = lane - 3;
-            m = &tmSB; dst = smem + C::OFF_SFB + st * C::SFB_BYTES + j * (kK64 * 512); x = 0;
-            y = 2 * ((tc.n0 / 128 + j) * k64_total + kK64 * s);
-          }
-          tma_load_2d(dst, m, &full[st], x, y);
-        }
-        if (split_issue) {
+        if (dep_done) {
+          // one converged instruction: A on lane 0, B on lane 1
+          if (lane < 2)
+            tma_load_2d(smem + (lane ? C::OFF_B + st * C::B_BYTES : C::OFF_A + st * C::A_BYTES), lane ? &tmB : &tmA,
+                        &full[st], x, lane ? tc.n0 : tc.m0);
+        } else {
+          // the weights first, then A once the kernel writing it has finished
+          if (lane == 1) tma_load_2d(smem + C::OFF_B + st * C::B_BYTES, &tmB, &full[st], x, tc.n0);
           griddep_wait();
           dep_done = true;
-          if (lane == 0)
-            tma_load_2d(smem + C::OFF_A + st * C::A_BYTES, &tmA, &full[st], s * kStageBytes, tc.m0);
-          else if (lane == 2)
-            tma_load_2d(smem + C::OFF_SFA + st * C::SFA_BYTES, &tmSA, &full[st], 0,
-                        2 * ((tc.m0 / 128) * k64_total + kK64 * s));
+          if (lane == 0) tma_load_2d(smem + C::OFF_A + st * C::A_BYTES, &tmA, &full[st], x, tc.m0);
         }
         last = g;
       }
@@ -255,6 +251,47 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       cluster_arrive();  // P
       cluster_wait();
     }
+  } else if (warp == C::SF_WARP) {
+    // ------------------------------------------------ scale producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmSA);
+      tma_prefetch_desc(&tmSB);
+      int q = 0, last = -1;
+      bool ok = true, dep_done = false;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
+        const Range rg = range_of(tc.split);
+        for (int j = 0; j < rg.nsf; ++j, ++q) {
+          const int s = q & 1;
+          if (q >= 2 && !mbar_wait(&sf_ready[s], ((q >> 1) & 1) ^ 1u, p.err, DEVERR_PRODUCER_WAIT)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = smem + C::OFF_SF + s * C::SF_SLOT;
+          const int atom = rg.k64_begin + j * kSFK;  // first K64 step of the slot
+          mbar_arrive_expect_tx(&sf_full[s], C::SF_SLOT);
+#pragma unroll
+          for (int h = 0; h < C::NSFB; ++h)
+            tma_load_2d(dst + (1 + h) * C::SF_ATOMS, &tmSB, &sf_full[s], 0,
+                        2 * ((tc.n0 / 128 + h) * k64_total + atom));
+          if (!dep_done) {
+            griddep_wait();
+            dep_done = true;
+          }
+          tma_load_2d(dst, &tmSA, &sf_full[s], 0, 2 * ((tc.m0 / 128) * k64_total + atom));
+          last = q;
+        }
+      }
+      if (last >= 0) mbar_wait(&sf_full[last & 1], (last >> 1) & 1, p.err, DEVERR_DRAIN_WAIT);
+    }
+    __syncwarp();
+    if constexpr (kClusterK) {
+      cluster_wait();    // A0
+      cluster_arrive();  // R
+      cluster_wait();
+      cluster_arrive();  // P
+      cluster_wait();
+    }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -263,12 +300,11 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
       const uint32_t sbo = 8u * p.branch_k * 2u;
       const uint32_t us = smem_u32(smem + C::OFF_U), ls = smem_u32(smem + C::OFF_L);
-      int g = 0, tl = 0, nbranch = 0;
+      int g = 0, q0 = 0, tl = 0, nbranch = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tl) {
         const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
-        int s_begin, n_st;
-        stage_range(tc.split, s_begin, n_st);
+        const Range rg = range_of(tc.split);
         // the epilogue must have drained the previous tile's accumulator
         if (!mbar_wait(acc_empty, (tl & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) break;
         tc_fence_after();
@@ -284,27 +320,37 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
           tc_commit(branch_empty);
           ++nbranch;
         }
-        for (int i = 0; i < n_st; ++i, ++g) {
+        int kloc = 0;  // K64 step within this split
+        for (int i = 0; ok && i < rg.n_st; ++i, ++g) {
           const int st = g % C::STAGES;
-          const uint32_t ph = (g / C::STAGES) & 1;
-          if (!mbar_wait(&sf_ready[st], ph, p.err, DEVERR_MMA_WAIT) ||
-              !mbar_wait(&full[st], ph, p.err, DEVERR_MMA_WAIT)) {
+          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_MMA_WAIT)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int s = s_begin + i;
-          const int nk = min(kK64, k64_total - kK64 * s);
-          const uint32_t sf_col = BN + st * C::SF_COLS;
           const uint32_t a_s = smem_u32(smem + C::OFF_A + st * C::A_BYTES);
           const uint32_t b_s = smem_u32(smem + C::OFF_B + st * C::B_BYTES);
-          for (int kk = 0; kk < nk; ++kk) {
-            mma_mxf4nvf4(tmem, smem_desc(a_s + kk * 32, 16, 512, 4), smem_desc(b_s + kk * 32, 16, 512, 4), idesc_fp4,
-                         tmem + sf_col + kk * 4, tmem + sf_col + C::SF_A_COLS + kk * (BN / 32), accum);
+          const int nk = min(C::K64, rg.n_k64 - i * C::K64);
+          for (int kk = 0; kk < nk; ++kk, ++kloc) {
+            const int cur = q0 + kloc / kSFK;  // scale slot of this step
+            const int ks = kloc % kSFK;
+            if (ks == 0) {
+              if (!mbar_wait(&sf_ready[cur & 1], (cur >> 1) & 1, p.err, DEVERR_MMA_WAIT)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            const uint32_t sf_col = BN + (cur & 1) * C::SF_COLS;
+            mma_mxf4nvf4(tmem, smem_desc(a_s + kk * 32, 16, 8 * C::ROWB, C::SWZ),
+                         smem_desc(b_s + kk * 32, 16, 8 * C::ROWB, C::SWZ), idesc_fp4, tmem + sf_col + ks * 4,
+                         tmem + sf_col + C::SF_A_COLS + ks * (BN / 32), accum);
             accum = 1;
+            if (ks == kSFK - 1 || kloc == rg.n_k64 - 1) tc_commit(&sf_tfree[cur & 1]);
           }
           tc_commit(&empty[st]);
         }
+        q0 += rg.nsf;
         tc_commit(acc_full);
       }
     }
@@ -327,47 +373,42 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     const float gs = __fmul_rn(p.g_a_ptr ? *p.g_a_ptr : p.g_a, p.g_b);
     const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
     uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
-    int tl = 0, g = 0;
+    int tl = 0, q = 0;
     bool sf_ok = true;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
       const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
-      // Scale blocks of this tile's stages: smem -> TMEM.  A warp's tcgen05.cp
-      // instructions run one after another (~115 cycles each), so the 4 * NSF
-      // copies of a stage are spread over the eight epilogue warps, which are
-      // otherwise idle while the tile accumulates.
-      {
-        int s_begin, n_st;
-        stage_range(tc.split, s_begin, n_st);
-        for (int i = 0; i < n_st; ++i, ++g) {
-          const int st = g % C::STAGES;
-          int wok = 1;
-          if (lane == 0) wok = (sf_ok && mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_EPILOGUE_WAIT)) ? 1 : 0;
-          wok = __shfl_sync(0xffffffffu, wok, 0);
-          if (!wok) {
-            sf_ok = false;
-            continue;
-          }
-          if (lane == 0) {
-            tc_fence_after();
-            const int s = s_begin + i;
-            const int nk = min(kK64, k64_total - kK64 * s);
-            const uint32_t sf_col = BN + st * C::SF_COLS;
-            for (int c = ew; c < kK64 * C::NSF; c += kEpiWarps) {
-              const int col = c / kK64, kk = c % kK64;
-              if (kk >= nk) continue;
-              if (col == 0)
-                tmem_cp_32x128b_x4(tmem + sf_col + kk * 4,
-                                   smem_desc(smem_u32(smem + C::OFF_SFA + st * C::SFA_BYTES) + kk * 512, 0, 128, 0));
-              else
-                tmem_cp_32x128b_x4(
-                    tmem + sf_col + C::SF_A_COLS + kk * (BN / 32) + (col - 1) * 4,
-                    smem_desc(smem_u32(smem + C::OFF_SFB + st * C::SFB_BYTES) + (col - 1) * (kK64 * 512) + kk * 512, 0,
-                              128, 0));
-            }
-            tc_commit(&sf_ready[st]);
-          }
-          __syncwarp();
+      const Range rg = range_of(tc.split);
+      // Scale blocks of this tile: smem ring -> TMEM ring.  A warp's tcgen05.cp
+      // instructions run one after another (~115 cycles each), so a slot's
+      // copies are spread over the eight epilogue warps, which are otherwise
+      // idle while the tile accumulates.
+      for (int j = 0; j < rg.nsf; ++j, ++q) {
+        const int s = q & 1;
+        int wok = 1;
+        if (lane == 0)
+          wok = (sf_ok && mbar_wait(&sf_full[s], (q >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT) &&
+                 (q < 2 || mbar_wait(&sf_tfree[s], ((q >> 1) & 1) ^ 1u, p.err, DEVERR_EPILOGUE_WAIT)))
+                    ? 1
+                    : 0;
+        wok = __shfl_sync(0xffffffffu, wok, 0);
+        if (!wok) {
+          sf_ok = false;
+          continue;
         }
+        if (lane == 0) {
+          tc_fence_after();
+          const int nk = min(kSFK, rg.n_k64 - j * kSFK);
+          const uint32_t src = smem_u32(smem + C::OFF_SF + s * C::SF_SLOT);
+          const uint32_t col0 = BN + s * C::SF_COLS;
+          for (int c = ew; c < kSFK * (1 + C::NSFB); c += kEpiWarps) {
+            const int blk = c / kSFK, kk = c % kSFK;
+            if (kk >= nk) continue;
+            const uint32_t col = blk == 0 ? col0 + kk * 4 : col0 + C::SF_A_COLS + kk * (BN / 32) + (blk - 1) * 4;
+            tmem_cp_32x128b_x4(tmem + col, smem_desc(src + blk * C::SF_ATOMS + kk * 512, 0, 128, 0));
+          }
+          tc_commit(&sf_ready[s]);
+        }
+        __syncwarp();
       }
       const bool ok = sf_ok && mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT);
       __syncwarp();
@@ -378,18 +419,19 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         // drain: fp32 accumulator -> bf16 pairs in registers, then release
         uint32_t packed[HC / 2];
 #pragma unroll
-        for (int q = 0; q < HC / 32; ++q) {
+        for (int qq = 0; qq < HC / 32; ++qq) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + q * 32, r);
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + qq * 32, r);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint4 braw = make_uint4(0u, 0u, 0u, 0u);
-            if (bias && c0 + q * 32 + 8 * j < p.N) braw = __ldg(reinterpret_cast<const uint4*>(bias + c0 + q * 32 + 8 * j));
+            if (bias && c0 + qq * 32 + 8 * j < p.N)
+              braw = __ldg(reinterpret_cast<const uint4*>(bias + c0 + qq * 32 + 8 * j));
             const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              packed[q * 16 + 4 * j + k] =
+              packed[qq * 16 + 4 * j + k] =
                   pack_bf16x2(__fmaf_rn(__uint_as_float(r[8 * j + 2 * k]), gs, __uint_as_float(bw[k] << 16)),
                               __fmaf_rn(__uint_as_float(r[8 * j + 2 * k + 1]), gs, __uint_as_float(bw[k] & 0xffff0000u)));
           }
@@ -419,11 +461,11 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       } else if constexpr (EPI == static_cast<int>(GemmEpilogue::RawF32)) {
         // fp32 out: direct row stores
 #pragma unroll 1
-        for (int q = 0; q < HC / 32; ++q) {
+        for (int qq = 0; qq < HC / 32; ++qq) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + q * 32, r);
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + qq * 32, r);
           tmem_ld_wait();
-          const int n = c0 + q * 32;
+          const int n = c0 + qq * 32;
           if (!ok || row >= p.M || n >= p.N) continue;
           float4* d4 = reinterpret_cast<float4*>(p.out_f32 + static_cast<size_t>(row) * p.N + n);
           const int nv = min(32, p.N - n) / 4;
@@ -450,14 +492,14 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         const uint32_t dst = dsmem_addr(smem_u32(ring + (tc.split * SLR + rloc % SLR) * BN + half * HC),
                                         static_cast<uint32_t>(rloc / SLR));
 #pragma unroll 1
-        for (int q = 0; q < HC / 32; ++q) {
+        for (int qq = 0; qq < HC / 32; ++qq) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + q * 32, r);
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + qq * 32, r);
           tmem_ld_wait();
           if (ok && row < p.M) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              dsmem_st_f4(dst + static_cast<uint32_t>((q * 32 + 4 * k) * 4),
+              dsmem_st_f4(dst + static_cast<uint32_t>((qq * 32 + 4 * k) * 4),
                           make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
                                       __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3])));
           }
@@ -507,10 +549,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int KS, int EPI>
 cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
-  using C = Cfg<BN>;
-  auto kern = fp4_gemm_kernel<BN, EPI>;
+  using C = Cfg<BN, KS>;
+  auto kern = fp4_gemm_kernel<BN, KS, EPI>;
   static const cudaError_t smem_attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (smem_attr != cudaSuccess) return smem_attr;
@@ -518,6 +560,7 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
+  if (p.k_stages != (p.K + KS - 1) / KS) return cudaErrorInvalidValue;
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN) * p.splits;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(C::THREADS, 1, 1);
@@ -539,28 +582,36 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   } else {
+    if (p.splits != 1) return cudaErrorInvalidValue;
     cfg.gridDim = dim3(std::min(tiles, sms), 1, 1);
   }
   return cudaLaunchKernelEx(&cfg, kern, m.a, m.b, m.u, m.l, m.y, m.sfa, m.sfb, p);
 }
 
-template <int BN>
+template <int BN, int KS>
 cudaError_t launch_bn(const GemmMaps& m, const GemmParams& p, GemmEpilogue epi, cudaStream_t st) {
   switch (epi) {
-    case GemmEpilogue::Bf16: return launch_t<BN, 0>(m, p, st);
-    case GemmEpilogue::RawF32: return launch_t<BN, 1>(m, p, st);
-    case GemmEpilogue::SplitK: return launch_t<BN, 2>(m, p, st);
+    case GemmEpilogue::Bf16: return launch_t<BN, KS, 0>(m, p, st);
+    case GemmEpilogue::RawF32: return launch_t<BN, KS, 1>(m, p, st);
+    case GemmEpilogue::SplitK: return launch_t<BN, KS, 2>(m, p, st);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-size_t gemm_smem_bytes(int bn) { return bn == 256 ? Cfg<256>::SMEM : Cfg<128>::SMEM; }
+GemmShape gemm_shape(int M, int N) {
+  GemmShape s;
+  s.bn = (M <= kBM || N < 256) ? 128 : 256;
+  s.ks = M <= kBM ? 128 : 256;
+  return s;
+}
 
-cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int bn, GemmEpilogue epi, cudaStream_t st) {
-  if (bn == 256) return launch_bn<256>(maps, p, epi, st);
-  if (bn == 128) return launch_bn<128>(maps, p, epi, st);
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
+                        cudaStream_t st) {
+  if (shape.bn == 256 && shape.ks == 256) return launch_bn<256, 256>(maps, p, epi, st);
+  if (shape.bn == 128 && shape.ks == 256) return launch_bn<128, 256>(maps, p, epi, st);
+  if (shape.bn == 128 && shape.ks == 128) return launch_bn<128, 128>(maps, p, epi, st);
   return cudaErrorInvalidValue;
 }
 

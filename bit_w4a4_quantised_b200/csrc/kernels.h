@@ -63,7 +63,7 @@ enum class GemmEpilogue { Bf16 = 0, RawF32 = 1, SplitK = 2 };
 
 struct GemmParams {
   int M, N, K;
-  int k_stages;            // K / 128 (one stage = 128 K)
+  int k_stages;            // ceil(K / ks), ks = K elements per pipeline stage
   int splits;              // 1, or 2 / 4 / 8 (split-K cluster; splits <= k_stages)
   const uint8_t* sfa;      // tiled, rows padded to 128
   const uint8_t* sfb;      // tiled, rows padded to 256
@@ -79,16 +79,24 @@ struct GemmParams {
 };
 
 struct GemmMaps {
-  CUtensorMap a;  // codes A [M, K/2] u8, box 64 B x 128 rows, 64B swizzle
-  CUtensorMap b;  // codes B [N, K/2] u8, box 64 B x BN rows, 64B swizzle
-  CUtensorMap u;  // branch A [M, r] bf16, box r x 128 rows
-  CUtensorMap l;  // branch B [N, r] bf16, box r x BN rows
+  CUtensorMap a;    // codes A [M, K/2] u8, box (ks/2) B x 128 rows, 128B (ks 256) / 64B (ks 128) swizzle
+  CUtensorMap b;    // codes B [N, K/2] u8, box (ks/2) B x bn rows, same swizzle
+  CUtensorMap u;    // branch A [M, r] bf16, box r x 128 rows
+  CUtensorMap l;    // branch B [N, r] bf16, box r x bn rows
   CUtensorMap y;    // output y [M, N] bf16, box 64 x 32 rows, 128B swizzle (bf16 epilogue)
-  CUtensorMap sfa;  // A scales viewed as u8 [atoms * 2, 256], box 256 x 4 (one stage, 1 KB)
+  CUtensorMap sfa;  // A scales viewed as u8 [rows * K / 16 / 256, 256], box 256 x 16 (eight K64 steps, 4 KB)
   CUtensorMap sfb;  // B scales, same view
 };
 
-cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int bn, GemmEpilogue epi, cudaStream_t st);
-size_t gemm_smem_bytes(int bn);
+// Tile width and K per pipeline stage for an M x N output.
+struct GemmShape {
+  int bn, ks;
+};
+GemmShape gemm_shape(int M, int N);
+
+// p.k_stages must be ceil(K / shape.ks); split-K (p.splits in {2, 4, 8}) needs
+// the SplitK epilogue and launches one cluster of p.splits CTAs per tile.
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
+                        cudaStream_t st);
 
 }  // namespace qwam

@@ -31,7 +31,7 @@ def tiled(S, rows_pad):
 
 @pytest.mark.parametrize("M,N,K", [
     (128, 128, 128), (128, 256, 256), (256, 384, 1024), (200, 144, 384),
-    (1, 16, 128), (64, 256, 3072), (130, 272, 640)])
+    (1, 16, 128), (64, 256, 3072), (130, 272, 640), (300, 512, 2176), (129, 128, 1408)])
 def test_fp4_gemm_matches_f64(M, N, K):
     import torch
     from bit_w4a4_quantised_b200 import binding as qw

@@ -27,6 +27,10 @@ CASES = {
     "m129_k768_n512_r32_b32": lambda: workloads.custom(129, 768, 512, 32, 32, seed=15, n_outliers=6),
     "m384_k1024_n768_r32_b128": lambda: workloads.custom(384, 1024, 768, 32, 128, seed=16, n_outliers=10),
     "m64_k4096_n1024_r32_b128": lambda: workloads.custom(64, 4096, 1024, 32, 128, seed=17, n_outliers=40),
+    # split-K with several scale-ring slots per split, the last one partial
+    "m48_k6144_n128_r32_b128": lambda: workloads.custom(48, 6144, 128, 32, 128, seed=18, n_outliers=60),
+    # persistent tiles with a partial last 256-K stage
+    "m260_k1408_n640_r16_b64": lambda: workloads.custom(260, 1408, 640, 16, 64, seed=19, n_outliers=14),
 }
 
 
