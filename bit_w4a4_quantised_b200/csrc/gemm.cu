@@ -373,17 +373,18 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     const float gs = __fmul_rn(p.g_a_ptr ? *p.g_a_ptr : p.g_a, p.g_b);
     const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
     uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
-    int tl = 0, q = 0;
+    // Scale blocks: smem ring -> TMEM ring.  A warp's tcgen05.cp instructions run
+    // one after another (~115 cycles each), so a slot's copies are spread over
+    // the eight epilogue warps, which are otherwise idle while a tile
+    // accumulates.  The first two slots of the next tile are copied as soon as
+    // this tile's accumulator is drained (both TMEM scale slots are free then),
+    // before this tile's stores, so the next tile's MMAs need not wait for them.
     bool sf_ok = true;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
-      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
-      const Range rg = range_of(tc.split);
-      // Scale blocks of this tile: smem ring -> TMEM ring.  A warp's tcgen05.cp
-      // instructions run one after another (~115 cycles each), so a slot's
-      // copies are spread over the eight epilogue warps, which are otherwise
-      // idle while the tile accumulates.
-      for (int j = 0; j < rg.nsf; ++j, ++q) {
-        const int s = q & 1;
+    int q_next = 0, t_cp = blockIdx.x, j_cp = 0;  // next scale slot to copy: global index, tile, slot in tile
+    auto cp_upto = [&](int q_end) {
+      while (q_next < q_end && t_cp < n_tiles) {
+        const Range rc = range_of(tile_coord(t_cp, tiles_m, tiles_n, BN, p.splits).split);
+        const int q = q_next, j = j_cp, s = q & 1;
         int wok = 1;
         if (lane == 0)
           wok = (sf_ok && mbar_wait(&sf_full[s], (q >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT) &&
@@ -393,11 +394,9 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         wok = __shfl_sync(0xffffffffu, wok, 0);
         if (!wok) {
           sf_ok = false;
-          continue;
-        }
-        if (lane == 0) {
+        } else if (lane == 0) {
           tc_fence_after();
-          const int nk = min(kSFK, rg.n_k64 - j * kSFK);
+          const int nk = min(kSFK, rc.n_k64 - j * kSFK);
           const uint32_t src = smem_u32(smem + C::OFF_SF + s * C::SF_SLOT);
           const uint32_t col0 = BN + s * C::SF_COLS;
           for (int c = ew; c < kSFK * (1 + C::NSFB); c += kEpiWarps) {
@@ -409,7 +408,18 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
           tc_commit(&sf_ready[s]);
         }
         __syncwarp();
+        ++q_next;
+        if (++j_cp == rc.nsf) {
+          j_cp = 0;
+          t_cp += gridDim.x;
+        }
       }
+    };
+    int tl = 0, q_tile = 0;  // first scale slot of the current tile
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
+      const Range rg = range_of(tc.split);
+      cp_upto(q_tile + rg.nsf);
       const bool ok = sf_ok && mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT);
       __syncwarp();
       tc_fence_after();
@@ -439,6 +449,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
+        cp_upto(q_tile + rg.nsf + 2);
         if (ok) {
           // stage 64 columns (32 rows x 128 B, 128B swizzle) per TMA store
 #pragma unroll
@@ -479,6 +490,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
+        cp_upto(q_tile + rg.nsf + 2);
       } else {
         // Split-K: this tile's MMAs are done (acc_full), so this CTA's operand
         // ring is idle.  Push accumulator rows to their owner's ring, laid out
@@ -507,6 +519,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
+        cp_upto(q_tile + rg.nsf + 2);
         cluster_arrive();  // P
         cluster_wait();
         uint16_t* y = static_cast<uint16_t*>(p.y);
@@ -535,6 +548,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
                          pack_bf16x2(__fmaf_rn(sacc.z, gs, b4[2]), __fmaf_rn(sacc.w, gs, b4[3])));
         }
       }
+      q_tile += rg.nsf;
     }
     if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
       if (lane == 0) bulk_wait<0>();
