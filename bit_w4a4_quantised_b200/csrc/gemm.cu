@@ -154,8 +154,13 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the next kernel in the stream may start its own set-up now
+  griddep_launch_dependents();
   // Split-K cluster barriers: A0 (every split CTA runs), R (every split's MMAs
   // are done, so its operand ring may take remote stores), P (all rows pushed).
+  // Up to 64 rows the pushed rows fit in the epilogue staging area, which the
+  // split-K epilogue does not otherwise use, and R is not needed.
+  const bool rx_stg = p.M <= 64 && kBM / 2 * BN * 4 <= kEpiWarps * C::STG_BYTES;
   if constexpr (kClusterK) cluster_arrive();  // A0
 
   // A split's K range: stages [s_begin, s_begin + n_st) (balanced: every split
@@ -245,9 +250,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     }
     __syncwarp();
     if constexpr (kClusterK) {
-      cluster_wait();    // A0
-      cluster_arrive();  // R
-      cluster_wait();
+      cluster_wait();  // A0
+      if (!rx_stg) {
+        cluster_arrive();  // R
+        cluster_wait();
+      }
       cluster_arrive();  // P
       cluster_wait();
     }
@@ -286,9 +293,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     }
     __syncwarp();
     if constexpr (kClusterK) {
-      cluster_wait();    // A0
-      cluster_arrive();  // R
-      cluster_wait();
+      cluster_wait();  // A0
+      if (!rx_stg) {
+        cluster_arrive();  // R
+        cluster_wait();
+      }
       cluster_arrive();  // P
       cluster_wait();
     }
@@ -356,9 +365,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     }
     __syncwarp();
     if constexpr (kClusterK) {
-      cluster_wait();    // A0
-      cluster_arrive();  // R
-      cluster_wait();
+      cluster_wait();  // A0
+      if (!rx_stg) {
+        cluster_arrive();  // R
+        cluster_wait();
+      }
       cluster_arrive();  // P
       cluster_wait();
     }
@@ -495,20 +506,22 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         // Split-K: this tile's MMAs are done (acc_full), so this CTA's operand
         // ring is idle.  Push accumulator rows to their owner's ring, laid out
         // [split][row in slice][BN]; the owner sums them in split order.
-        const int SLR = kBM / p.splits;  // rows per owner
-        float* ring = reinterpret_cast<float*>(smem + C::OFF_A);
-        cluster_wait();    // A0
-        cluster_arrive();  // R
-        cluster_wait();
+        const int SLR = (rx_stg ? kBM / 2 : kBM) / p.splits;  // rows per owner
+        float* ring = reinterpret_cast<float*>(smem + (rx_stg ? C::OFF_STG : C::OFF_A));
+        cluster_wait();  // A0
+        if (!rx_stg) {
+          cluster_arrive();  // R
+          cluster_wait();
+        }
         const int rloc = qd * 32 + lane;
         const uint32_t dst = dsmem_addr(smem_u32(ring + (tc.split * SLR + rloc % SLR) * BN + half * HC),
-                                        static_cast<uint32_t>(rloc / SLR));
+                                        static_cast<uint32_t>(min(rloc / SLR, p.splits - 1)));
 #pragma unroll 1
         for (int qq = 0; qq < HC / 32; ++qq) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + qq * 32, r);
           tmem_ld_wait();
-          if (ok && row < p.M) {
+          if (ok && row < p.M) {  // rows >= M are not pushed (rx_stg: M <= 64 rows)
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               dsmem_st_f4(dst + static_cast<uint32_t>((qq * 32 + 4 * k) * 4),

@@ -63,7 +63,7 @@ struct PCfg {
   static constexpr bool kProj = R > 0 && MODE != 2;   // this launch computes c
   static constexpr bool kNeedA = kProj;               // cluster exchange of partial c
   static constexpr bool kNeedB = MODE == 0;           // cluster exchange of amax
-  static constexpr bool kCluster = kNeedA || kNeedB;  // smem read by peers: final barrier
+  static constexpr bool kCluster = kNeedA || kNeedB;  // a cluster launch (peers store into this smem)
   static constexpr bool kSmall = W == 32;
   static constexpr int UC = R > 0 ? R / 2 : 1;        // c columns per row thread (two per row)
   static constexpr int X_BYTES = kRows * kChunk * 2;  // two 64-column SW128 boxes
@@ -330,7 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = C::kMMA ? *tmem_slot : 0u;
   // Cluster barriers, in order: A0 (every CTA of the cluster is running, so its
   // shared memory may take remote stores), A1 / A2 (partial c scattered / summed
-  // c gathered), B (CTA amax published; Fused), C (no more remote access: exit).
+  // c gathered), B (CTA amax published; Fused).  Every remote store precedes its
+  // writer's arrival at the last of these, so once a CTA has passed that
+  // barrier no peer touches its shared memory again and it may exit.
   if constexpr (C::kCluster) cluster_arrive();  // A0
   // the GEMM that consumes this launch's output may start its weight loads now
   griddep_launch_dependents();
@@ -349,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int last = -1;
     bool ok = true;
+    bool dep_done = false;  // griddep_wait() done: T may be read
     auto issue = [&](int i) {
       const int slot = i & 1;
       if (slot != my_slot || !ok) return;
@@ -377,7 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pp = lane - 6;
         m = pp ? &maps.v_lo : &maps.v_hi; dst = s + C::OFF_V + pp * 256 * R; x = 0; y = col;
       }
-      if (m) tma_load_2d(dst, m, &full[slot], x, y);
+      // This warp's first load: the layer constants (P, V, chan) go out while the
+      // previous kernel in the stream may still run; T only after it finished.
+      if (m && (dep_done || lane >= 2)) tma_load_2d(dst, m, &full[slot], x, y);
+      if (!dep_done) {
+        griddep_wait();
+        dep_done = true;
+        if (m && lane < 2) tma_load_2d(dst, m, &full[slot], x, y);
+      }
       if (lane == 0 && (kind & LD_CH)) bulk_load(s + C::OFF_CH, p.chan + col, C::CH_BYTES, &full[slot]);
       last = i;
     };
@@ -415,11 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     if (lane == 0 && last >= 0) mbar_wait(&full[last & 1], (last >> 1) & 1, p.err, DEVERR_DRAIN_WAIT);
     __syncwarp();
-    if constexpr (C::kCluster) {
-      cluster_wait();  // the last barrier arrived at (B, else A2)
-      cluster_arrive();  // C
-      cluster_wait();
-    }
+    if constexpr (C::kCluster) cluster_wait();  // the last barrier arrived at (B, else A2)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if constexpr (C::kMMA) {
@@ -507,13 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         cluster_arrive();  // B
       }
     }
-    if constexpr (C::kCluster) {
-      cluster_wait();    // the last barrier arrived at (B, else A2)
-      cluster_arrive();  // C
-      cluster_wait();
-    }
+    if constexpr (C::kCluster) cluster_wait();  // the last barrier arrived at (B, else A2)
   } else {
     // ------------------------------------------------------------ row threads
+    // outputs (and the workspace they live in) may still be read by the
+    // previous kernel in the stream until it has finished
+    griddep_wait();
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int hf = warp >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
@@ -727,10 +732,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (MODE == 2) {
       if (part == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = g;
     }
-    if constexpr (C::kCluster) {
-      cluster_arrive();
-      cluster_wait();
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -755,15 +756,17 @@ cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p, cudaStream_
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (C::kCluster) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.parts;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = p.parts;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
   return cudaLaunchKernelEx(&cfg, kern, maps, p);
 }
