@@ -89,11 +89,13 @@ qwam_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
 }
 
 // Scale buffer of `rows_padded` rows (multiple of 128) and K columns in the tiled
-// layout, viewed as u8 [rows_padded * K / 16 / 256, 256]: one slot of the GEMM's
-// scale ring (eight 512-byte atoms = eight K64 steps of 128 rows) is a 256 x 16 box.
-qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, int K) {
+// layout, viewed as u8 [rows_padded * K / 16 / 256, 256]: a 512-byte atom (one
+// K64 step of 128 rows) is two rows, so one GEMM stage of ks K elements of one
+// 128-row block is a 256 x (ks / 32) box.
+qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, int K, int ks) {
   const uint64_t total = static_cast<uint64_t>(rows_padded) * K / 16;
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, total / 256, 256, 256, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, total / 256, 256, 256, static_cast<uint32_t>(ks / 32),
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // Packed E2M1 operand [rows, K/2] u8 as the GEMM reads it: one box per stage of
@@ -213,7 +215,7 @@ struct qwam_layer {
   uint16_t* bias;
   float g_w;
   size_t sf_bytes;
-  CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256, map_sfb;
+  CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256, map_sfb_k128, map_sfb_k256;
   ProMaps vmaps;  // P^T and V (hi/lo) tensor maps for the prologue; x is per call
 };
 
@@ -377,7 +379,9 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
       (s_ = make_codes_map(&h->map_b128_k256, h->codes, N, K, 256, 128)) != QWAM_OK ||
       (s_ = make_codes_map(&h->map_b256_k256, h->codes, N, K, 256, 256)) != QWAM_OK)
     return cleanup(s_);
-  if ((s_ = make_sf_map(&h->map_sfb, h->sf, round_up(static_cast<size_t>(N), 256), K)) != QWAM_OK) return cleanup(s_);
+  if ((s_ = make_sf_map(&h->map_sfb_k128, h->sf, round_up(static_cast<size_t>(N), 256), K, 128)) != QWAM_OK ||
+      (s_ = make_sf_map(&h->map_sfb_k256, h->sf, round_up(static_cast<size_t>(N), 256), K, 256)) != QWAM_OK)
+    return cleanup(s_);
   if (r > 0) {
     if ((s_ = make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r))) !=
             QWAM_OK ||
@@ -442,8 +446,8 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, a->base + lay.codes, M, h->K, pl.ks, 128));
   maps.b = pl.bn == 256 ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
-  QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K));
-  maps.sfb = h->map_sfb;
+  QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks));
+  maps.sfb = pl.ks == 256 ? h->map_sfb_k256 : h->map_sfb_k128;
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
@@ -554,8 +558,8 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, base + lay.codes, M, h->K, pl.ks, 128));
   maps.b = pl.bn == 256 ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
-  QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K));
-  maps.sfb = h->map_sfb;
+  QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks));
+  maps.sfb = pl.ks == 256 ? h->map_sfb_k256 : h->map_sfb_k128;
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
@@ -719,8 +723,8 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   maps.u = maps.a;
   maps.l = maps.b;
   maps.y = maps.a;
-  QW_TRY(make_sf_map(&maps.sfa, a_scales, round_up(static_cast<size_t>(M), 128), K));
-  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), sh.bn), K));
+  QW_TRY(make_sf_map(&maps.sfa, a_scales, round_up(static_cast<size_t>(M), 128), K, sh.ks));
+  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), sh.bn), K, sh.ks));
   GemmParams p{};
   p.M = M; p.N = N; p.K = K;
   p.k_stages = (K + sh.ks - 1) / sh.ks;

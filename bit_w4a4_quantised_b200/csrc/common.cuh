@@ -25,6 +25,7 @@ enum : uint32_t {
   DEVERR_EPILOGUE_WAIT = 1u << 2,
   DEVERR_DRAIN_WAIT = 1u << 3,
   DEVERR_BRANCH_WAIT = 1u << 4,
+  DEVERR_SCALE_WAIT = 1u << 5,
 };
 
 // A bounded wait gives up after this long (device global timer, nanoseconds).

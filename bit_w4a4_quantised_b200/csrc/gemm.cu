@@ -14,22 +14,23 @@
 //
 // Persistent kernel, one CTA per SM, tiles of 128 x BN, K in stages of KS
 // elements (KS / 2 bytes of packed E2M1 per row: one 128B- or 64B-swizzle
-// atom), K64 per MMA.  On this part the TMA engine costs a roughly fixed time
-// per box, so the operands come in few, large boxes: one A and one B box per
-// stage, and the E4M3 scale blocks on a ring of their own, eight K64 steps
-// (4 KB per 128 rows) per box.  Roles:
-//   producer warps  one per operand ring slot (a TMA instruction holds its warp
-//                   for a fixed ~600 cycles); the first stage's weight box goes
+// atom), K64 per MMA.  A stage is one box each of A, B, the A scale blocks and
+// each 128-row block of B scales, all issued by different lanes of one
+// instruction: on this part a lane's TMA boxes run one after another at a
+// roughly fixed cost per box, while boxes from different lanes overlap.
+// Roles:
+//   producer warps  one per ring slot (a TMA instruction holds its warp for
+//                   several hundred cycles); the first stage's weight boxes go
 //                   out before the wait on the kernel that writes A.
-//   scale warp      loads the scale ring.
 //   MMA warp        owns TMEM; issues only tcgen05.mma (bf16 branch, then FP4).
-//   epilogue warps  eight, two per TMEM lane quarter (column halves).  While a
-//                   tile accumulates they copy the scale blocks into a TMEM
-//                   scale ring (tcgen05.cp; a warp's copies run one after
-//                   another, so eight warps share them).  Then they drain the
-//                   accumulator to registers, release it to the next tile, add
-//                   bias, round to bf16, stage through 128B-swizzled smem and
-//                   store with TMA (ragged M / N are clipped by the tensor map).
+//   copy warps      four; move each stage's scale blocks from shared memory
+//                   into a four-slot TMEM scale ring (tcgen05.cp; one warp's
+//                   copies run one after another, so four warps share them).
+//   epilogue warps  eight, two per TMEM lane quarter (column halves).  Stage
+//                   the tile's bias in shared memory, drain the accumulator
+//                   to registers, release it to the next tile, round to bf16,
+//                   stage through 128B-swizzled smem and store with TMA
+//                   (ragged M / N are clipped by the tensor map).
 // Split-K (small M): the splits of an output tile form one cluster (split
 // fastest in the grid, one work item per CTA).  Once every split's MMAs are
 // done, each pushes its fp32 accumulator rows to the CTA that owns them (a
@@ -46,7 +47,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kEpiWarps = 8;
-constexpr int kSFK = 8;  // K64 steps per scale-ring slot
+constexpr int kCopyWarps = 4;
+constexpr int kScaleSlots = 4;  // TMEM scale ring, one stage per slot
 
 template <int BN, int KS>
 struct Cfg {
@@ -55,35 +57,40 @@ struct Cfg {
   static constexpr uint32_t SWZ = ROWB == 128 ? 2u : 4u;    // UMMA layout: 128B / 64B swizzle
   static constexpr int STAGES = KS == 256 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8);
   static constexpr int NSFB = BN / 128;                     // 128-row scale blocks of B
-  static constexpr int SF_ATOMS = kSFK * 512;               // one 128-row scale block of a slot
-  static constexpr int SF_SLOT = SF_ATOMS * (1 + NSFB);
-  static constexpr int SF_WARP = STAGES;
-  static constexpr int MMA_WARP = STAGES + 1;
-  static constexpr int EPI_WARP0 = STAGES + 2;
+  static constexpr int SF_BLK = K64 * 512;                  // one 128-row scale block of a stage
+  static constexpr int NBOX = 3 + NSFB;                     // boxes per stage: A, B, A scales, B scale blocks
+  static constexpr int MMA_WARP = STAGES;
+  static constexpr int CP_WARP0 = STAGES + 1;
+  static constexpr int EPI_WARP0 = CP_WARP0 + kCopyWarps;
   static constexpr int THREADS = 32 * (EPI_WARP0 + kEpiWarps);
   static constexpr int A_BYTES = kBM * ROWB;
   static constexpr int B_BYTES = BN * ROWB;
+  static constexpr int SF_BYTES = (1 + NSFB) * SF_BLK;
+  static constexpr int STAGE_TX = A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int U_BYTES = kBM * 64;
   static constexpr int L_BYTES = BN * 64;
   static constexpr int STG_BYTES = 4096;                    // per epilogue warp: 32 rows x 128 B
+  static constexpr int BIAS_BYTES = BN;                     // per epilogue warp: BN / 2 bf16
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_U = OFF_SF + 2 * SF_SLOT;
+  static constexpr int OFF_U = OFF_SF + STAGES * SF_BYTES;
   static constexpr int OFF_L = OFF_U + U_BYTES;
   static constexpr int OFF_STG = OFF_L + L_BYTES;
-  static constexpr int OFF_BAR = OFF_STG + kEpiWarps * STG_BYTES;
-  static constexpr int NBAR = 2 * STAGES + 6 + 4;
+  static constexpr int OFF_BIAS = OFF_STG + kEpiWarps * STG_BYTES;
+  static constexpr int OFF_BAR = OFF_BIAS + kEpiWarps * BIAS_BYTES;
+  static constexpr int NBAR = 2 * STAGES + 2 * kScaleSlots + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  // TMEM columns: accumulator [0, BN), then two scale slots, each kSFK K64
+  // TMEM columns: accumulator [0, BN), then kScaleSlots scale slots, each K64
   // steps of A (4 columns) then of B (BN / 32 columns).
-  static constexpr int SF_A_COLS = kSFK * 4;
-  static constexpr int SF_COLS = SF_A_COLS + kSFK * (BN / 32);
-  static constexpr int TMEM_USED = BN + 2 * SF_COLS;
+  static constexpr int SF_A_COLS = K64 * 4;
+  static constexpr int SF_COLS = SF_A_COLS + K64 * (BN / 32);
+  static constexpr int TMEM_USED = BN + kScaleSlots * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(NBOX <= 32, "one lane per box");
   static_assert(kBM * BN * 4 <= STAGES * (A_BYTES + B_BYTES), "split-K receive area fits in the operand ring");
 };
 
@@ -112,12 +119,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
   using C = Cfg<BN, KS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES] A/B landed
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES] operands and scales landed
   uint64_t* empty = full + C::STAGES;                               // [STAGES] MMAs done with the slot
-  uint64_t* sf_full = empty + C::STAGES;                            // [2] scale boxes landed
-  uint64_t* sf_ready = sf_full + 2;                                 // [2] scales copied to TMEM (smem free)
-  uint64_t* sf_tfree = sf_ready + 2;                                // [2] MMAs done with the TMEM scale slot
-  uint64_t* branch_full = sf_tfree + 2;
+  uint64_t* sf_ready = empty + C::STAGES;                           // [kScaleSlots] scales copied into TMEM
+  uint64_t* sf_tfree = sf_ready + kScaleSlots;                      // [kScaleSlots] MMAs done with the TMEM slot
+  uint64_t* branch_full = sf_tfree + kScaleSlots;
   uint64_t* branch_empty = branch_full + 1;
   uint64_t* acc_full = branch_empty + 1;
   uint64_t* acc_empty = acc_full + 1;
@@ -135,9 +141,8 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sf_full[i], 1);
-      mbar_init(&sf_ready[i], kEpiWarps);
+    for (int i = 0; i < kScaleSlots; ++i) {
+      mbar_init(&sf_ready[i], kCopyWarps);
       mbar_init(&sf_tfree[i], 1);
     }
     mbar_init(branch_full, 1);
@@ -162,12 +167,24 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
   // split-K epilogue does not otherwise use, and R is not needed.
   const bool rx_stg = p.M <= 64 && kBM / 2 * BN * 4 <= kEpiWarps * C::STG_BYTES;
   if constexpr (kClusterK) cluster_arrive();  // A0
+  // every role other than the epilogue ends with the same cluster barriers
+  auto cluster_tail = [&]() {
+    if constexpr (kClusterK) {
+      cluster_wait();  // A0
+      if (!rx_stg) {
+        cluster_arrive();  // R
+        cluster_wait();
+      }
+      cluster_arrive();  // P
+      cluster_wait();
+    }
+  };
 
   // A split's K range: stages [s_begin, s_begin + n_st) (balanced: every split
   // gets at least one stage when splits <= k_stages), K64 steps
-  // [k64_begin, k64_begin + n_k64), scale slots of kSFK steps.
+  // [k64_begin, k64_begin + n_k64).
   struct Range {
-    int s_begin, n_st, k64_begin, n_k64, nsf;
+    int s_begin, n_st, k64_begin, n_k64;
   };
   auto range_of = [&](int split) {
     Range r;
@@ -175,25 +192,33 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     r.n_st = (split + 1) * p.k_stages / p.splits - r.s_begin;
     r.k64_begin = r.s_begin * C::K64;
     r.n_k64 = min(r.n_st * C::K64, k64_total - r.k64_begin);
-    r.nsf = (r.n_k64 + kSFK - 1) / kSFK;
     return r;
   };
 
   if (warp < C::STAGES) {
-    // ------------------------------------------------ operand producers: warp st owns slot st
+    // ------------------------------------------------ producers: warp st owns ring slot st
     const int st = warp;
     if (lane == 0 && st == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
+      tma_prefetch_desc(&tmSA);
+      tma_prefetch_desc(&tmSB);
       if (p.has_branch) {
         tma_prefetch_desc(&tmU);
         tma_prefetch_desc(&tmL);
       }
     }
+    // this lane's box of a stage: 0 A, 1 B, 2 A scales, 3.. B scale blocks;
+    // weight boxes (B and its scales) do not depend on the kernel before this one
+    const bool weight_box = lane == 1 || lane >= 3;
+    const CUtensorMap* map = lane == 0 ? &tmA : (lane == 1 ? &tmB : (lane == 2 ? &tmSA : &tmSB));
+    uint8_t* const dst = smem + (lane == 0   ? C::OFF_A + st * C::A_BYTES
+                                 : lane == 1 ? C::OFF_B + st * C::B_BYTES
+                                             : C::OFF_SF + st * C::SF_BYTES + (lane - 2) * C::SF_BLK);
     int g = 0;  // stage counter of this CTA
     int last = -1, nbranch = 0;
     bool ok = true;
-    bool dep_done = false;  // griddep_wait() done: A and U may be read
+    bool dep_done = false;  // griddep_wait() done: A, its scales and U may be read
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
       const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
       const Range rg = range_of(tc.split);
@@ -225,20 +250,30 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
           ok = false;
           break;
         }
-        const int x = (rg.s_begin + i) * C::ROWB;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::A_BYTES + C::B_BYTES);
+        const int kst = rg.s_begin + i;
+        // operands: x = byte column, y = row; scales (u8 rows of 256 B, two per
+        // K64 step of a 128-row block): x = 0, y = 2 * (block * K/64 + step)
+        int cx = 0, cy;
+        if (lane < 2) {
+          cx = kst * C::ROWB;
+          cy = lane ? tc.n0 : tc.m0;
+        } else {
+          const int blk = lane == 2 ? tc.m0 / kBM : tc.n0 / 128 + (lane - 3);
+          cy = 2 * (blk * k64_total + kst * C::K64);
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::STAGE_TX);
         __syncwarp();
         if (dep_done) {
-          // one converged instruction: A on lane 0, B on lane 1
-          if (lane < 2)
-            tma_load_2d(smem + (lane ? C::OFF_B + st * C::B_BYTES : C::OFF_A + st * C::A_BYTES), lane ? &tmB : &tmA,
-                        &full[st], x, lane ? tc.n0 : tc.m0);
+          if (lane < C::NBOX) tma_load_2d(dst, map, &full[st], cx, cy);
         } else {
-          // the weights first, then A once the kernel writing it has finished
-          if (lane == 1) tma_load_2d(smem + C::OFF_B + st * C::B_BYTES, &tmB, &full[st], x, tc.n0);
+          // the weight boxes first, then A and its scales once the kernel
+          // writing them has finished
+          if (weight_box && lane < C::NBOX) tma_load_2d(dst, map, &full[st], cx, cy);
           griddep_wait();
           dep_done = true;
-          if (lane == 0) tma_load_2d(smem + C::OFF_A + st * C::A_BYTES, &tmA, &full[st], x, tc.m0);
+          if (!weight_box) {
+            if (lane < C::NBOX) tma_load_2d(dst, map, &full[st], cx, cy);
+          }
         }
         last = g;
       }
@@ -249,58 +284,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
       if (nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
     }
     __syncwarp();
-    if constexpr (kClusterK) {
-      cluster_wait();  // A0
-      if (!rx_stg) {
-        cluster_arrive();  // R
-        cluster_wait();
-      }
-      cluster_arrive();  // P
-      cluster_wait();
-    }
-  } else if (warp == C::SF_WARP) {
-    // ------------------------------------------------ scale producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmSA);
-      tma_prefetch_desc(&tmSB);
-      int q = 0, last = -1;
-      bool ok = true, dep_done = false;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
-        const Range rg = range_of(tc.split);
-        for (int j = 0; j < rg.nsf; ++j, ++q) {
-          const int s = q & 1;
-          if (q >= 2 && !mbar_wait(&sf_ready[s], ((q >> 1) & 1) ^ 1u, p.err, DEVERR_PRODUCER_WAIT)) {
-            ok = false;
-            break;
-          }
-          uint8_t* dst = smem + C::OFF_SF + s * C::SF_SLOT;
-          const int atom = rg.k64_begin + j * kSFK;  // first K64 step of the slot
-          mbar_arrive_expect_tx(&sf_full[s], C::SF_SLOT);
-#pragma unroll
-          for (int h = 0; h < C::NSFB; ++h)
-            tma_load_2d(dst + (1 + h) * C::SF_ATOMS, &tmSB, &sf_full[s], 0,
-                        2 * ((tc.n0 / 128 + h) * k64_total + atom));
-          if (!dep_done) {
-            griddep_wait();
-            dep_done = true;
-          }
-          tma_load_2d(dst, &tmSA, &sf_full[s], 0, 2 * ((tc.m0 / 128) * k64_total + atom));
-          last = q;
-        }
-      }
-      if (last >= 0) mbar_wait(&sf_full[last & 1], (last >> 1) & 1, p.err, DEVERR_DRAIN_WAIT);
-    }
-    __syncwarp();
-    if constexpr (kClusterK) {
-      cluster_wait();  // A0
-      if (!rx_stg) {
-        cluster_arrive();  // R
-        cluster_wait();
-      }
-      cluster_arrive();  // P
-      cluster_wait();
-    }
+    cluster_tail();
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -309,7 +293,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
       const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
       const uint32_t sbo = 8u * p.branch_k * 2u;
       const uint32_t us = smem_u32(smem + C::OFF_U), ls = smem_u32(smem + C::OFF_L);
-      int g = 0, q0 = 0, tl = 0, nbranch = 0;
+      int g = 0, tl = 0, nbranch = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tl) {
         const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
@@ -329,50 +313,65 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
           tc_commit(branch_empty);
           ++nbranch;
         }
-        int kloc = 0;  // K64 step within this split
-        for (int i = 0; ok && i < rg.n_st; ++i, ++g) {
-          const int st = g % C::STAGES;
-          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_MMA_WAIT)) {
+        for (int i = 0; i < rg.n_st; ++i, ++g) {
+          const int st = g % C::STAGES, sl = g % kScaleSlots;
+          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_MMA_WAIT) ||
+              !mbar_wait(&sf_ready[sl], (g / kScaleSlots) & 1, p.err, DEVERR_MMA_WAIT)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_s = smem_u32(smem + C::OFF_A + st * C::A_BYTES);
           const uint32_t b_s = smem_u32(smem + C::OFF_B + st * C::B_BYTES);
+          const uint32_t sfa = tmem + BN + sl * C::SF_COLS, sfb = sfa + C::SF_A_COLS;
           const int nk = min(C::K64, rg.n_k64 - i * C::K64);
-          for (int kk = 0; kk < nk; ++kk, ++kloc) {
-            const int cur = q0 + kloc / kSFK;  // scale slot of this step
-            const int ks = kloc % kSFK;
-            if (ks == 0) {
-              if (!mbar_wait(&sf_ready[cur & 1], (cur >> 1) & 1, p.err, DEVERR_MMA_WAIT)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            const uint32_t sf_col = BN + (cur & 1) * C::SF_COLS;
+          for (int kk = 0; kk < nk; ++kk) {
             mma_mxf4nvf4(tmem, smem_desc(a_s + kk * 32, 16, 8 * C::ROWB, C::SWZ),
-                         smem_desc(b_s + kk * 32, 16, 8 * C::ROWB, C::SWZ), idesc_fp4, tmem + sf_col + ks * 4,
-                         tmem + sf_col + C::SF_A_COLS + ks * (BN / 32), accum);
+                         smem_desc(b_s + kk * 32, 16, 8 * C::ROWB, C::SWZ), idesc_fp4, sfa + kk * 4,
+                         sfb + kk * (BN / 32), accum);
             accum = 1;
-            if (ks == kSFK - 1 || kloc == rg.n_k64 - 1) tc_commit(&sf_tfree[cur & 1]);
           }
           tc_commit(&empty[st]);
+          tc_commit(&sf_tfree[sl]);
         }
-        q0 += rg.nsf;
+        if (!ok) break;
         tc_commit(acc_full);
       }
     }
     __syncwarp();
-    if constexpr (kClusterK) {
-      cluster_wait();  // A0
-      if (!rx_stg) {
-        cluster_arrive();  // R
-        cluster_wait();
+    cluster_tail();
+  } else if (warp < C::EPI_WARP0) {
+    // ------------------------------------------------ scale copies: smem stage -> TMEM slot
+    const int cw = warp - C::CP_WARP0;
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        const Range rg = range_of(tile_coord(t, tiles_m, tiles_n, BN, p.splits).split);
+        for (int i = 0; i < rg.n_st; ++i, ++g) {
+          const int st = g % C::STAGES, sl = g % kScaleSlots;
+          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_SCALE_WAIT) ||
+              (g >= kScaleSlots &&
+               !mbar_wait(&sf_tfree[sl], ((g / kScaleSlots) & 1) ^ 1u, p.err, DEVERR_SCALE_WAIT))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(C::K64, rg.n_k64 - i * C::K64);
+          const uint32_t src = smem_u32(smem + C::OFF_SF + st * C::SF_BYTES);
+          const uint32_t col0 = BN + sl * C::SF_COLS;
+          for (int c = cw; c < C::K64 * (1 + C::NSFB); c += kCopyWarps) {
+            const int blk = c / C::K64, kk = c % C::K64;
+            if (kk >= nk) continue;
+            const uint32_t col = blk == 0 ? col0 + kk * 4 : col0 + C::SF_A_COLS + kk * (BN / 32) + (blk - 1) * 4;
+            tmem_cp_32x128b_x4(tmem + col, smem_desc(src + blk * C::SF_BLK + kk * 512, 0, 128, 0));
+          }
+          tc_commit(&sf_ready[sl]);
+        }
       }
-      cluster_arrive();  // P
-      cluster_wait();
     }
+    __syncwarp();
+    cluster_tail();
   } else {
     // ------------------------------------------------ epilogue
     const int ew = warp - C::EPI_WARP0;  // 0..7
@@ -384,58 +383,24 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     const float gs = __fmul_rn(p.g_a_ptr ? *p.g_a_ptr : p.g_a, p.g_b);
     const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
     uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
-    // Scale blocks: smem ring -> TMEM ring.  A warp's tcgen05.cp instructions run
-    // one after another (~115 cycles each), so a slot's copies are spread over
-    // the eight epilogue warps, which are otherwise idle while a tile
-    // accumulates.  The first two slots of the next tile are copied as soon as
-    // this tile's accumulator is drained (both TMEM scale slots are free then),
-    // before this tile's stores, so the next tile's MMAs need not wait for them.
-    bool sf_ok = true;
-    int q_next = 0, t_cp = blockIdx.x, j_cp = 0;  // next scale slot to copy: global index, tile, slot in tile
-    auto cp_upto = [&](int q_end) {
-      while (q_next < q_end && t_cp < n_tiles) {
-        const Range rc = range_of(tile_coord(t_cp, tiles_m, tiles_n, BN, p.splits).split);
-        const int q = q_next, j = j_cp, s = q & 1;
-        int wok = 1;
-        if (lane == 0)
-          wok = (sf_ok && mbar_wait(&sf_full[s], (q >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT) &&
-                 (q < 2 || mbar_wait(&sf_tfree[s], ((q >> 1) & 1) ^ 1u, p.err, DEVERR_EPILOGUE_WAIT)))
-                    ? 1
-                    : 0;
-        wok = __shfl_sync(0xffffffffu, wok, 0);
-        if (!wok) {
-          sf_ok = false;
-        } else if (lane == 0) {
-          tc_fence_after();
-          const int nk = min(kSFK, rc.n_k64 - j * kSFK);
-          const uint32_t src = smem_u32(smem + C::OFF_SF + s * C::SF_SLOT);
-          const uint32_t col0 = BN + s * C::SF_COLS;
-          for (int c = ew; c < kSFK * (1 + C::NSFB); c += kEpiWarps) {
-            const int blk = c / kSFK, kk = c % kSFK;
-            if (kk >= nk) continue;
-            const uint32_t col = blk == 0 ? col0 + kk * 4 : col0 + C::SF_A_COLS + kk * (BN / 32) + (blk - 1) * 4;
-            tmem_cp_32x128b_x4(tmem + col, smem_desc(src + blk * C::SF_ATOMS + kk * 512, 0, 128, 0));
-          }
-          tc_commit(&sf_ready[s]);
-        }
-        __syncwarp();
-        ++q_next;
-        if (++j_cp == rc.nsf) {
-          j_cp = 0;
-          t_cp += gridDim.x;
-        }
-      }
-    };
-    int tl = 0, q_tile = 0;  // first scale slot of the current tile
+    uint4* bias_s = reinterpret_cast<uint4*>(smem + C::OFF_BIAS + ew * C::BIAS_BYTES);  // this warp's HC bf16
+    int tl = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
       const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
-      const Range rg = range_of(tc.split);
-      cp_upto(q_tile + rg.nsf);
-      const bool ok = sf_ok && mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT);
-      __syncwarp();
-      tc_fence_after();
       const int row = tc.m0 + qd * 32 + lane;
       const int c0 = tc.n0 + half * HC;
+      if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
+        // this warp's bias columns, fetched while the tile accumulates
+        if (lane < HC / 8) {
+          uint4 braw = make_uint4(0u, 0u, 0u, 0u);
+          if (bias && c0 + 8 * lane < p.N) braw = __ldg(reinterpret_cast<const uint4*>(bias + c0 + 8 * lane));
+          bias_s[lane] = braw;
+        }
+        __syncwarp();
+      }
+      const bool ok = mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      __syncwarp();
+      tc_fence_after();
       if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
         // drain: fp32 accumulator -> bf16 pairs in registers, then release
         uint32_t packed[HC / 2];
@@ -446,9 +411,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            uint4 braw = make_uint4(0u, 0u, 0u, 0u);
-            if (bias && c0 + qq * 32 + 8 * j < p.N)
-              braw = __ldg(reinterpret_cast<const uint4*>(bias + c0 + qq * 32 + 8 * j));
+            const uint4 braw = bias_s[qq * 4 + j];
             const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -460,7 +423,6 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
-        cp_upto(q_tile + rg.nsf + 2);
         if (ok) {
           // stage 64 columns (32 rows x 128 B, 128B swizzle) per TMA store
 #pragma unroll
@@ -501,7 +463,6 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
-        cp_upto(q_tile + rg.nsf + 2);
       } else {
         // Split-K: this tile's MMAs are done (acc_full), so this CTA's operand
         // ring is idle.  Push accumulator rows to their owner's ring, laid out
@@ -532,7 +493,6 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
-        cp_upto(q_tile + rg.nsf + 2);
         cluster_arrive();  // P
         cluster_wait();
         uint16_t* y = static_cast<uint16_t*>(p.y);
@@ -561,7 +521,6 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
                          pack_bf16x2(__fmaf_rn(sacc.z, gs, b4[2]), __fmaf_rn(sacc.w, gs, b4[3])));
         }
       }
-      q_tile += rg.nsf;
     }
     if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
       if (lane == 0) bulk_wait<0>();
@@ -575,7 +534,6 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
-
 template <int BN, int KS, int EPI>
 cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   using C = Cfg<BN, KS>;

@@ -84,8 +84,8 @@ struct GemmMaps {
   CUtensorMap u;    // branch A [M, r] bf16, box r x 128 rows
   CUtensorMap l;    // branch B [N, r] bf16, box r x bn rows
   CUtensorMap y;    // output y [M, N] bf16, box 64 x 32 rows, 128B swizzle (bf16 epilogue)
-  CUtensorMap sfa;  // A scales viewed as u8 [rows * K / 16 / 256, 256], box 256 x 16 (eight K64 steps, 4 KB)
-  CUtensorMap sfb;  // B scales, same view
+  CUtensorMap sfa;  // A scales viewed as u8 [rows * K / 16 / 256, 256], box 256 x (ks / 32): one stage of 128 rows
+  CUtensorMap sfb;  // B scales, same view and box
 };
 
 // Tile width and K per pipeline stage for an M x N output.
