@@ -110,11 +110,12 @@ CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZL
 // ---- GEMM launch plan ------------------------------------------------------
 struct Plan {
   int bn, ks, k_stages, splits;
+  bool pair;  // 256 x bn tiles on CTA pairs (no split-K)
 };
 
 // Split-K when the output tiles leave SMs idle: the largest power of two <= 8
 // (one portable cluster per tile) with splits <= k_stages and tiles * splits
-// within one wave of the SMs.
+// within one wave of the SMs.  Otherwise 256-column tiles run on CTA pairs.
 Plan plan_gemm(int M, int N, int K) {
   Plan p{};
   const GemmShape sh = gemm_shape(M, N);
@@ -129,6 +130,7 @@ Plan plan_gemm(int M, int N, int K) {
       p.splits = c;
       break;
     }
+  p.pair = sh.pair && p.splits == 1;
   return p;
 }
 
@@ -445,19 +447,19 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   QW_TRY(arena_get(h->dev, lay.total, &a));
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, a->base + lay.codes, M, h->K, pl.ks, 128));
-  maps.b = pl.bn == 256 ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
+  maps.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
   QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks));
   maps.sfb = pl.ks == 256 ? h->map_sfb_k256 : h->map_sfb_k128;
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
-    maps.l = pl.bn == 256 ? h->map_l256 : h->map_l128;
+    maps.l = pl.bn == 256 && !pl.pair ? h->map_l256 : h->map_l128;
   } else {
     maps.u = maps.a;
     maps.l = maps.b;
   }
   if (pl.splits == 1)
-    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 32,
+    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B));
   else
     maps.y = maps.a;
@@ -474,7 +476,7 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   p.bias = h->bias;
   p.y = y;
   p.err = arena_err(*a);
-  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
+  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks, pl.pair}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
                       st));
   return QWAM_OK;
 }
@@ -557,19 +559,19 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
 
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, base + lay.codes, M, h->K, pl.ks, 128));
-  maps.b = pl.bn == 256 ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
+  maps.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
   QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks));
   maps.sfb = pl.ks == 256 ? h->map_sfb_k256 : h->map_sfb_k128;
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
-    maps.l = pl.bn == 256 ? h->map_l256 : h->map_l128;
+    maps.l = pl.bn == 256 && !pl.pair ? h->map_l256 : h->map_l128;
   } else {
     maps.u = maps.a;
     maps.l = maps.b;
   }
   if (pl.splits == 1)
-    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 32,
+    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B));
   else
     maps.y = maps.a;
@@ -586,7 +588,7 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   p.bias = h->bias;
   p.y = y;
   p.err = err;
-  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
+  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks, pl.pair}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
                       st));
   return QWAM_OK;
 }
@@ -719,7 +721,7 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   const GemmShape sh = gemm_shape(M, N);
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, a_codes, M, K, sh.ks, 128));
-  QW_TRY(make_codes_map(&maps.b, b_codes, N, K, sh.ks, sh.bn));
+  QW_TRY(make_codes_map(&maps.b, b_codes, N, K, sh.ks, sh.pair ? sh.bn / 2 : sh.bn));
   maps.u = maps.a;
   maps.l = maps.b;
   maps.y = maps.a;

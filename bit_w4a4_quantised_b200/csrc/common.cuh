@@ -88,6 +88,33 @@ __device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return f2_from(d);
 }
+// a * b + c per lane with one rounding (bit-identical to __fmaf_rn)
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_from(d);
+}
+// bf16(x0 * g + b0) | bf16(x1 * g + b1) << 16 with the bias pair given as bf16
+// bits (b0 in bits 0..15): one packed fp32 FMA (each lane bit-identical to
+// __fmaf_rn) and one packed round-to-nearest-even conversion.
+__device__ __forceinline__ uint32_t fma_bf16x2(float x0, float x1, float g, uint32_t b01) {
+  uint32_t d;
+  asm("{\n\t.reg .b64 xa, ga, ba, da;\n\t.reg .b32 b0, b1;\n\t.reg .f32 lo, hi;\n\t"
+      "shl.b32 b0, %4, 16;\n\tand.b32 b1, %4, 0xffff0000;\n\t"
+      "mov.b64 xa, {%1, %2};\n\tmov.b64 ga, {%3, %3};\n\tmov.b64 ba, {b0, b1};\n\t"
+      "fma.rn.f32x2 da, xa, ga, ba;\n\tmov.b64 {lo, hi}, da;\n\t"
+      "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+      : "=r"(d)
+      : "f"(x0), "f"(x1), "f"(g), "r"(b01));
+  return d;
+}
+// Two fp32 -> bf16 (round to nearest even, as __float2bfloat16_rn) packed in one
+// word: lo in bits 0..15, hi in bits 16..31.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
 
 // ---------------------------------------------------------------------------
 // mbarrier
@@ -332,6 +359,66 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[
                : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// CTA-pair (cta_group::2) forms.  One MMA instruction, issued by the even CTA
+// of a two-CTA cluster, computes a 256-row tile: A rows and B rows are split
+// across the two CTAs' shared memory and each CTA's TMEM holds its own 128
+// accumulator rows.  Barrier operands are cluster shared addresses (dsmem_addr).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive once on the mbarrier at cluster address `bar` (either CTA of the pair)
+// when every pair-wide tcgen05 operation issued so far by this thread is done.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Scale blocks from each CTA's shared memory into its own TMEM (same offsets in
+// both CTAs), issued once by the even CTA for the pair.
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// TMA load into this CTA's shared memory whose bytes are counted on an mbarrier
+// of the pair's even CTA (cluster shared address `bar`).  Not a multicast load.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+// Arrive on an mbarrier of either CTA of the cluster (cluster shared address).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
 
 }  // namespace qwam

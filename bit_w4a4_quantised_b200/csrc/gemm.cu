@@ -50,25 +50,30 @@ constexpr int kEpiWarps = 8;
 constexpr int kCopyWarps = 4;
 constexpr int kScaleSlots = 4;  // TMEM scale ring, one stage per slot
 
-template <int BN, int KS>
+template <int BN, int KS, bool PAIR = false>
 struct Cfg {
+  static constexpr int TM = PAIR ? 2 * kBM : kBM;          // rows of an output tile
+  static constexpr int HB = PAIR ? BN / 2 : BN;             // B (and L) rows held by one CTA
   static constexpr int ROWB = KS / 2;                       // operand bytes per row per stage
   static constexpr int K64 = KS / 64;                       // MMAs per stage
   static constexpr uint32_t SWZ = ROWB == 128 ? 2u : 4u;    // UMMA layout: 128B / 64B swizzle
-  static constexpr int STAGES = KS == 256 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8);
+  static constexpr int STAGES = PAIR ? 4 : (KS == 256 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
   static constexpr int NSFB = BN / 128;                     // 128-row scale blocks of B
   static constexpr int SF_BLK = K64 * 512;                  // one 128-row scale block of a stage
   static constexpr int NBOX = 3 + NSFB;                     // boxes per stage: A, B, A scales, B scale blocks
-  static constexpr int MMA_WARP = STAGES;
-  static constexpr int CP_WARP0 = STAGES + 1;
+  // producer warps, taking stages in turn (three keep the CTA at 16 warps, so
+  // the epilogue keeps 128 registers)
+  static constexpr int NPROD = STAGES < 3 ? STAGES : 3;
+  static constexpr int MMA_WARP = NPROD;
+  static constexpr int CP_WARP0 = NPROD + 1;
   static constexpr int EPI_WARP0 = CP_WARP0 + kCopyWarps;
   static constexpr int THREADS = 32 * (EPI_WARP0 + kEpiWarps);
   static constexpr int A_BYTES = kBM * ROWB;
-  static constexpr int B_BYTES = BN * ROWB;
+  static constexpr int B_BYTES = HB * ROWB;
   static constexpr int SF_BYTES = (1 + NSFB) * SF_BLK;
   static constexpr int STAGE_TX = A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int U_BYTES = kBM * 64;
-  static constexpr int L_BYTES = BN * 64;
+  static constexpr int L_BYTES = HB * 64;
   static constexpr int STG_BYTES = 4096;                    // per epilogue warp: 32 rows x 128 B
   static constexpr int BIAS_BYTES = BN;                     // per epilogue warp: BN / 2 bf16
   static constexpr int OFF_A = 0;
@@ -91,7 +96,7 @@ struct Cfg {
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(NBOX <= 32, "one lane per box");
-  static_assert(kBM * BN * 4 <= STAGES * (A_BYTES + B_BYTES), "split-K receive area fits in the operand ring");
+  static_assert(PAIR || kBM * BN * 4 <= STAGES * (A_BYTES + B_BYTES), "split-K receive area fits in the operand ring");
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -104,19 +109,20 @@ struct TileCoord {
 
 // Tiles run M-fastest so consecutive CTAs reuse the same weight tile from L2;
 // with split-K the split index is fastest (a tile's splits are one cluster).
-__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int bn, int splits) {
+// m0 is the first row of the tile (tm rows).
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n, int tm, int bn, int splits) {
   const int sp = t % splits;
   const int rest = t / splits;
-  return {(rest % tiles_m) * kBM, (rest / tiles_m % tiles_n) * bn, sp};
+  return {(rest % tiles_m) * tm, (rest / tiles_m % tiles_n) * bn, sp};
 }
 
-template <int BN, int KS, int EPI>
-__global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
+template <int BN, int KS, int EPI, bool PAIR>
+__global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmSA,
                     const __grid_constant__ CUtensorMap tmSB, const GemmParams p) {
-  using C = Cfg<BN, KS>;
+  using C = Cfg<BN, KS, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES] operands and scales landed
@@ -131,10 +137,37 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
   constexpr bool kClusterK = EPI == static_cast<int>(GemmEpilogue::SplitK);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_m = (p.M + kBM - 1) / kBM;
+  const int tiles_m = (p.M + C::TM - 1) / C::TM;
   const int tiles_n = (p.N + BN - 1) / BN;
   const int n_tiles = tiles_m * tiles_n * p.splits;
   const int k64_total = p.K / 64;
+  // CTA pair: rank 0 issues the MMAs and the scale copies for both CTAs; each
+  // CTA loads its own 128 rows of A and its half of the B rows, and every load
+  // of either CTA counts its bytes on rank 0's barrier.
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  auto coord = [&](int t) {
+    TileCoord tc = tile_coord(t, tiles_m, tiles_n, C::TM, BN, p.splits);
+    tc.m0 += static_cast<int>(rank) * kBM;  // this CTA's rows
+    return tc;
+  };
+  // barrier addresses as the pair-wide forms take them
+  auto lead = [&](uint64_t* b) { return PAIR ? dsmem_addr(smem_u32(b), 0u) : smem_u32(b); };
+  // tcgen05 commits: to rank 0 only, or to the same barrier in both CTAs
+  auto commit_lead = [&](uint64_t* b) {
+    if constexpr (PAIR) tc_commit_pair(dsmem_addr(smem_u32(b), 0u));
+    else tc_commit(b);
+  };
+  auto commit_both = [&](uint64_t* b) {
+    if constexpr (PAIR) {
+      tc_commit_pair(dsmem_addr(smem_u32(b), 0u));
+      tc_commit_pair(dsmem_addr(smem_u32(b), 1u));
+    } else {
+      tc_commit(b);
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
@@ -148,15 +181,25 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     mbar_init(branch_full, 1);
     mbar_init(branch_empty, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(acc_empty, kEpiWarps * (PAIR ? 2 : 1));
     fence_barrier_init();
   }
   if (warp == C::MMA_WARP) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {
+    // both CTAs' barriers are initialised before either signals the other's
+    cluster_arrive();
+    cluster_wait();
+  }
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // the next kernel in the stream may start its own set-up now
@@ -195,10 +238,9 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     return r;
   };
 
-  if (warp < C::STAGES) {
-    // ------------------------------------------------ producers: warp st owns ring slot st
-    const int st = warp;
-    if (lane == 0 && st == 0) {
+  if (warp < C::NPROD) {
+    // ------------------------------------------------ producers: warp w issues stages g = w mod NPROD
+    if (lane == 0 && warp == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       tma_prefetch_desc(&tmSA);
@@ -212,37 +254,46 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     // weight boxes (B and its scales) do not depend on the kernel before this one
     const bool weight_box = lane == 1 || lane >= 3;
     const CUtensorMap* map = lane == 0 ? &tmA : (lane == 1 ? &tmB : (lane == 2 ? &tmSA : &tmSB));
-    uint8_t* const dst = smem + (lane == 0   ? C::OFF_A + st * C::A_BYTES
-                                 : lane == 1 ? C::OFF_B + st * C::B_BYTES
-                                             : C::OFF_SF + st * C::SF_BYTES + (lane - 2) * C::SF_BLK);
+    const int dst_base = lane == 0 ? C::OFF_A : (lane == 1 ? C::OFF_B : C::OFF_SF + (lane - 2) * C::SF_BLK);
+    const int dst_step = lane == 0 ? C::A_BYTES : (lane == 1 ? C::B_BYTES : C::SF_BYTES);
     int g = 0;  // stage counter of this CTA
     int last = -1, nbranch = 0;
     bool ok = true;
     bool dep_done = false;  // griddep_wait() done: A, its scales and U may be read
-    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
+    for (int t = unit; ok && t < n_tiles; t += n_units) {
+      const TileCoord tc = coord(t);
       const Range rg = range_of(tc.split);
-      if (p.has_branch && tc.split == 0 && st == C::STAGES - 1) {
+      if (p.has_branch && tc.split == 0 && warp == C::NPROD - 1) {
         // branch operands of this tile, once the previous tile's branch MMAs are done
         int bok = 1;
         if (lane == 0) {
           bok = (nbranch == 0 || mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_PRODUCER_WAIT)) ? 1 : 0;
-          if (bok) mbar_arrive_expect_tx(branch_full, static_cast<uint32_t>((kBM + BN) * p.branch_k * 2));
+          if (bok && leader)
+            mbar_arrive_expect_tx(branch_full, static_cast<uint32_t>((PAIR ? 2 : 1) * (kBM + C::HB) * p.branch_k * 2));
         }
         bok = __shfl_sync(0xffffffffu, bok, 0);
         if (!bok) break;
         // L (weights) may load before the activation producer has finished; U not
-        if (lane == 1) tma_load_2d(smem + C::OFF_L, &tmL, branch_full, 0, tc.n0);
+        const int l_row = tc.n0 + static_cast<int>(rank) * C::HB;
+        if (lane == 1) {
+          if constexpr (PAIR) tma_load_2d_pair(smem + C::OFF_L, &tmL, lead(branch_full), 0, l_row);
+          else tma_load_2d(smem + C::OFF_L, &tmL, branch_full, 0, l_row);
+        }
         if (!dep_done) {
           griddep_wait();
           dep_done = true;
         }
-        if (lane == 0) tma_load_2d(smem + C::OFF_U, &tmU, branch_full, 0, tc.m0);
+        if (lane == 0) {
+          if constexpr (PAIR) tma_load_2d_pair(smem + C::OFF_U, &tmU, lead(branch_full), 0, tc.m0);
+          else tma_load_2d(smem + C::OFF_U, &tmU, branch_full, 0, tc.m0);
+        }
         ++nbranch;
       }
       for (int i = 0; i < rg.n_st; ++i, ++g) {
-        if (g % C::STAGES != st) continue;
+        if (g % C::NPROD != warp) continue;
+        const int st = g % C::STAGES;
         const uint32_t ph = (g / C::STAGES) & 1;
+        uint8_t* const dst = smem + dst_base + st * dst_step;
         int wok = 1;
         if (lane == 0) wok = mbar_wait(&empty[st], ph ^ 1u, p.err, DEVERR_PRODUCER_WAIT) ? 1 : 0;
         wok = __shfl_sync(0xffffffffu, wok, 0);
@@ -256,47 +307,54 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         int cx = 0, cy;
         if (lane < 2) {
           cx = kst * C::ROWB;
-          cy = lane ? tc.n0 : tc.m0;
+          cy = lane ? tc.n0 + static_cast<int>(rank) * C::HB : tc.m0;
         } else {
           const int blk = lane == 2 ? tc.m0 / kBM : tc.n0 / 128 + (lane - 3);
           cy = 2 * (blk * k64_total + kst * C::K64);
         }
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::STAGE_TX);
+        if (lane == 0 && leader) mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * C::STAGE_TX);
         __syncwarp();
+        auto load = [&]() {
+          if constexpr (PAIR) tma_load_2d_pair(dst, map, lead(&full[st]), cx, cy);
+          else tma_load_2d(dst, map, &full[st], cx, cy);
+        };
         if (dep_done) {
-          if (lane < C::NBOX) tma_load_2d(dst, map, &full[st], cx, cy);
+          if (lane < C::NBOX) load();
         } else {
           // the weight boxes first, then A and its scales once the kernel
           // writing them has finished
-          if (weight_box && lane < C::NBOX) tma_load_2d(dst, map, &full[st], cx, cy);
+          if (weight_box && lane < C::NBOX) load();
           griddep_wait();
           dep_done = true;
           if (!weight_box) {
-            if (lane < C::NBOX) tma_load_2d(dst, map, &full[st], cx, cy);
+            if (lane < C::NBOX) load();
           }
         }
         last = g;
       }
     }
-    // every copy this warp started must land before the CTA exits
+    // every copy this warp started must land before the CTA exits (in a pair
+    // rank 0 counts them; every MMA commit to this CTA's barriers must arrive)
     if (lane == 0) {
-      if (last >= 0) mbar_wait(&full[st], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
-      if (nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
+      if (leader && last >= 0) mbar_wait(&full[last % C::STAGES], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
+      if (leader && nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
+      if (PAIR && last >= 0) mbar_wait(&empty[last % C::STAGES], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
+      if (PAIR && nbranch > 0) mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
     }
     __syncwarp();
     cluster_tail();
   } else if (warp == C::MMA_WARP) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_fp4 = idesc_mxf4(kBM, BN);
-      const uint32_t idesc_br = idesc_bf16(kBM, BN);
+    // ------------------------------------------------ MMA issuer (rank 0 of a pair)
+    if (lane == 0 && leader) {
+      const uint32_t idesc_fp4 = idesc_mxf4(C::TM, BN);
+      const uint32_t idesc_br = idesc_bf16(C::TM, BN);
       const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
       const uint32_t sbo = 8u * p.branch_k * 2u;
       const uint32_t us = smem_u32(smem + C::OFF_U), ls = smem_u32(smem + C::OFF_L);
       int g = 0, tl = 0, nbranch = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tl) {
-        const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
+      for (int t = unit; ok && t < n_tiles; t += n_units, ++tl) {
+        const TileCoord tc = coord(t);
         const Range rg = range_of(tc.split);
         // the epilogue must have drained the previous tile's accumulator
         if (!mbar_wait(acc_empty, (tl & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) break;
@@ -306,11 +364,12 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
           if (!mbar_wait(branch_full, nbranch & 1, p.err, DEVERR_BRANCH_WAIT)) break;
           tc_fence_after();
           for (int kk = 0; kk < p.branch_k / 16; ++kk) {
-            mma_bf16(tmem, smem_desc(us + kk * 32, 16, sbo, layout), smem_desc(ls + kk * 32, 16, sbo, layout),
-                     idesc_br, accum);
+            const uint64_t ud = smem_desc(us + kk * 32, 16, sbo, layout), ld = smem_desc(ls + kk * 32, 16, sbo, layout);
+            if constexpr (PAIR) mma_bf16_pair(tmem, ud, ld, idesc_br, accum);
+            else mma_bf16(tmem, ud, ld, idesc_br, accum);
             accum = 1;
           }
-          tc_commit(branch_empty);
+          commit_both(branch_empty);
           ++nbranch;
         }
         for (int i = 0; i < rg.n_st; ++i, ++g) {
@@ -326,28 +385,29 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
           const uint32_t sfa = tmem + BN + sl * C::SF_COLS, sfb = sfa + C::SF_A_COLS;
           const int nk = min(C::K64, rg.n_k64 - i * C::K64);
           for (int kk = 0; kk < nk; ++kk) {
-            mma_mxf4nvf4(tmem, smem_desc(a_s + kk * 32, 16, 8 * C::ROWB, C::SWZ),
-                         smem_desc(b_s + kk * 32, 16, 8 * C::ROWB, C::SWZ), idesc_fp4, sfa + kk * 4,
-                         sfb + kk * (BN / 32), accum);
+            const uint64_t ad = smem_desc(a_s + kk * 32, 16, 8 * C::ROWB, C::SWZ);
+            const uint64_t bd = smem_desc(b_s + kk * 32, 16, 8 * C::ROWB, C::SWZ);
+            if constexpr (PAIR) mma_mxf4nvf4_pair(tmem, ad, bd, idesc_fp4, sfa + kk * 4, sfb + kk * (BN / 32), accum);
+            else mma_mxf4nvf4(tmem, ad, bd, idesc_fp4, sfa + kk * 4, sfb + kk * (BN / 32), accum);
             accum = 1;
           }
-          tc_commit(&empty[st]);
-          tc_commit(&sf_tfree[sl]);
+          commit_both(&empty[st]);
+          commit_lead(&sf_tfree[sl]);
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        commit_both(acc_full);
       }
     }
     __syncwarp();
     cluster_tail();
   } else if (warp < C::EPI_WARP0) {
-    // ------------------------------------------------ scale copies: smem stage -> TMEM slot
+    // ------------------------------------------------ scale copies: smem stage -> TMEM slot (rank 0 of a pair)
     const int cw = warp - C::CP_WARP0;
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int g = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const Range rg = range_of(tile_coord(t, tiles_m, tiles_n, BN, p.splits).split);
+      for (int t = unit; ok && t < n_tiles; t += n_units) {
+        const Range rg = range_of(coord(t).split);
         for (int i = 0; i < rg.n_st; ++i, ++g) {
           const int st = g % C::STAGES, sl = g % kScaleSlots;
           if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_SCALE_WAIT) ||
@@ -364,9 +424,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
             const int blk = c / C::K64, kk = c % C::K64;
             if (kk >= nk) continue;
             const uint32_t col = blk == 0 ? col0 + kk * 4 : col0 + C::SF_A_COLS + kk * (BN / 32) + (blk - 1) * 4;
-            tmem_cp_32x128b_x4(tmem + col, smem_desc(src + blk * C::SF_BLK + kk * 512, 0, 128, 0));
+            const uint64_t sd = smem_desc(src + blk * C::SF_BLK + kk * 512, 0, 128, 0);
+            if constexpr (PAIR) tmem_cp_32x128b_x4_pair(tmem + col, sd);
+            else tmem_cp_32x128b_x4(tmem + col, sd);
           }
-          tc_commit(&sf_ready[sl]);
+          commit_lead(&sf_ready[sl]);
         }
       }
     }
@@ -382,11 +444,15 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
     griddep_wait();  // g_a is written by the kernel before this one
     const float gs = __fmul_rn(p.g_a_ptr ? *p.g_a_ptr : p.g_a, p.g_b);
     const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
-    uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
+    // staging: a 32-row block per warp, the four blocks of a column half
+    // stacked in lane-quarter order (128 rows: one TMA store box)
+    uint8_t* stg = smem + C::OFF_STG + (half * 4 + qd) * C::STG_BYTES;
+    uint8_t* const stg_half = smem + C::OFF_STG + half * 4 * C::STG_BYTES;
+    const bool store_issuer = qd == 0 && lane == 0;  // one thread per column half
     uint4* bias_s = reinterpret_cast<uint4*>(smem + C::OFF_BIAS + ew * C::BIAS_BYTES);  // this warp's HC bf16
     int tl = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
-      const TileCoord tc = tile_coord(t, tiles_m, tiles_n, BN, p.splits);
+    for (int t = unit; t < n_tiles; t += n_units, ++tl) {
+      const TileCoord tc = coord(t);
       const int row = tc.m0 + qd * 32 + lane;
       const int c0 = tc.n0 + half * HC;
       if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
@@ -402,46 +468,66 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
       __syncwarp();
       tc_fence_after();
       if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
-        // drain: fp32 accumulator -> bf16 pairs in registers, then release
-        uint32_t packed[HC / 2];
+        // drain: y = bf16(acc * gs + bias).  The four warps of a column half
+        // stage 64 columns of their 128 rows (128B swizzle) and one thread
+        // stores them with one TMA box.  Every 64-column block but the last
+        // goes out before the accumulator is released; the last waits in
+        // registers until the staging blocks are free.  The half's named
+        // barrier is reached by all four warps on every path.
+        constexpr int NH = HC / 64;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC;
+        auto chunk = [&](int k) { return reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)); };
+        // 8 columns (qq * 32 + 8 j ..) of a 32-column TMEM load -> 4 bf16 pairs
+        auto convert = [&](const uint32_t* r, int qq, int j) {
+          const uint4 bw = bias_s[qq * 4 + j];
+          return make_uint4(fma_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1]), gs, bw.x),
+                            fma_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]), gs, bw.y),
+                            fma_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]), gs, bw.z),
+                            fma_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]), gs, bw.w));
+        };
+        auto half_sync = [&]() { named_bar(1 + half, 128); };
+        auto store_block = [&](int hh) {
+          fence_proxy_async();
+          half_sync();
+          if (store_issuer && ok) {
+            tma_store_2d(&tmY, stg_half, c0 + hh * 64, tc.m0);
+            bulk_commit();
+          }
+        };
 #pragma unroll
-        for (int qq = 0; qq < HC / 32; ++qq) {
+        for (int hh = 0; hh < NH - 1; ++hh) {
+          if (store_issuer) bulk_wait_read<0>();  // the staging blocks are free
+          half_sync();
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(taddr + (2 * hh + q2) * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) *chunk(4 * q2 + j) = convert(r, 2 * hh + q2, j);
+          }
+          store_block(hh);
+        }
+        uint4 last[8];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC + qq * 32, r);
+          tmem_ld_32x32b_x32(taddr + (2 * (NH - 1) + q2) * 32, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 braw = bias_s[qq * 4 + j];
-            const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              packed[qq * 16 + 4 * j + k] =
-                  pack_bf16x2(__fmaf_rn(__uint_as_float(r[8 * j + 2 * k]), gs, __uint_as_float(bw[k] << 16)),
-                              __fmaf_rn(__uint_as_float(r[8 * j + 2 * k + 1]), gs, __uint_as_float(bw[k] & 0xffff0000u)));
-          }
+          for (int j = 0; j < 4; ++j) last[4 * q2 + j] = convert(r, 2 * (NH - 1) + q2, j);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
-        if (ok) {
-          // stage 64 columns (32 rows x 128 B, 128B swizzle) per TMA store
-#pragma unroll
-          for (int cc = 0; cc < HC / 64; ++cc) {
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(packed[cc * 32 + 4 * j], packed[cc * 32 + 4 * j + 1], packed[cc * 32 + 4 * j + 2],
-                             packed[cc * 32 + 4 * j + 3]);
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&tmY, stg, c0 + cc * 64, tc.m0 + qd * 32);
-              bulk_commit();
-            }
-          }
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(lead(acc_empty));
+          else mbar_arrive(acc_empty);
         }
+        if (store_issuer) bulk_wait_read<0>();
+        half_sync();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) *chunk(k) = last[k];
+        store_block(NH - 1);
       } else if constexpr (EPI == static_cast<int>(GemmEpilogue::RawF32)) {
         // fp32 out: direct row stores
 #pragma unroll 1
@@ -462,7 +548,10 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(lead(acc_empty));
+          else mbar_arrive(acc_empty);
+        }
       } else {
         // Split-K: this tile's MMAs are done (acc_full), so this CTA's operand
         // ring is idle.  Push accumulator rows to their owner's ring, laid out
@@ -529,15 +618,22 @@ __global__ void __launch_bounds__(Cfg<BN, KS>::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {
+    // neither CTA leaves while the other may still signal its barriers
+    cluster_arrive();
+    cluster_wait();
+  }
   if (warp == C::MMA_WARP) {
     __syncwarp();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
-template <int BN, int KS, int EPI>
+
+template <int BN, int KS, int EPI, bool PAIR>
 cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
-  using C = Cfg<BN, KS>;
-  auto kern = fp4_gemm_kernel<BN, KS, EPI>;
+  using C = Cfg<BN, KS, PAIR>;
+  auto kern = fp4_gemm_kernel<BN, KS, EPI, PAIR>;
   static const cudaError_t smem_attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (smem_attr != cudaSuccess) return smem_attr;
@@ -546,7 +642,7 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
   if (p.k_stages != (p.K + KS - 1) / KS) return cudaErrorInvalidValue;
-  const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN) * p.splits;
+  const int tiles = ((p.M + C::TM - 1) / C::TM) * ((p.N + BN - 1) / BN) * p.splits;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
@@ -554,18 +650,36 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (EPI == static_cast<int>(GemmEpilogue::SplitK)) {
     // one work item per CTA; the splits of a tile are one cluster
-    if (p.splits < 2 || p.splits > 8 || (p.splits & (p.splits - 1)) || p.splits > p.k_stages)
+    if (PAIR || p.splits < 2 || p.splits > 8 || (p.splits & (p.splits - 1)) || p.splits > p.k_stages)
       return cudaErrorInvalidValue;
     cfg.gridDim = dim3(tiles, 1, 1);
-    attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = p.splits;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
+  } else if (PAIR) {
+    // persistent CTA pairs: as many as can be resident at once (a GPC with an
+    // odd number of free SMs leaves one idle)
+    if (p.splits != 1) return cudaErrorInvalidValue;
+    attr[1].val.clusterDim.x = 2;
+    cfg.numAttrs = 2;
+    static int pairs_per_dev[64] = {};
+    int pairs = dev >= 0 && dev < 64 ? pairs_per_dev[dev] : 0;
+    if (pairs <= 0) {
+      cfg.gridDim = dim3(sms & ~1, 1, 1);
+      if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess || pairs <= 0) {
+        (void)cudaGetLastError();
+        pairs = sms / 2;
+      }
+      pairs = std::min(pairs, sms / 2);
+      if (dev >= 0 && dev < 64) pairs_per_dev[dev] = pairs;
+    }
+    cfg.gridDim = dim3(2 * std::min(tiles, pairs), 1, 1);
   } else {
     if (p.splits != 1) return cudaErrorInvalidValue;
     cfg.gridDim = dim3(std::min(tiles, sms), 1, 1);
@@ -573,12 +687,14 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, m.a, m.b, m.u, m.l, m.y, m.sfa, m.sfb, p);
 }
 
-template <int BN, int KS>
+template <int BN, int KS, bool PAIR>
 cudaError_t launch_bn(const GemmMaps& m, const GemmParams& p, GemmEpilogue epi, cudaStream_t st) {
   switch (epi) {
-    case GemmEpilogue::Bf16: return launch_t<BN, KS, 0>(m, p, st);
-    case GemmEpilogue::RawF32: return launch_t<BN, KS, 1>(m, p, st);
-    case GemmEpilogue::SplitK: return launch_t<BN, KS, 2>(m, p, st);
+    case GemmEpilogue::Bf16: return launch_t<BN, KS, 0, PAIR>(m, p, st);
+    case GemmEpilogue::RawF32: return launch_t<BN, KS, 1, PAIR>(m, p, st);
+    case GemmEpilogue::SplitK:
+      if constexpr (PAIR) return cudaErrorInvalidValue;
+      else return launch_t<BN, KS, 2, false>(m, p, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -589,14 +705,19 @@ GemmShape gemm_shape(int M, int N) {
   GemmShape s;
   s.bn = (M <= kBM || N < 256) ? 128 : 256;
   s.ks = M <= kBM ? 128 : 256;
+  s.pair = s.bn == 256;
   return s;
 }
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
                         cudaStream_t st) {
-  if (shape.bn == 256 && shape.ks == 256) return launch_bn<256, 256>(maps, p, epi, st);
-  if (shape.bn == 128 && shape.ks == 256) return launch_bn<128, 256>(maps, p, epi, st);
-  if (shape.bn == 128 && shape.ks == 128) return launch_bn<128, 128>(maps, p, epi, st);
+  if (shape.pair) {
+    if (shape.bn == 256 && shape.ks == 256) return launch_bn<256, 256, true>(maps, p, epi, st);
+    return cudaErrorInvalidValue;
+  }
+  if (shape.bn == 256 && shape.ks == 256) return launch_bn<256, 256, false>(maps, p, epi, st);
+  if (shape.bn == 128 && shape.ks == 256) return launch_bn<128, 256, false>(maps, p, epi, st);
+  if (shape.bn == 128 && shape.ks == 128) return launch_bn<128, 128, false>(maps, p, epi, st);
   return cudaErrorInvalidValue;
 }
 

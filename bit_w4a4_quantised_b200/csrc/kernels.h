@@ -83,19 +83,24 @@ struct GemmMaps {
   CUtensorMap b;    // codes B [N, K/2] u8, box (ks/2) B x bn rows, same swizzle
   CUtensorMap u;    // branch A [M, r] bf16, box r x 128 rows
   CUtensorMap l;    // branch B [N, r] bf16, box r x bn rows
-  CUtensorMap y;    // output y [M, N] bf16, box 64 x 32 rows, 128B swizzle (bf16 epilogue)
+  CUtensorMap y;    // output y [M, N] bf16, box 64 x 128 rows, 128B swizzle (bf16 epilogue)
   CUtensorMap sfa;  // A scales viewed as u8 [rows * K / 16 / 256, 256], box 256 x (ks / 32): one stage of 128 rows
   CUtensorMap sfb;  // B scales, same view and box
 };
 
-// Tile width and K per pipeline stage for an M x N output.
+// Tile width, K per pipeline stage and CTA pairing for an M x N output.  With
+// pair set, a two-CTA cluster computes 256 x bn tiles (cta_group::2) and each
+// CTA reads bn / 2 rows of B: the B (and L) tensor maps must have bn / 2-row
+// boxes.  gemm_shape proposes pair for bn == 256; a split-K plan turns it off.
 struct GemmShape {
   int bn, ks;
+  bool pair;
 };
 GemmShape gemm_shape(int M, int N);
 
 // p.k_stages must be ceil(K / shape.ks); split-K (p.splits in {2, 4, 8}) needs
-// the SplitK epilogue and launches one cluster of p.splits CTAs per tile.
+// the SplitK epilogue, shape.pair false, and launches one cluster of p.splits
+// CTAs per tile.
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
                         cudaStream_t st);
 
