@@ -88,21 +88,39 @@ qwam_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
   return QWAM_OK;
 }
 
-// Scale buffer of `rows_padded` rows (multiple of 128) and K columns in the tiled
-// layout, viewed as u8 [rows_padded * K / 16 / 256, 256]: a 512-byte atom (one
-// K64 step of 128 rows) is two rows, so one GEMM stage of ks K elements of one
-// 128-row block is a 256 x (ks / 32) box.
-qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, int K, int ks) {
-  const uint64_t total = static_cast<uint64_t>(rows_padded) * K / 16;
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, total / 256, 256, 256, static_cast<uint32_t>(ks / 32),
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
+qwam_status make_map3(CUtensorMap* m, const void* base, const cuuint64_t (&dims)[3], const cuuint64_t (&strides)[2],
+                      const cuuint32_t (&box)[3], CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail(QWAM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QWAM_ERR_CUDA, "cuTensorMapEncodeTiled failed with code %d", static_cast<int>(r));
+  return QWAM_OK;
 }
 
-// Packed E2M1 operand [rows, K/2] u8 as the GEMM reads it: one box per stage of
-// ks K elements (ks / 2 bytes, one swizzle atom wide) by box_rows rows.
+// The GEMM's four boxes per stage all come through 3-D maps, so one converged
+// TMA instruction issues them (one box per lane).
+//
+// Scale buffer of `rows_padded` rows (multiple of 128) and K columns in the tiled
+// layout, viewed as u8 [rows_padded / 128][K / 32][256]: a 512-byte atom (one K64
+// step of 128 rows) is two 256-byte rows, so one stage of ks K elements of
+// `blocks` consecutive 128-row blocks is a 256 x (ks / 32) x blocks box.
+qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, int K, int ks, int blocks) {
+  const cuuint64_t dims[3] = {256, static_cast<cuuint64_t>(K / 32), static_cast<cuuint64_t>(rows_padded / 128)};
+  const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(K) * 8};
+  const cuuint32_t box[3] = {256, static_cast<cuuint32_t>(ks / 32), static_cast<cuuint32_t>(blocks)};
+  return make_map3(m, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Packed E2M1 operand [rows, K/2] u8 as the GEMM reads it (a unit third
+// dimension): one box per stage of ks K elements (ks / 2 bytes, one swizzle atom
+// wide) by box_rows rows.
 qwam_status make_codes_map(CUtensorMap* m, const void* base, int rows, int K, int ks, int box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, K / 2, rows, K / 2, ks / 2, box_rows,
-                  ks == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(K / 2) * rows};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(ks / 2), static_cast<cuuint32_t>(box_rows), 1};
+  return make_map3(m, base, dims, strides, box, ks == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B; }
@@ -217,7 +235,8 @@ struct qwam_layer {
   uint16_t* bias;
   float g_w;
   size_t sf_bytes;
-  CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256, map_sfb_k128, map_sfb_k256;
+  CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256;
+  CUtensorMap map_sfb_k128, map_sfb_k256_b1, map_sfb_k256_b2;  // B scales: K per stage, 128-row blocks per box
   ProMaps vmaps;  // P^T and V (hi/lo) tensor maps for the prologue; x is per call
 };
 
@@ -381,8 +400,9 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
       (s_ = make_codes_map(&h->map_b128_k256, h->codes, N, K, 256, 128)) != QWAM_OK ||
       (s_ = make_codes_map(&h->map_b256_k256, h->codes, N, K, 256, 256)) != QWAM_OK)
     return cleanup(s_);
-  if ((s_ = make_sf_map(&h->map_sfb_k128, h->sf, round_up(static_cast<size_t>(N), 256), K, 128)) != QWAM_OK ||
-      (s_ = make_sf_map(&h->map_sfb_k256, h->sf, round_up(static_cast<size_t>(N), 256), K, 256)) != QWAM_OK)
+  if ((s_ = make_sf_map(&h->map_sfb_k128, h->sf, round_up(static_cast<size_t>(N), 256), K, 128, 1)) != QWAM_OK ||
+      (s_ = make_sf_map(&h->map_sfb_k256_b1, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 1)) != QWAM_OK ||
+      (s_ = make_sf_map(&h->map_sfb_k256_b2, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 2)) != QWAM_OK)
     return cleanup(s_);
   if (r > 0) {
     if ((s_ = make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r))) !=
@@ -448,8 +468,8 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, a->base + lay.codes, M, h->K, pl.ks, 128));
   maps.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
-  QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks));
-  maps.sfb = pl.ks == 256 ? h->map_sfb_k256 : h->map_sfb_k128;
+  QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks, 1));
+  maps.sfb = pl.ks == 128 ? h->map_sfb_k128 : (pl.bn == 256 ? h->map_sfb_k256_b2 : h->map_sfb_k256_b1);
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
@@ -560,8 +580,8 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   GemmMaps maps{};
   QW_TRY(make_codes_map(&maps.a, base + lay.codes, M, h->K, pl.ks, 128));
   maps.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
-  QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks));
-  maps.sfb = pl.ks == 256 ? h->map_sfb_k256 : h->map_sfb_k128;
+  QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks, 1));
+  maps.sfb = pl.ks == 128 ? h->map_sfb_k128 : (pl.bn == 256 ? h->map_sfb_k256_b2 : h->map_sfb_k256_b1);
   if (h->r > 0) {
     QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base + lay.ub, h->r, M, h->r * 2, h->r, 128,
                     branch_swizzle(h->r)));
@@ -725,8 +745,8 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   maps.u = maps.a;
   maps.l = maps.b;
   maps.y = maps.a;
-  QW_TRY(make_sf_map(&maps.sfa, a_scales, round_up(static_cast<size_t>(M), 128), K, sh.ks));
-  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), sh.bn), K, sh.ks));
+  QW_TRY(make_sf_map(&maps.sfa, a_scales, round_up(static_cast<size_t>(M), 128), K, sh.ks, 1));
+  QW_TRY(make_sf_map(&maps.sfb, b_scales, round_up(static_cast<size_t>(N), sh.bn), K, sh.ks, sh.bn / 128));
   GemmParams p{};
   p.M = M; p.N = N; p.K = K;
   p.k_stages = (K + sh.ks - 1) / sh.ks;

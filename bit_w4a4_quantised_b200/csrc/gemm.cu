@@ -14,10 +14,11 @@
 //
 // Persistent kernel, one CTA per SM, tiles of 128 x BN, K in stages of KS
 // elements (KS / 2 bytes of packed E2M1 per row: one 128B- or 64B-swizzle
-// atom), K64 per MMA.  A stage is one box each of A, B, the A scale blocks and
-// each 128-row block of B scales, all issued by different lanes of one
-// instruction: on this part a lane's TMA boxes run one after another at a
-// roughly fixed cost per box, while boxes from different lanes overlap.
+// atom), K64 per MMA.  A stage is one box each of A, B, the A scales and the B
+// scales (every 128-row block of the tile in one 3-D box), all issued by
+// different lanes of one instruction: on this part a lane's TMA boxes run one
+// after another at a roughly fixed cost per box, while boxes from different
+// lanes overlap.
 // Roles:
 //   producer warps  one per ring slot (a TMA instruction holds its warp for
 //                   several hundred cycles); the first stage's weight boxes go
@@ -60,7 +61,7 @@ struct Cfg {
   static constexpr int STAGES = PAIR ? 4 : (KS == 256 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
   static constexpr int NSFB = BN / 128;                     // 128-row scale blocks of B
   static constexpr int SF_BLK = K64 * 512;                  // one 128-row scale block of a stage
-  static constexpr int NBOX = 3 + NSFB;                     // boxes per stage: A, B, A scales, B scale blocks
+  static constexpr int NBOX = 4;                            // boxes per stage: A, B, A scales, B scales
   // producer warps, taking stages in turn (three keep the CTA at 16 warps, so
   // the epilogue keeps 128 registers)
   static constexpr int NPROD = STAGES < 3 ? STAGES : 3;
@@ -250,9 +251,9 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         tma_prefetch_desc(&tmL);
       }
     }
-    // this lane's box of a stage: 0 A, 1 B, 2 A scales, 3.. B scale blocks;
-    // weight boxes (B and its scales) do not depend on the kernel before this one
-    const bool weight_box = lane == 1 || lane >= 3;
+    // this lane's box of a stage: 0 A, 1 B, 2 A scales, 3 B scales; weight
+    // boxes (B and its scales) do not depend on the kernel before this one
+    const bool weight_box = lane == 1 || lane == 3;
     const CUtensorMap* map = lane == 0 ? &tmA : (lane == 1 ? &tmB : (lane == 2 ? &tmSA : &tmSB));
     const int dst_base = lane == 0 ? C::OFF_A : (lane == 1 ? C::OFF_B : C::OFF_SF + (lane - 2) * C::SF_BLK);
     const int dst_step = lane == 0 ? C::A_BYTES : (lane == 1 ? C::B_BYTES : C::SF_BYTES);
@@ -302,21 +303,21 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
           break;
         }
         const int kst = rg.s_begin + i;
-        // operands: x = byte column, y = row; scales (u8 rows of 256 B, two per
-        // K64 step of a 128-row block): x = 0, y = 2 * (block * K/64 + step)
-        int cx = 0, cy;
+        // operands: x = byte column, y = row, z = 0; scales (256-byte rows, two
+        // per K64 step of a 128-row block): x = 0, y = 2 * step, z = block
+        int cx = 0, cy, cz = 0;
         if (lane < 2) {
           cx = kst * C::ROWB;
           cy = lane ? tc.n0 + static_cast<int>(rank) * C::HB : tc.m0;
         } else {
-          const int blk = lane == 2 ? tc.m0 / kBM : tc.n0 / 128 + (lane - 3);
-          cy = 2 * (blk * k64_total + kst * C::K64);
+          cy = 2 * kst * C::K64;
+          cz = lane == 2 ? tc.m0 / kBM : tc.n0 / 128;
         }
         if (lane == 0 && leader) mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * C::STAGE_TX);
         __syncwarp();
         auto load = [&]() {
-          if constexpr (PAIR) tma_load_2d_pair(dst, map, lead(&full[st]), cx, cy);
-          else tma_load_2d(dst, map, &full[st], cx, cy);
+          if constexpr (PAIR) tma_load_3d_pair(dst, map, lead(&full[st]), cx, cy, cz);
+          else tma_load_3d(dst, map, &full[st], cx, cy, cz);
         };
         if (dep_done) {
           if (lane < C::NBOX) load();
