@@ -232,6 +232,7 @@ struct qwam_layer {
   uint16_t *v_hi, *v_lo;    // V [K, r] bf16 hi/lo
   uint16_t *px_hi, *px_lo;  // P^T = (diag(1/s) H V)^T [r, K] bf16 hi/lo
   float* inv_s;
+  float* inv_s_pm;  // row-pipeline form of 1/s: [K / 128][2][128], * 1/sqrt(b), then negated
   uint16_t* bias;
   float g_w;
   size_t sf_bytes;
@@ -244,7 +245,7 @@ namespace {
 
 void free_layer(qwam_layer* h) {
   if (!h) return;
-  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->px_hi, h->px_lo, h->inv_s, h->bias};
+  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->px_hi, h->px_lo, h->inv_s, h->inv_s_pm, h->bias};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   h->magic = 0;
@@ -325,7 +326,9 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   float* u_tmp = nullptr;
   uint32_t* scratch = nullptr;  // [0] amax, [1] err, [2] g_w (fp32)
   uint16_t *pw_hi = nullptr, *pw_lo = nullptr;  // P^T of the weight side, diag(s) H V
+  float* s_pm = nullptr;                         // row-pipeline form of s for the weight pass
   auto cleanup = [&](qwam_status s) {
+    if (s_pm) cudaFree(s_pm);
     if (u_tmp) cudaFree(u_tmp);
     if (scratch) cudaFree(scratch);
     if (pw_hi) cudaFree(pw_hi);
@@ -341,6 +344,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
       (s_ = dmalloc(&h->px_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->px_lo, K * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&pw_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&pw_lo, K * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->inv_s, static_cast<size_t>(K) * 4)) != QWAM_OK ||
+      (s_ = dmalloc(&h->inv_s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK || (s_ = dmalloc(&s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK ||
       (s_ = dmalloc(&u_tmp, static_cast<size_t>(N) * rr * 4)) != QWAM_OK || (s_ = dmalloc(&scratch, 64)) != QWAM_OK)
     return cleanup(s_);
   if (bias && (s_ = dmalloc(&h->bias, static_cast<size_t>(N) * 2)) != QWAM_OK) return cleanup(s_);
@@ -355,6 +359,9 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   QW_CUDA_CLEAN(cudaMemsetAsync(scratch, 0, 64, st));
   if (bias) QW_CUDA_CLEAN(cudaMemcpyAsync(h->bias, bias, static_cast<size_t>(N) * 2, cudaMemcpyDeviceToDevice, st));
   QW_CUDA_CLEAN(launch_recip(s, h->inv_s, K, scratch + 1, st));
+  const float hscale = 1.0f / std::sqrt(static_cast<float>(b));
+  QW_CUDA_CLEAN(launch_chan_pm(h->inv_s, hscale, K, h->inv_s_pm, st));
+  QW_CUDA_CLEAN(launch_chan_pm(s, hscale, K, s_pm, st));
   ProMaps wmaps{};  // the weight pass uses P of the weight side
   if (r > 0) {
     QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, st));
@@ -374,11 +381,11 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
     if ((s_ = pmap(&wmaps.p_hi, pw_hi)) != QWAM_OK || (s_ = pmap(&wmaps.p_lo, pw_lo)) != QWAM_OK) return cleanup(s_);
   }
   PrologueParams prm{};
-  prm.chan = s;
+  prm.chan = s_pm;
   prm.rows = N;
   prm.K = K;
   prm.b = b;
-  prm.hscale = 1.0f / std::sqrt(static_cast<float>(b));
+  prm.hscale = hscale;
   prm.u_glob = u_tmp;
   prm.codes = h->codes;
   prm.sf = h->sf;
@@ -414,6 +421,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
     h->map_l128 = h->map_b128_k128;
     h->map_l256 = h->map_b256_k256;
   }
+  cudaFree(s_pm);
   cudaFree(u_tmp);
   cudaFree(scratch);
   cudaFree(pw_hi);
@@ -439,7 +447,7 @@ qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, flo
   Arena* a = nullptr;
   QW_TRY(arena_get(h->dev, lay.total, &a));
   PrologueParams prm{};
-  prm.chan = h->inv_s;
+  prm.chan = h->inv_s_pm;
   prm.rows = M;
   prm.K = h->K;
   prm.b = h->b;
@@ -562,7 +570,7 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
   uint32_t* err = reinterpret_cast<uint32_t*>(base + 8);
 
   PrologueParams prm{};
-  prm.chan = h->inv_s;
+  prm.chan = h->inv_s_pm;
   prm.rows = M;
   prm.K = h->K;
   prm.b = h->b;

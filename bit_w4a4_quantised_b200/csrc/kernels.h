@@ -22,7 +22,7 @@ struct ProMaps {
 };
 
 struct PrologueParams {
-  const float* chan;      // fp32 [K]
+  const float* chan;      // fp32 [K / 128][2][128]: chan * hscale, then -(chan * hscale), per chunk
   int rows;
   int K;
   int b;                  // Hadamard block (power of two, <= 128)
@@ -51,6 +51,8 @@ cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r,
                             cudaStream_t st);
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st);
+// out [K / 128][2][128] fp32: chunk c holds chan[128c..] * hscale, then its negation.
+cudaError_t launch_chan_pm(const float* chan, float hscale, int K, float* out, cudaStream_t st);
 cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, cudaStream_t st);
 // P^T = (diag(chan) H V)^T split into bf16 hi/lo, [r, K] each; H block size b.
 cudaError_t launch_make_proj(const float* V, const float* chan, int K, int r, int b, uint16_t* p_hi, uint16_t* p_lo,

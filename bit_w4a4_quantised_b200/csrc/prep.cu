@@ -54,6 +54,18 @@ __global__ void recip_kernel(const float* __restrict__ s, float* __restrict__ in
   inv_s[i] = __frcp_rn(v);
 }
 
+// Row-pipeline channel vector: per 128-column chunk, [chan * hscale | -(chan * hscale)]
+// (fp32 products, round to nearest), so the rotation reads a signed, scaled
+// factor instead of multiplying by hscale and selecting a sign per element.
+__global__ void chan_pm_kernel(const float* __restrict__ chan, float hscale, int K, float* __restrict__ out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= K) return;
+  const float v = __fmul_rn(chan[i], hscale);
+  const int chunk = i >> 7, j = i & 127;
+  out[chunk * 256 + j] = v;
+  out[chunk * 256 + 128 + j] = -v;
+}
+
 __global__ void split_v_kernel(const float* __restrict__ V, int K, int r, uint16_t* v_hi, uint16_t* v_lo) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= K * r) return;
@@ -92,6 +104,12 @@ __global__ void make_proj_kernel(const float* __restrict__ V, const float* __res
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st) {
   recip_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chan_pm(const float* chan, float hscale, int K, float* out, cudaStream_t st) {
+  if (K % 128) return cudaErrorInvalidValue;
+  chan_pm_kernel<<<(K + 255) / 256, 256, 0, st>>>(chan, hscale, K, out);
   return cudaGetLastError();
 }
 

@@ -69,7 +69,7 @@ struct PCfg {
   static constexpr int X_BYTES = kRows * kChunk * 2;  // two 64-column SW128 boxes
   static constexpr int P_BYTES = 512 * R;             // P^T: [kb][hi, lo] boxes of R rows x 128 B
   static constexpr int V_BYTES = 512 * R;             // V hi/lo: 2 boxes of 128 rows x 2R B
-  static constexpr int CH_BYTES = kChunk * 4;
+  static constexpr int CH_BYTES = kChunk * 8;         // chan * hscale and its negation
   static constexpr int OFF_P = X_BYTES;
   static constexpr int OFF_V = OFF_P + P_BYTES;
   static constexpr int OFF_CH = OFF_V + V_BYTES;
@@ -121,38 +121,41 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
 
 // This thread's W columns [W*s0, W*s0 + W) of tile row `row` of one chunk:
 //   out = ((T * chan) H_b) restricted to those columns, times 1/sqrt(b).
-// The Hadamard bits above log2(W) combine the chunk's column ranges s that lie
-// in the same b-block (sign (-1)^popcount of the in-block bits of s & s0,
-// Sylvester order); the bits
-// below are butterflies (lo + hi, lo - hi) in registers.  Identical code and op
-// order in every sweep, so recomputed Z is bit-identical.
+// chan (shared memory) holds this chunk's chan * hscale in [0, 128) and its
+// negation in [128, 256).  The Hadamard bits above log2(W) combine the chunk's
+// column ranges s that lie in the same b-block: each contributes T * (+-chan *
+// hscale), the sign (-1)^popcount of the in-block bits of s & s0 (Sylvester
+// order) chosen by reading the negated half; the thread's own range first, the
+// others added with one packed FMA per pair.  The bits below log2(W) are
+// butterflies (lo + hi, lo - hi) in registers.  Identical
+// code and op order in every sweep, so recomputed Z is bit-identical.
 template <int W>
-__device__ __forceinline__ void rotate_cols(const uint8_t* xs, const float* chan, int row, int s0, int b, float hscale,
+__device__ __forceinline__ void rotate_cols(const uint8_t* xs, const float* chan, int row, int s0, int b,
                                             float (&v)[W]) {
   constexpr int NSEG = kChunk / W;
   float2* v2 = reinterpret_cast<float2*>(v);  // element pairs (2i, 2i + 1)
+  // own range first (d = 0: v = T * c), then the others of the b-block (v += T * c)
 #pragma unroll
-  for (int i = 0; i < W; ++i) v[i] = 0.0f;
-#pragma unroll
-  for (int s = 0; s < NSEG; ++s) {
-    if ((s ^ s0) * W >= b) continue;  // other b-block
+  for (int d = 0; d < NSEG; ++d) {
+    if (d * W >= b) continue;  // range s0 ^ d lies in another b-block
+    const int s = s0 ^ d;
     const bool neg = (__popc(s & s0 & ((b - 1) / W)) & 1) != 0;  // in-block segment bits only
     const int col = s * W;                        // first column of range s
     const uint8_t* box = xs + (col >> 6) * 16384 + row * 128;
     const int c16 = (col & 63) >> 3;              // first 16-byte chunk inside the box row
+    const float* cs = chan + (neg ? kChunk : 0) + col;
 #pragma unroll
     for (int g = 0; g < W / 8; ++g) {
       const uint4 w = *reinterpret_cast<const uint4*>(box + (((c16 + g) ^ (row & 7)) << 4));
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-      const float4 c0 = *reinterpret_cast<const float4*>(chan + col + 8 * g);
-      const float4 c1 = *reinterpret_cast<const float4*>(chan + col + 8 * g + 4);
+      const float4 c0 = *reinterpret_cast<const float4*>(cs + 8 * g);
+      const float4 c1 = *reinterpret_cast<const float4*>(cs + 8 * g + 4);
       const float2 cc[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
                             make_float2(c1.z, c1.w)};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 t = make_float2(__uint_as_float(ws[e] << 16), __uint_as_float(ws[e] & 0xffff0000u));
-        const float2 a = f2_mul(t, cc[e]);
-        v2[4 * g + e] = neg ? f2_sub(v2[4 * g + e], a) : f2_add(v2[4 * g + e], a);
+        v2[4 * g + e] = d == 0 ? f2_mul(t, cc[e]) : f2_fma(t, cc[e], v2[4 * g + e]);
       }
     }
   }
@@ -178,9 +181,6 @@ __device__ __forceinline__ void rotate_cols(const uint8_t* xs, const float* chan
       }
     }
   }
-  const float2 hs = make_float2(hscale, hscale);
-#pragma unroll
-  for (int i = 0; i < W / 2; ++i) v2[i] = f2_mul(v2[i], hs);
 }
 
 // Quantise this thread's W values of row `row`, chunk columns starting at `col`.
@@ -188,18 +188,11 @@ template <int W>
 __device__ __forceinline__ void quantise_cols(const PrologueParams& p, const float (&v)[W], int row, int col,
                                               float g) {
   uint32_t cw[W / 8];
+  uint32_t S[W / 16];
+  quant_blocks16<W / 16>(v, g, cw, S);
   uint32_t sfw = 0u;
 #pragma unroll
-  for (int k = 0; k < W / 16; ++k) {
-    float blk[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) blk[e] = v[16 * k + e];
-    uint32_t c2[2];
-    const uint32_t S = quant_block16(blk, g, c2);
-    cw[2 * k] = c2[0];
-    cw[2 * k + 1] = c2[1];
-    sfw |= S << (8 * k);
-  }
+  for (int k = 0; k < W / 16; ++k) sfw |= S[k] << (8 * k);
   uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + col / 2);
 #pragma unroll
   for (int k = 0; k < W / 32; ++k) dst[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
@@ -275,7 +268,7 @@ __device__ __forceinline__ uint32_t load_bytes(uint32_t kind) {
   if (kind & LD_X) n += kRows * kChunk * 2;
   if (kind & LD_P) n += 512 * R;
   if (kind & LD_V) n += 512 * R;
-  if (kind & LD_CH) n += kChunk * 4;
+  if (kind & LD_CH) n += kChunk * 8;
   return n;
 }
 
@@ -334,7 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // writer's arrival at the last of these, so once a CTA has passed that
   // barrier no peer touches its shared memory again and it may exit.
   if constexpr (C::kCluster) cluster_arrive();  // A0
-  // the GEMM that consumes this launch's output may start its weight loads now
+  // The next kernel may start its set-up now.  Stats first waits for the kernel
+  // before it, so once Quantise (its dependent) runs, T is final and Quantise
+  // may load it before its own wait.
+  if constexpr (MODE == 1) griddep_wait();
   griddep_launch_dependents();
   const uint32_t d2_tmem = tmem;
   const uint32_t u_tmem = tmem + 128;
@@ -381,14 +377,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = pp ? &maps.v_lo : &maps.v_hi; dst = s + C::OFF_V + pp * 256 * R; x = 0; y = col;
       }
       // This warp's first load: the layer constants (P, V, chan) go out while the
-      // previous kernel in the stream may still run; T only after it finished.
-      if (m && (dep_done || lane >= 2)) tma_load_2d(dst, m, &full[slot], x, y);
+      // previous kernel in the stream may still run; T only after it finished
+      // (Quantise: T was final before it launched).
+      if (m && (dep_done || lane >= 2 || MODE == 2)) tma_load_2d(dst, m, &full[slot], x, y);
       if (!dep_done) {
-        griddep_wait();
+        if constexpr (MODE != 2) griddep_wait();  // Quantise's producers read nothing Stats writes
         dep_done = true;
-        if (m && lane < 2) tma_load_2d(dst, m, &full[slot], x, y);
+        if (m && lane < 2 && MODE != 2) tma_load_2d(dst, m, &full[slot], x, y);
       }
-      if (lane == 0 && (kind & LD_CH)) bulk_load(s + C::OFF_CH, p.chan + col, C::CH_BYTES, &full[slot]);
+      if (lane == 0 && (kind & LD_CH)) bulk_load(s + C::OFF_CH, p.chan + 2 * col, C::CH_BYTES, &full[slot]);
       last = i;
     };
     // The producers pass each cluster barrier before any load whose ring slot
@@ -652,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = i & 1;
       mbar_wait(&full[slot], (i >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
       const uint8_t* s = smem + slot * C::SLOT;
-      if (zact) rotate_cols<W>(s, reinterpret_cast<const float*>(s + C::OFF_CH), zrow, s0, p.b, p.hscale, z);
+      if (zact) rotate_cols<W>(s, reinterpret_cast<const float*>(s + C::OFF_CH), zrow, s0, p.b, z);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
       if constexpr (R > 0) {

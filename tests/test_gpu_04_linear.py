@@ -31,6 +31,9 @@ CASES = {
     "m48_k6144_n128_r32_b128": lambda: workloads.custom(48, 6144, 128, 32, 128, seed=18, n_outliers=60),
     # persistent tiles with a partial last 256-K stage
     "m260_k1408_n640_r16_b64": lambda: workloads.custom(260, 1408, 640, 16, 64, seed=19, n_outliers=14),
+    # 256 x 256 tiles on CTA pairs (no split-K): ragged M, then ragged M and N
+    "m1000_k1024_n2560_r32_b128": lambda: workloads.custom(1000, 1024, 2560, 32, 128, seed=23, n_outliers=10),
+    "m1000_k768_n2320_r16_b64": lambda: workloads.custom(1000, 768, 2320, 16, 64, seed=24, n_outliers=8),
 }
 
 
