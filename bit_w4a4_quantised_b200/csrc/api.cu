@@ -234,6 +234,7 @@ struct qwam_layer {
   float* inv_s;
   float* inv_s_pm;  // row-pipeline form of 1/s: [K / 128][2][128], * 1/sqrt(b), then negated
   uint16_t* bias;
+  uint16_t* hmat;   // bf16 [128, 128]: the H_b blocks of one 128-column chunk (+-1)
   float g_w;
   size_t sf_bytes;
   CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256;
@@ -245,7 +246,7 @@ namespace {
 
 void free_layer(qwam_layer* h) {
   if (!h) return;
-  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->px_hi, h->px_lo, h->inv_s, h->inv_s_pm, h->bias};
+  void* ptrs[] = {h->codes, h->sf, h->L, h->v_hi, h->v_lo, h->px_hi, h->px_lo, h->inv_s, h->inv_s_pm, h->bias, h->hmat};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   h->magic = 0;
@@ -345,6 +346,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
       (s_ = dmalloc(&pw_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&pw_lo, K * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->inv_s, static_cast<size_t>(K) * 4)) != QWAM_OK ||
       (s_ = dmalloc(&h->inv_s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK || (s_ = dmalloc(&s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK ||
+      (s_ = dmalloc(&h->hmat, 128 * 128 * 2)) != QWAM_OK ||
       (s_ = dmalloc(&u_tmp, static_cast<size_t>(N) * rr * 4)) != QWAM_OK || (s_ = dmalloc(&scratch, 64)) != QWAM_OK)
     return cleanup(s_);
   if (bias && (s_ = dmalloc(&h->bias, static_cast<size_t>(N) * 2)) != QWAM_OK) return cleanup(s_);
@@ -362,7 +364,21 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   const float hscale = 1.0f / std::sqrt(static_cast<float>(b));
   QW_CUDA_CLEAN(launch_chan_pm(h->inv_s, hscale, K, h->inv_s_pm, st));
   QW_CUDA_CLEAN(launch_chan_pm(s, hscale, K, s_pm, st));
+  // H_b restricted to one 128-column chunk, in Sylvester order: +-1 where row and
+  // column lie in the same b-block, 0 elsewhere (1/sqrt(b) is in the channel
+  // vector); the B operand of the prologue's tensor-core rotation.
+  {
+    std::vector<uint16_t> hm(128 * 128);
+    for (int n = 0; n < 128; ++n)
+      for (int k = 0; k < 128; ++k)
+        hm[n * 128 + k] = (n ^ k) >= b ? 0 : ((__builtin_popcount(n & k & (b - 1)) & 1) ? 0xBF80u : 0x3F80u);
+    QW_CUDA_CLEAN(cudaMemcpy(h->hmat, hm.data(), hm.size() * 2, cudaMemcpyHostToDevice));
+    if ((s_ = make_map(&h->vmaps.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->hmat, 128, 128, 256, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK)
+      return cleanup(s_);
+  }
   ProMaps wmaps{};  // the weight pass uses P of the weight side
+  wmaps.h = h->vmaps.h;
   if (r > 0) {
     QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, st));
     QW_CUDA_CLEAN(launch_make_proj(V, s, K, r, b, pw_hi, pw_lo, st));

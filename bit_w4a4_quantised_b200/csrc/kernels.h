@@ -19,6 +19,7 @@ struct ProMaps {
   CUtensorMap p_lo;
   CUtensorMap v_hi;  // V bf16 [K, r] (hi/lo split), box r x 128 rows, 2r-byte swizzle
   CUtensorMap v_lo;
+  CUtensorMap h;     // H_b blocks of one 128-column chunk (+-1, block diagonal) bf16 [128, 128], box 64 x 128, 128B swizzle
 };
 
 struct PrologueParams {

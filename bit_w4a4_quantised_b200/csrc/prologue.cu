@@ -59,36 +59,48 @@ enum : uint32_t { LD_X = 1u, LD_P = 2u, LD_V = 4u, LD_CH = 8u };
 // W = columns of a chunk per row thread: 64 (normal) or 32 (small layout).
 template <int R, int MODE, int W>
 struct PCfg {
-  static constexpr bool kMMA = R > 0;
+  // Stats / Quantise: the rotation runs on the tensor core, Z = (A_hi + A_lo) H -
+  // c V^T into TMEM, with A = T * chan * hscale split into bf16 hi/lo by the rows
+  static constexpr bool kTC = MODE != 0;
+  static constexpr bool kMMA = R > 0 || kTC;
   static constexpr bool kProj = R > 0 && MODE != 2;   // this launch computes c
   static constexpr bool kNeedA = kProj;               // cluster exchange of partial c
   static constexpr bool kNeedB = MODE == 0;           // cluster exchange of amax
   static constexpr bool kCluster = kNeedA || kNeedB;  // a cluster launch (peers store into this smem)
   static constexpr bool kSmall = W == 32;
   static constexpr int UC = R > 0 ? R / 2 : 1;        // c columns per row thread (two per row)
-  static constexpr int X_BYTES = kRows * kChunk * 2;  // two 64-column SW128 boxes
+  static constexpr int X_BYTES = kRows * kChunk * 2;  // two 64-column SW128 boxes (TC: then A_hi)
+  static constexpr int ALO_BYTES = kTC ? X_BYTES : 0; // TC: A_lo, same layout as the x tile
   static constexpr int P_BYTES = 512 * R;             // P^T: [kb][hi, lo] boxes of R rows x 128 B
   static constexpr int V_BYTES = 512 * R;             // V hi/lo: 2 boxes of 128 rows x 2R B
   static constexpr int CH_BYTES = kChunk * 8;         // chan * hscale and its negation
-  static constexpr int OFF_P = X_BYTES;
-  static constexpr int OFF_V = OFF_P + P_BYTES;
+  static constexpr int OFF_ALO = X_BYTES;
+  static constexpr int OFF_P = X_BYTES + ALO_BYTES;
+  static constexpr int OFF_V = kTC ? OFF_P : OFF_P + P_BYTES;  // TC: a load carries P or V, never both
   static constexpr int OFF_CH = OFF_V + V_BYTES;
   static constexpr int SLOT = (OFF_CH + CH_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_UA = 2 * SLOT;             // c hi/lo: A operand of the deflation
+  static constexpr int OFF_H = 2 * SLOT;              // TC: H_b blocks of one chunk, bf16 [128][128]
+  static constexpr int H_BYTES = kTC ? kRows * kChunk * 2 : 0;
+  static constexpr int OFF_UA = OFF_H + H_BYTES;      // c hi/lo (TC: -c): A operand of the deflation
   static constexpr int UA_BYTES = 512 * R;
   // Cluster sum of c, reduce-scatter then all-gather, both pushed with remote
   // stores: RS[rank][row in slice][R] receives the partials of this CTA's row
   // slice from every rank; UG[row][R + 4] receives the summed rows.
-  static constexpr int OFF_RS = OFF_UA + UA_BYTES;
+  // TC: RS and UG live in the two A_lo areas, which the rows write only after the
+  // exchange (and which no TMA load touches)
   static constexpr int RS_BYTES = kProj ? kRows * R * 4 : 0;
   static constexpr int UG_STRIDE = R + 4;
-  static constexpr int OFF_UG = OFF_RS + RS_BYTES;
   static constexpr int UG_BYTES = kProj ? kRows * UG_STRIDE * 4 : 0;
-  static constexpr int OFF_BAR = OFF_UG + UG_BYTES;
+  static constexpr int OFF_RS = kTC ? OFF_ALO : OFF_UA + UA_BYTES;
+  static constexpr int OFF_UG = kTC ? SLOT + OFF_ALO : OFF_RS + RS_BYTES;
+  static constexpr int OFF_BAR = kTC ? OFF_UA + UA_BYTES : OFF_UG + UG_BYTES;
   static constexpr int OFF_RED = OFF_BAR + 128;       // warp maxima [0, 8), CTA maxima by rank [8, 16)
   static constexpr int SMEM = OFF_RED + 128 + 1024;
-  static constexpr uint32_t TMEM_COLS = 256;          // D2 [0, 128), T P^T hi | lo [128, 128 + 2R)
+  // TMEM: D2 [0, 128) (TC: two Z accumulators [0, 256)), then T P^T hi | lo (2R columns)
+  static constexpr uint32_t U_COL = kTC ? 256 : 128;
+  static constexpr uint32_t TMEM_COLS = (kTC && R > 0) ? 512 : 256;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(!kTC || (RS_BYTES <= ALO_BYTES && UG_BYTES <= ALO_BYTES), "exchange areas fit in A_lo");
   static_assert(!kSmall || MODE == 0, "the small layout is a Fused-only form");
 };
 
@@ -183,6 +195,37 @@ __device__ __forceinline__ void rotate_cols(const uint8_t* xs, const float* chan
   }
 }
 
+// Tensor-core rotation, row side: this thread's W columns [W*s0, W*s0 + W) of
+// tile row `row`: a = T * (chan * hscale) in fp32, split a = hi + lo into bf16
+// (round to nearest; lo = bf16(a - hi)), hi written over T in place (the same
+// swizzled position, which only this thread reads) and lo at that position of
+// the A_lo tile.  The MMA then forms (A_hi + A_lo) H_b.
+template <int W>
+__device__ __forceinline__ void split_cols(uint8_t* xs, uint8_t* lo_tile, const float* chan, int row, int s0) {
+  const int col = s0 * W;
+#pragma unroll
+  for (int g = 0; g < W / 8; ++g) {
+    const int cg = col + 8 * g;  // 64-column box cg / 64, 16-byte chunk (cg % 64) / 8
+    const int off = (cg >> 6) * 16384 + row * 128 + ((((cg & 63) >> 3) ^ (row & 7)) << 4);
+    const uint4 w = *reinterpret_cast<const uint4*>(xs + off);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    const float4 c0 = *reinterpret_cast<const float4*>(chan + cg);
+    const float4 c1 = *reinterpret_cast<const float4*>(chan + cg + 4);
+    const float2 cc[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
+                          make_float2(c1.z, c1.w)};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = f2_mul(make_float2(__uint_as_float(ws[e] << 16), __uint_as_float(ws[e] & 0xffff0000u)), cc[e]);
+      hw[e] = bf16x2_rn(a.x, a.y);
+      const float2 r = f2_sub(a, make_float2(__uint_as_float(hw[e] << 16), __uint_as_float(hw[e] & 0xffff0000u)));
+      lw[e] = bf16x2_rn(r.x, r.y);
+    }
+    *reinterpret_cast<uint4*>(xs + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
 // Quantise this thread's W values of row `row`, chunk columns starting at `col`.
 template <int W>
 __device__ __forceinline__ void quantise_cols(const PrologueParams& p, const float (&v)[W], int row, int col,
@@ -246,7 +289,7 @@ template <int R, int MODE>
 __device__ __forceinline__ Sched schedule(int nch) {
   Sched s;
   const bool proj = R > 0 && MODE != 2;
-  s.merged = proj && nch == 1;
+  s.merged = proj && nch == 1 && MODE == 0;  // the tensor-core rotation keeps P and V in one area
   s.nproj = (proj && !s.merged) ? nch : 0;
   s.zsweeps = (MODE == 0 && nch > 1) ? 2 : 1;
   s.total = s.nproj + s.zsweeps * nch;
@@ -288,9 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + 2;    // [2] MMA and row warps done with the slot
   uint64_t* u_full = bars + 4;   // projection MMAs done
   uint64_t* ua_full = bars + 5;  // row warps wrote c hi/lo
-  uint64_t* d2_full = bars + 6;  // deflation MMAs of a chunk done
-  uint64_t* d2_free = bars + 7;  // row warps read the deflation result
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* d2_full = bars + 6;  // [2] deflation (TC: Z) MMAs of a chunk done; one buffer unless TC
+  uint64_t* d2_free = bars + 8;  // [2] row warps read that result
+  uint64_t* a_ready = bars + 10; // [2] TC: row warps wrote A_hi / A_lo of the slot
+  uint64_t* h_full = bars + 12;  // TC: H_b landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -303,12 +348,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kRowWarps + (C::kMMA ? 1 : 0));
+      // TC: the MMA warp is the last reader of a slot (the rows read T before it)
+      mbar_init(&empty[i], C::kTC ? 1 : kRowWarps + (C::kMMA ? 1 : 0));
+      mbar_init(&d2_full[i], 1);
+      mbar_init(&d2_free[i], kRowWarps);
+      mbar_init(&a_ready[i], kRowWarps);
     }
     mbar_init(u_full, 1);
     mbar_init(ua_full, kRowWarps);
-    mbar_init(d2_full, 1);
-    mbar_init(d2_free, kRowWarps);
+    mbar_init(h_full, 1);
     fence_barrier_init();
   }
   if constexpr (C::kMMA) {
@@ -333,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (MODE == 1) griddep_wait();
   griddep_launch_dependents();
   const uint32_t d2_tmem = tmem;
-  const uint32_t u_tmem = tmem + 128;
+  const uint32_t u_tmem = tmem + C::U_COL;
 
   if (warp >= kProdWarp && warp < kMmaWarp) {
     // ------------------------------------------------------------ producers
@@ -343,6 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (R > 0) {
         tma_prefetch_desc(&maps.p_hi); tma_prefetch_desc(&maps.p_lo);
         tma_prefetch_desc(&maps.v_hi); tma_prefetch_desc(&maps.v_lo);
+      }
+    }
+    if constexpr (C::kTC) {
+      // H_b (a layer constant) once, both 64-column boxes
+      if (my_slot == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(h_full, C::H_BYTES);
+        __syncwarp();
+        if (lane < 2) tma_load_2d(smem + C::OFF_H + lane * 16384, &maps.h, h_full, 64 * lane, 0);
       }
     }
     int last = -1;
@@ -421,6 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     pass_b();
     __syncwarp();
     if (lane == 0 && last >= 0) mbar_wait(&full[last & 1], (last >> 1) & 1, p.err, DEVERR_DRAIN_WAIT);
+    if constexpr (C::kTC)
+      if (lane == 0 && my_slot == 0) mbar_wait(h_full, 0, p.err, DEVERR_DRAIN_WAIT);
     __syncwarp();
     if constexpr (C::kCluster) cluster_wait();  // the last barrier arrived at (B, else A2)
   } else if (warp == kMmaWarp) {
@@ -464,45 +522,95 @@ __global__ void __launch_bounds__(kThreads, 1)
         cluster_wait();
         cluster_arrive();  // A2
       }
-      // deflation of one chunk: D2[128 x 128] = c (hi/lo) . V_chunk^T (hi/lo)
-      const uint32_t sbo_u = 8u * 2u * R;
-      const uint32_t swz_u = umma_swizzle_code(2 * R);
-      auto deflate = [&]() {
-        const int slot = i & 1;
-        if (!mbar_wait(&full[slot], (i >> 1) & 1, p.err, DEVERR_MMA_WAIT)) return false;
-        if (!mbar_wait(d2_free, (j & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) return false;
-        tc_fence_after();
-        const uint32_t vs = smem_u32(smem + slot * C::SLOT + C::OFF_V);
-        const uint32_t ua = smem_u32(smem + C::OFF_UA);
+      if constexpr (C::kTC) {
+        // Z of chunk c = (A_hi + A_lo) H_b - c V^T into TMEM buffer c % 2, once the
+        // rows have written A of the chunk's slot and read the buffer's last Z
+        auto zmma = [&](int c) {
+          const int li = sch.nproj + c, slot = li & 1, db = c & 1;
+          if (!mbar_wait(&full[slot], (li >> 1) & 1, p.err, DEVERR_MMA_WAIT)) return false;
+          if (!mbar_wait(&a_ready[slot], (c >> 1) & 1, p.err, DEVERR_MMA_WAIT)) return false;
+          if (!mbar_wait(&d2_free[db], ((c >> 1) & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) return false;
+          tc_fence_after();
+          const uint32_t d = d2_tmem + 128u * db;
+          const uint32_t xs = smem_u32(smem + slot * C::SLOT), hs = smem_u32(smem + C::OFF_H);
 #pragma unroll
-        for (int k = 0; k < R / 16; ++k) {
-          const uint64_t ah = smem_desc(ua + k * 32, 16, sbo_u, swz_u);
-          const uint64_t al = smem_desc(ua + 256 * R + k * 32, 16, sbo_u, swz_u);
-          const uint64_t bh = smem_desc(vs + k * 32, 16, sbo_u, swz_u);
-          const uint64_t bl = smem_desc(vs + 256 * R + k * 32, 16, sbo_u, swz_u);
-          mma_bf16(d2_tmem, al, bh, idesc_bf16(128, 128), k > 0 ? 1u : 0u);
-          mma_bf16(d2_tmem, ah, bl, idesc_bf16(128, 128), 1u);
-          mma_bf16(d2_tmem, ah, bh, idesc_bf16(128, 128), 1u);
+          for (int part = 0; part < 2; ++part)  // A_hi, then A_lo
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t a = smem_desc(xs + part * C::OFF_ALO + kb * 16384 + k * 32, 16, 1024, 2);
+                const uint64_t b = smem_desc(hs + kb * 16384 + k * 32, 16, 1024, 2);
+                mma_bf16(d, a, b, idesc_bf16(128, 128), (part | kb | k) ? 1u : 0u);
+              }
+          if constexpr (R > 0) {
+            // + (-c)(V^T): UA holds -c, split hi/lo like V
+            const uint32_t sbo_u = 8u * 2u * R;
+            const uint32_t swz_u = umma_swizzle_code(2 * R);
+            const uint32_t vs = xs + C::OFF_V;
+            const uint32_t ua = smem_u32(smem + C::OFF_UA);
+#pragma unroll
+            for (int k = 0; k < R / 16; ++k) {
+              const uint64_t ah = smem_desc(ua + k * 32, 16, sbo_u, swz_u);
+              const uint64_t al = smem_desc(ua + 256 * R + k * 32, 16, sbo_u, swz_u);
+              const uint64_t bh = smem_desc(vs + k * 32, 16, sbo_u, swz_u);
+              const uint64_t bl = smem_desc(vs + 256 * R + k * 32, 16, sbo_u, swz_u);
+              mma_bf16(d, al, bh, idesc_bf16(128, 128), 1u);
+              mma_bf16(d, ah, bl, idesc_bf16(128, 128), 1u);
+              mma_bf16(d, ah, bh, idesc_bf16(128, 128), 1u);
+            }
+          }
+          tc_commit(&d2_full[db]);
+          tc_commit(&empty[slot]);
+          return true;
+        };
+        if (lane == 0) {
+          if constexpr (R > 0) ok = ok && mbar_wait(ua_full, 0, p.err, DEVERR_MMA_WAIT);
+          ok = ok && mbar_wait(h_full, 0, p.err, DEVERR_MMA_WAIT);
+          for (int c = 0; ok && c < nch; ++c) ok = zmma(c);
         }
-        tc_commit(d2_full);
-        tc_commit(&empty[slot]);
-        ++i;
-        ++j;
-        return true;
-      };
-      if (lane == 0) {
-        ok = ok && mbar_wait(ua_full, 0, p.err, DEVERR_MMA_WAIT);
-        for (int c = 0; ok && c < nch; ++c) ok = deflate();
-      }
-      __syncwarp();
-      if constexpr (C::kNeedB) {
-        cluster_wait();    // A2
-        cluster_arrive();  // B
-      }
-      if (sch.zsweeps == 2) {
-        if (lane == 0)
-          for (int c = 0; ok && c < nch; ++c) ok = deflate();
         __syncwarp();
+      } else {
+        // deflation of one chunk: D2[128 x 128] = c (hi/lo) . V_chunk^T (hi/lo)
+        const uint32_t sbo_u = 8u * 2u * R;
+        const uint32_t swz_u = umma_swizzle_code(2 * R);
+        auto deflate = [&]() {
+          const int slot = i & 1;
+          if (!mbar_wait(&full[slot], (i >> 1) & 1, p.err, DEVERR_MMA_WAIT)) return false;
+          if (!mbar_wait(d2_free, (j & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) return false;
+          tc_fence_after();
+          const uint32_t vs = smem_u32(smem + slot * C::SLOT + C::OFF_V);
+          const uint32_t ua = smem_u32(smem + C::OFF_UA);
+  #pragma unroll
+          for (int k = 0; k < R / 16; ++k) {
+            const uint64_t ah = smem_desc(ua + k * 32, 16, sbo_u, swz_u);
+            const uint64_t al = smem_desc(ua + 256 * R + k * 32, 16, sbo_u, swz_u);
+            const uint64_t bh = smem_desc(vs + k * 32, 16, sbo_u, swz_u);
+            const uint64_t bl = smem_desc(vs + 256 * R + k * 32, 16, sbo_u, swz_u);
+            mma_bf16(d2_tmem, al, bh, idesc_bf16(128, 128), k > 0 ? 1u : 0u);
+            mma_bf16(d2_tmem, ah, bl, idesc_bf16(128, 128), 1u);
+            mma_bf16(d2_tmem, ah, bh, idesc_bf16(128, 128), 1u);
+          }
+          tc_commit(d2_full);
+          tc_commit(&empty[slot]);
+          ++i;
+          ++j;
+          return true;
+        };
+        if (lane == 0) {
+          ok = ok && mbar_wait(ua_full, 0, p.err, DEVERR_MMA_WAIT);
+          for (int c = 0; ok && c < nch; ++c) ok = deflate();
+        }
+        __syncwarp();
+        if constexpr (C::kNeedB) {
+          cluster_wait();    // A2
+          cluster_arrive();  // B
+        }
+        if (sch.zsweeps == 2) {
+          if (lane == 0)
+            for (int c = 0; ok && c < nch; ++c) ok = deflate();
+          __syncwarp();
+        }
       }
     } else {
       if constexpr (C::kNeedB) {
@@ -537,8 +645,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < C::UC; ++k) u[k] = 0.0f;
     int i = 0, j = 0;
 
-    // projection-only loads: the rows do not read them
-    for (int c = 0; c < sch.nproj; ++c, ++i) {
+    // projection-only loads: the rows do not read them (TC: the MMA warp alone
+    // releases them)
+    for (int c = 0; c < sch.nproj && !C::kTC; ++c, ++i) {
       mbar_wait(&full[i & 1], (i >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[i & 1]);
@@ -628,7 +737,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int jj = 0; jj < C::UC / 8; ++jj) {
           uint4 hi, lo;
-          split8(u + 8 * jj, hi, lo);
+          float uu[8];  // TC: -c, so the Z accumulation subtracts c V^T
+#pragma unroll
+          for (int e = 0; e < 8; ++e) uu[e] = C::kTC ? -u[8 * jj + e] : u[8 * jj + e];
+          split8(uu, hi, lo);
           const int ch = uc0 / 8 + jj;
 #pragma unroll
           for (int rep = 0; rep < (C::kSmall ? 4 : 1); ++rep) {
@@ -676,11 +788,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++i;
     };
 
+    // TC: A_hi / A_lo of chunk c into its slot (the MMA warp then forms Z), and
+    // Z of chunk c read back from TMEM buffer c % 2
+    auto prep_a = [&](int c) {
+      const int li = sch.nproj + c, slot = li & 1;
+      mbar_wait(&full[slot], (li >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      uint8_t* s = smem + slot * C::SLOT;
+      if (zact) split_cols<W>(s, s + C::OFF_ALO, reinterpret_cast<const float*>(s + C::OFF_CH), zrow, s0);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_ready[slot]);
+    };
+    auto read_z = [&](int c) {
+      const int db = c & 1;
+      mbar_wait(&d2_full[db], (c >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      __syncwarp();
+      tc_fence_after();
+      if (zact) {
+#pragma unroll
+        for (int pc = 0; pc < W / 32; ++pc) {
+          uint32_t r32[32];
+          tmem_ld_32x32b_x32(d2_tmem + 128u * db + lane_base + s0 * W + pc * 32, r32);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) z[pc * 32 + k] = __uint_as_float(r32[k]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d2_free[db]);
+    };
+
     float g = 1.0f;
     if constexpr (MODE == 2) g = global_scale_from_amax(__uint_as_float(*p.amax_glob));
     float amax = 0.0f;
+    if constexpr (C::kTC) prep_a(0);
     for (int c = 0; c < nch; ++c) {
-      zchunk();
+      if constexpr (C::kTC) {
+        if (c + 1 < nch) prep_a(c + 1);
+        read_z(c);
+      } else {
+        zchunk();
+      }
       const int col = col0 + c * kChunk + s0 * W;
       if constexpr (MODE == 2) {
         if (zvalid) quantise_cols<W>(p, z, zrow_g, col, g);
