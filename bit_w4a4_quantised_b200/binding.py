@@ -34,6 +34,7 @@ SIGNATURES = {
     "qwam_plan_info": (_I, [_I, _P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                             ctypes.POINTER(_I)]),
     "qwam_device_error": (_I, [ctypes.POINTER(ctypes.c_uint32)]),
+    "qwam_selfcheck_rounding": (_I, [ctypes.POINTER(ctypes.c_uint64), ctypes.c_uint64, ctypes.c_void_p]),
     "qwam_last_error": (ctypes.c_char_p, []),
     "qwam_status_string": (ctypes.c_char_p, [_I]),
     "qwam_version": (_I, []),
@@ -255,6 +256,14 @@ def device_error() -> int:
     if st not in (0, 7):
         _check(st)
     return code.value
+
+
+def selfcheck_rounding(random_pairs: int = 1 << 26) -> list:
+    """Mismatch counts [a / 6, 1 / e, E4M3 code of u / g] of the quantiser's
+    FMA-based arithmetic against the IEEE fp32 operations (qwam_selfcheck_rounding)."""
+    out = (ctypes.c_uint64 * 3)()
+    _check(load().qwam_selfcheck_rounding(out, random_pairs, None))
+    return [int(v) for v in out]
 
 
 def version() -> int:

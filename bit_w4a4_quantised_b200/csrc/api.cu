@@ -798,6 +798,22 @@ qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* 
   return QWAM_OK;
 }
 
+qwam_status qwam_selfcheck_rounding(uint64_t* mismatches, uint64_t random_pairs, void* stream) {
+  if (!mismatches) return fail(QWAM_ERR_INVALID_ARG, "mismatches is NULL");
+  unsigned long long* d = nullptr;
+  QW_CUDA(cudaMalloc(&d, 3 * sizeof(unsigned long long)));
+  const cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaMemsetAsync(d, 0, 3 * sizeof(unsigned long long), st);
+  if (e == cudaSuccess) e = launch_rounding_check(d, random_pairs, st);
+  unsigned long long h[3] = {0, 0, 0};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h, d, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFree(d);
+  if (e != cudaSuccess) return fail(QWAM_ERR_CUDA, "rounding self-check failed: %s", cudaGetErrorString(e));
+  for (int k = 0; k < 3; ++k) mismatches[k] = h[k];
+  return QWAM_OK;
+}
+
 qwam_status qwam_device_error(uint32_t* code) {
   if (!code) return fail(QWAM_ERR_INVALID_ARG, "code is NULL");
   *code = 0;

@@ -52,6 +52,9 @@ cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r,
                             cudaStream_t st);
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st);
+// counts[0..2] += mismatches of the quantiser's a / 6 and 1 / a (every positive
+// fp32 a) and of the E4M3 code of u / g, against the IEEE fp32 operations.
+cudaError_t launch_rounding_check(unsigned long long* counts, unsigned long long n_pairs, cudaStream_t st);
 // out [K / 128][2][128] fp32: chunk c holds chan[128c..] * hscale, then its negation.
 cudaError_t launch_chan_pm(const float* chan, float hscale, int K, float* out, cudaStream_t st);
 cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_t* v_lo, cudaStream_t st);

@@ -39,7 +39,7 @@ __global__ void quantize_blocks_kernel(const float* __restrict__ T, int rows, in
       v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
     }
     uint32_t c2[2];
-    const uint32_t S = quant_block16(v, g, c2);
+    const uint32_t S = quant_block16(v, g, rcp_rn(g), c2);
     *reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2) + kb * 8) = make_uint2(c2[0], c2[1]);
     sf[sf_offset(row, kb, K)] = static_cast<uint8_t>(S);
   }
@@ -104,6 +104,49 @@ __global__ void make_proj_kernel(const float* __restrict__ V, const float* __res
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st) {
   recip_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, err);
+  return cudaGetLastError();
+}
+
+// Self-check of the quantiser's FMA-based arithmetic against the fp32 IEEE
+// operations: rcp_rn(e) vs __frcp_rn(e) and div6_rn(a) vs __fdiv_rn(a, 6) for
+// every positive finite fp32 input; the E4M3 code of u / g vs the code of
+// __fdiv_rn(u, g) for every u >= 0 at four divisors spread over the exponent
+// range and for n_pairs pseudo-random (u, g) pairs.  counts[0..2] += mismatches.
+__global__ void rounding_check_kernel(unsigned long long* counts, unsigned long long n_pairs) {
+  const unsigned long long stride = static_cast<unsigned long long>(gridDim.x) * blockDim.x;
+  const unsigned long long tid = static_cast<unsigned long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  unsigned long long bad[3] = {0, 0, 0};
+  for (unsigned long long i = tid + 1; i < 0x7f800000ull; i += stride) {
+    const float a = __uint_as_float(static_cast<uint32_t>(i));
+    bad[0] += __float_as_uint(div6_rn(a)) != __float_as_uint(__fdiv_rn(a, 6.0f));
+    bad[1] += __float_as_uint(rcp_rn(a)) != __float_as_uint(__frcp_rn(a));
+  }
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t ge = k == 0 ? 27u : (k == 1 ? 97u : (k == 2 ? 157u : 227u));  // 2^-100, 2^-30, 2^30, 2^100
+    const float g = __uint_as_float(ge << 23 | (0x2F1A5Bu * (k + 1) & 0x7FFFFFu));
+    const float y = rcp_rn(g);
+    for (unsigned long long i = tid; i < 0x7f800000ull; i += stride) {
+      const float u = __uint_as_float(static_cast<uint32_t>(i));
+      bad[2] += e4m3_of_quotient(u, g, y) != e4m3_rn_satfinite(__fdiv_rn(u, g));
+    }
+  }
+  for (unsigned long long j = tid; j < n_pairs; j += stride) {
+    // splitmix64 of the pair index: two significands and exponents
+    unsigned long long z = j * 0x9E3779B97F4A7C15ull + 0x632BE59BD9B4E019ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    const uint32_t ue = 1u + static_cast<uint32_t>((z >> 46) % 253u), ge = 1u + static_cast<uint32_t>((z >> 54) % 253u);
+    const float u = __uint_as_float((ue << 23) | static_cast<uint32_t>(z & 0x7FFFFFu));
+    const float g = __uint_as_float((ge << 23) | static_cast<uint32_t>((z >> 23) & 0x7FFFFFu));
+    bad[2] += e4m3_of_quotient(u, g, rcp_rn(g)) != e4m3_rn_satfinite(__fdiv_rn(u, g));
+  }
+  for (int k = 0; k < 3; ++k)
+    if (bad[k]) atomicAdd(&counts[k], bad[k]);
+}
+
+cudaError_t launch_rounding_check(unsigned long long* counts, unsigned long long n_pairs, cudaStream_t st) {
+  rounding_check_kernel<<<148 * 8, 256, 0, st>>>(counts, n_pairs);
   return cudaGetLastError();
 }
 

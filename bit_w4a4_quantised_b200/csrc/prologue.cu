@@ -229,10 +229,10 @@ __device__ __forceinline__ void split_cols(uint8_t* xs, uint8_t* lo_tile, const 
 // Quantise this thread's W values of row `row`, chunk columns starting at `col`.
 template <int W>
 __device__ __forceinline__ void quantise_cols(const PrologueParams& p, const float (&v)[W], int row, int col,
-                                              float g) {
+                                              float g, float y_g) {
   uint32_t cw[W / 8];
   uint32_t S[W / 16];
-  quant_blocks16<W / 16>(v, g, cw, S);
+  quant_blocks16<W / 16>(v, g, y_g, cw, S);
   uint32_t sfw = 0u;
 #pragma unroll
   for (int k = 0; k < W / 16; ++k) sfw |= S[k] << (8 * k);
@@ -821,6 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     float g = 1.0f;
     if constexpr (MODE == 2) g = global_scale_from_amax(__uint_as_float(*p.amax_glob));
+    float y_g = rcp_rn(g);
     float amax = 0.0f;
     if constexpr (C::kTC) prep_a(0);
     for (int c = 0; c < nch; ++c) {
@@ -832,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int col = col0 + c * kChunk + s0 * W;
       if constexpr (MODE == 2) {
-        if (zvalid) quantise_cols<W>(p, z, zrow_g, col, g);
+        if (zvalid) quantise_cols<W>(p, z, zrow_g, col, g, y_g);
       } else if (zact) {
 #pragma unroll
         for (int k = 0; k < W; ++k) amax = fmaxf(amax, fabsf(z[k]));
@@ -862,16 +863,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       float A = 0.0f;
       for (int rk = 0; rk < p.parts; ++rk) A = fmaxf(A, red[kRowWarps + rk]);
       g = global_scale_from_amax(A);
+      y_g = rcp_rn(g);
       if constexpr (R > 0) {
         if (part == 0 && uvalid) write_branch<C::UC>(p, u, R, urow_g, uc0, g);
       }
       if (part == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = g;
       if (nch == 1) {
-        if (zvalid) quantise_cols<W>(p, z, zrow_g, col0 + s0 * W, g);
+        if (zvalid) quantise_cols<W>(p, z, zrow_g, col0 + s0 * W, g, y_g);
       } else {
         for (int c = 0; c < nch; ++c) {
           zchunk();
-          if (zvalid) quantise_cols<W>(p, z, zrow_g, col0 + c * kChunk + s0 * W, g);
+          if (zvalid) quantise_cols<W>(p, z, zrow_g, col0 + c * kChunk + s0 * W, g, y_g);
         }
       }
     }

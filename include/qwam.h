@@ -176,6 +176,20 @@ qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* 
  * QWAM_ERR_TIMEOUT when *code != 0. */
 qwam_status qwam_device_error(uint32_t* code);
 
+/* Self-check of the quantiser's arithmetic on the current device.  The block
+ * scale's two divisions and the reciprocal of the scale are computed with fp32
+ * FMAs (an estimate, an exact residual, one correction) instead of the IEEE
+ * division / reciprocal sequences, with results required to be identical:
+ * mismatches[0] counts inputs where a / 6 differs from the IEEE division and
+ * mismatches[1] where 1 / e differs from the IEEE reciprocal, over every
+ * positive finite fp32 input; mismatches[2] counts (u, g) pairs whose E4M3 code
+ * of u / g differs from the code of the IEEE quotient, over every u >= 0 at four
+ * divisors and `random_pairs` pseudo-random pairs.  All zero means identical.
+ * `mismatches` is host memory with three entries.  Allocates 24 bytes of device
+ * memory and synchronises the stream.  The card (section "What ASP is...") has
+ * no counterpart; the op order it checks is the quantiser's (NVFP4 format). */
+qwam_status qwam_selfcheck_rounding(uint64_t* mismatches, uint64_t random_pairs, void* stream);
+
 /* Message for the last failing call on this thread ("" if none). */
 const char* qwam_last_error(void);
 

@@ -91,3 +91,12 @@ def test_all_zero_tensor():
     gpu, ora = run_both(T)
     assert_same(gpu, ora)
     assert ora[2] == 1.0
+
+
+def test_fma_quotients_match_ieee_ops():
+    # the quantiser's a / 6 and 1 / e (FMA-corrected) must equal the IEEE fp32
+    # division / reciprocal for every positive fp32 input, and the E4M3 code of
+    # its u / g the code of the IEEE quotient (every u at four divisors, 2^28
+    # random pairs)
+    from bit_w4a4_quantised_b200 import binding as qw
+    assert qw.selfcheck_rounding(1 << 28) == [0, 0, 0]
