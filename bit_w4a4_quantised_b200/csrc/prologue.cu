@@ -48,9 +48,6 @@ constexpr int kRows = 128;
 constexpr int kChunk = 128;
 constexpr int kRowWarps = 8;
 constexpr int kRowThreads = 32 * kRowWarps;
-constexpr int kProdWarp = 8;  // warps 8 (slot 0) and 9 (slot 1)
-constexpr int kMmaWarp = 10;
-constexpr int kThreads = 32 * 11;
 constexpr int kMaxParts = 8;
 
 // What one ring load brings in.
@@ -68,6 +65,18 @@ struct PCfg {
   static constexpr bool kNeedB = MODE == 0;           // cluster exchange of amax
   static constexpr bool kCluster = kNeedA || kNeedB;  // a cluster launch (peers store into this smem)
   static constexpr bool kSmall = W == 32;
+  // Warp roles.  Fused: rows 0-7, producers 8-9, MMA 10.  TC: split warps 0-7
+  // (A_hi / A_lo of each chunk), rows 8-15 (exchange, Z from TMEM, amax or the
+  // quantiser), producers 16-17, MMA 18, 19 spare (warpgroups of four for the
+  // register split below).
+  static constexpr int SPLIT_WARPS = kTC ? 8 : 0;
+  static constexpr int ROW0 = SPLIT_WARPS;
+  static constexpr int PROD0 = ROW0 + kRowWarps;  // one producer per ring slot
+  static constexpr int MMA_WARP = PROD0 + 2;
+  static constexpr int THREADS = 32 * (kTC ? 20 : 11);
+  // TC register split (launch: 640 threads x 96): split warps 56, rows 152,
+  // producers / MMA / spare 64; 256 x 56 + 256 x 152 + 128 x 64 = 640 x 96.
+  static constexpr int REG_SPLIT = 56, REG_ROWS = 152, REG_OTHER = 64;
   static constexpr int UC = R > 0 ? R / 2 : 1;        // c columns per row thread (two per row)
   static constexpr int X_BYTES = kRows * kChunk * 2;  // two 64-column SW128 boxes (TC: then A_hi)
   static constexpr int ALO_BYTES = kTC ? X_BYTES : 0; // TC: A_lo, same layout as the x tile
@@ -321,7 +330,7 @@ __device__ __forceinline__ int load_chunk(const Sched& s, int i, int nch) {
 }
 
 template <int R, int MODE, int W>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
     prologue_kernel(const __grid_constant__ ProMaps maps, const PrologueParams p) {
   using C = PCfg<R, MODE, W>;
   extern __shared__ uint8_t smem_raw[];
@@ -360,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if constexpr (C::kMMA) {
-    if (warp == kMmaWarp) {
+    if (warp == C::MMA_WARP) {
       tmem_alloc(tmem_slot, C::TMEM_COLS);
       tmem_relinquish();
     }
@@ -383,9 +392,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t d2_tmem = tmem;
   const uint32_t u_tmem = tmem + C::U_COL;
 
-  if (warp >= kProdWarp && warp < kMmaWarp) {
+  static_assert(!C::kTC || (C::THREADS == 640 &&
+                             256 * C::REG_SPLIT + 256 * C::REG_ROWS + 128 * C::REG_OTHER == 640 * 96),
+                "register split of the launch");
+  // Each warpgroup changes its register count at one point, at the top of its
+  // role branch (the instruction is warpgroup-wide).
+  if (warp >= C::PROD0) {
+  if constexpr (C::kTC) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_OTHER));
+  if (warp < C::MMA_WARP) {
     // ------------------------------------------------------------ producers
-    const int my_slot = warp - kProdWarp;
+    const int my_slot = warp - C::PROD0;
     if (lane == 0 && my_slot == 0) {
       tma_prefetch_desc(&maps.x);
       if constexpr (R > 0) {
@@ -481,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && my_slot == 0) mbar_wait(h_full, 0, p.err, DEVERR_DRAIN_WAIT);
     __syncwarp();
     if constexpr (C::kCluster) cluster_wait();  // the last barrier arrived at (B, else A2)
-  } else if (warp == kMmaWarp) {
+  } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if constexpr (C::kMMA) {
       bool ok = true;
@@ -620,17 +636,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if constexpr (C::kCluster) cluster_wait();  // the last barrier arrived at (B, else A2)
   } else {
+    // ------------------------------------------------------------ spare warp (TC)
+    if constexpr (C::kNeedA) {
+      cluster_wait();    // A0
+      cluster_arrive();  // A1
+      cluster_wait();
+      cluster_arrive();  // A2
+    }
+    if constexpr (C::kCluster) cluster_wait();
+  }
+  } else if (C::kTC && warp < C::ROW0) {
+    if constexpr (C::kTC) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_SPLIT));
+    // ------------------------------------------------------------ split warps (TC)
+    // A_hi / A_lo of every chunk, as soon as its load has landed; warp w takes
+    // row (w % 4) * 32 + lane, columns [64 (w / 4), 64 (w / 4) + 64).
+    const int zrow = (warp & 3) * 32 + lane, s0 = warp >> 2;
+    auto prep_a = [&](int c) {
+      const int li = sch.nproj + c, slot = li & 1;
+      mbar_wait(&full[slot], (li >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      uint8_t* s = smem + slot * C::SLOT;
+      split_cols<W>(s, s + C::OFF_ALO, reinterpret_cast<const float*>(s + C::OFF_CH), zrow, s0);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_ready[slot]);
+    };
+    // Stats: the exchange of c uses the A_lo areas and needs every thread at its
+    // cluster barriers, so these warps pass the barriers first and write A only
+    // once the rows have read the gathered c (ua_full).
+    if constexpr (C::kNeedA) {
+      cluster_wait();    // A0
+      cluster_arrive();  // A1
+      cluster_wait();
+      cluster_arrive();  // A2
+      mbar_wait(ua_full, 0, p.err, DEVERR_EPILOGUE_WAIT);
+      __syncwarp();
+    }
+    for (int c = 0; c < nch; ++c) prep_a(c);
+    __syncwarp();
+    if constexpr (C::kCluster) cluster_wait();  // A2
+  } else {
+    if constexpr (C::kTC) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_ROWS));
     // ------------------------------------------------------------ row threads
     // outputs (and the workspace they live in) may still be read by the
     // previous kernel in the stream until it has finished
     griddep_wait();
-    const int q = warp & 3;   // TMEM lane quarter this warp may access
-    const int hf = warp >> 2;
+    const int rw = warp - C::ROW0;  // row warp 0..7
+    const int q = warp & 3;         // TMEM lane quarter this warp may access
+    const int hf = rw >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     // Z work: row zrow (tile-local), columns [W * s0, W * s0 + W) of each chunk
-    const bool zact = C::kSmall ? (warp < 4) : true;
+    const bool zact = C::kSmall ? (rw < 4) : true;
     const int zrow = C::kSmall ? lane : q * 32 + lane;
-    const int s0 = C::kSmall ? warp : hf;
+    const int s0 = C::kSmall ? rw : hf;
     const int zrow_g = m0 + zrow;
     const bool zvalid = zact && zrow_g < p.rows;
     // c work: row urow, columns [uc0, uc0 + UC)
@@ -690,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cluster_arrive();  // A1
       cluster_wait();
-      for (int it = threadIdx.x; it < SL * (R / 4); it += kRowThreads) {
+      for (int it = 32 * rw + lane; it < SL * (R / 4); it += kRowThreads) {
         const int srow = it / (R / 4), c4 = it % (R / 4);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int rk = 0; rk < p.parts; ++rk) {  // rank order: deterministic
@@ -788,17 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++i;
     };
 
-    // TC: A_hi / A_lo of chunk c into its slot (the MMA warp then forms Z), and
-    // Z of chunk c read back from TMEM buffer c % 2
-    auto prep_a = [&](int c) {
-      const int li = sch.nproj + c, slot = li & 1;
-      mbar_wait(&full[slot], (li >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
-      uint8_t* s = smem + slot * C::SLOT;
-      if (zact) split_cols<W>(s, s + C::OFF_ALO, reinterpret_cast<const float*>(s + C::OFF_CH), zrow, s0);
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_ready[slot]);
-    };
+    // TC: Z of chunk c, read back from TMEM buffer c % 2
     auto read_z = [&](int c) {
       const int db = c & 1;
       mbar_wait(&d2_full[db], (c >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
@@ -823,11 +870,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (MODE == 2) g = global_scale_from_amax(__uint_as_float(*p.amax_glob));
     float y_g = rcp_rn(g);
     float amax = 0.0f;
-    if constexpr (C::kTC) prep_a(0);
     for (int c = 0; c < nch; ++c) {
       if constexpr (C::kTC) {
-        if (c + 1 < nch) prep_a(c + 1);
-        read_z(c);
+        read_z(c);  // the split warps prepare A
       } else {
         zchunk();
       }
@@ -842,18 +887,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (MODE == 0 && !C::kNeedA) cluster_wait();  // A0, before the remote stores below
     if constexpr (MODE != 2) {
       const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
-      if (lane == 0) red[warp] = __uint_as_float(wmax);
+      if (lane == 0) red[rw] = __uint_as_float(wmax);
       named_bar(1, kRowThreads);
-      if (threadIdx.x < 32) {
+      if (rw == 0) {
         float cmax = red[0];
 #pragma unroll
         for (int w = 1; w < kRowWarps; ++w) cmax = fmaxf(cmax, red[w]);
         if constexpr (MODE == 1) {
-          if (threadIdx.x == 0) atomicMax(p.amax_glob, __float_as_uint(cmax));
-        } else if (threadIdx.x < p.parts) {
+          if (lane == 0) atomicMax(p.amax_glob, __float_as_uint(cmax));
+        } else if (lane < p.parts) {
           // push this CTA's maximum into slot [8 + rank] of every rank
           const uint32_t slot = smem_u32(red + kRowWarps + cluster_rank());
-          dsmem_st_f32(dsmem_addr(slot, static_cast<uint32_t>(threadIdx.x)), cmax);
+          dsmem_st_f32(dsmem_addr(slot, static_cast<uint32_t>(lane)), cmax);
         }
       }
     }
@@ -867,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (R > 0) {
         if (part == 0 && uvalid) write_branch<C::UC>(p, u, R, urow_g, uc0, g);
       }
-      if (part == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = g;
+      if (part == 0 && blockIdx.y == 0 && rw == 0 && lane == 0) *p.g_out = g;
       if (nch == 1) {
         if (zvalid) quantise_cols<W>(p, z, zrow_g, col0 + s0 * W, g, y_g);
       } else {
@@ -878,13 +923,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if constexpr (MODE == 2) {
-      if (part == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = g;
+      if (part == 0 && blockIdx.y == 0 && rw == 0 && lane == 0) *p.g_out = g;
     }
   }
   tc_fence_before();
   __syncthreads();
   if constexpr (C::kMMA) {
-    if (warp == kMmaWarp) {
+    if (warp == C::MMA_WARP) {
       __syncwarp();
       tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -901,7 +946,7 @@ cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p, cudaStream_
   if (p.parts < 1 || p.parts > kMaxParts || (p.parts & (p.parts - 1))) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.parts, (p.rows + kRows - 1) / kRows, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
