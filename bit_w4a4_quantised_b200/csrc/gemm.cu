@@ -469,12 +469,14 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
       __syncwarp();
       tc_fence_after();
       if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
-        // drain: y = bf16(acc * gs + bias).  The four warps of a column half
-        // stage 64 columns of their 128 rows (128B swizzle) and one thread
-        // stores them with one TMA box.  Every 64-column block but the last
-        // goes out before the accumulator is released; the last waits in
-        // registers until the staging blocks are free.  The half's named
-        // barrier is reached by all four warps on every path.
+        // drain: y = bf16(acc * gs + bias).  The whole column half is read out
+        // of TMEM and packed to bf16 pairs in registers first, so the
+        // accumulator goes back to the MMA warp before any store is issued
+        // (a TMA store can hold its thread while the engine is busy with the
+        // operand loads).  Then the four warps of a column half stage 64
+        // columns of their 128 rows at a time (128B swizzle) and one thread
+        // stores them with one TMA box.  The half's named barrier is reached
+        // by all four warps on every path.
         constexpr int NH = HC / 64;
         const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC;
         auto chunk = [&](int k) { return reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)); };
@@ -487,36 +489,14 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
                             fma_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]), gs, bw.w));
         };
         auto half_sync = [&]() { named_bar(1 + half, 128); };
-        auto store_block = [&](int hh) {
-          fence_proxy_async();
-          half_sync();
-          if (store_issuer && ok) {
-            tma_store_2d(&tmY, stg_half, c0 + hh * 64, tc.m0);
-            bulk_commit();
-          }
-        };
+        uint4 v[HC / 8];
 #pragma unroll
-        for (int hh = 0; hh < NH - 1; ++hh) {
-          if (store_issuer) bulk_wait_read<0>();  // the staging blocks are free
-          half_sync();
-#pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(taddr + (2 * hh + q2) * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 4; ++j) *chunk(4 * q2 + j) = convert(r, 2 * hh + q2, j);
-          }
-          store_block(hh);
-        }
-        uint4 last[8];
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
+        for (int qq = 0; qq < HC / 32; ++qq) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + (2 * (NH - 1) + q2) * 32, r);
+          tmem_ld_32x32b_x32(taddr + qq * 32, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) last[4 * q2 + j] = convert(r, 2 * (NH - 1) + q2, j);
+          for (int j = 0; j < 4; ++j) v[4 * qq + j] = convert(r, qq, j);
         }
         tc_fence_before();
         __syncwarp();
@@ -524,11 +504,19 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
           if constexpr (PAIR) mbar_arrive_cluster(lead(acc_empty));
           else mbar_arrive(acc_empty);
         }
-        if (store_issuer) bulk_wait_read<0>();
-        half_sync();
 #pragma unroll
-        for (int k = 0; k < 8; ++k) *chunk(k) = last[k];
-        store_block(NH - 1);
+        for (int hh = 0; hh < NH; ++hh) {
+          if (store_issuer) bulk_wait_read<0>();  // the staging blocks are free
+          half_sync();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) *chunk(k) = v[8 * hh + k];
+          fence_proxy_async();
+          half_sync();
+          if (store_issuer && ok) {
+            tma_store_2d(&tmY, stg_half, c0 + hh * 64, tc.m0);
+            bulk_commit();
+          }
+        }
       } else if constexpr (EPI == static_cast<int>(GemmEpilogue::RawF32)) {
         // fp32 out: direct row stores
 #pragma unroll 1
