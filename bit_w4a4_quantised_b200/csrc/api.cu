@@ -484,6 +484,15 @@ qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, flo
   return QWAM_OK;
 }
 
+// y [M, N] bf16 for the TMA store of the bf16 epilogue: 128-row boxes of 64
+// columns (128B swizzle), or of 32 columns (64B swizzle) on CTA pairs (a
+// 16 KB staging area; a fifth operand stage in the room this frees measured
+// slower than four).
+qwam_status make_y_map(CUtensorMap* m, void* y, int N, int M, bool pair) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, static_cast<uint64_t>(N) * 2, pair ? 32 : 64, 128,
+                  pair ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
   const Plan pl = plan_gemm(M, h->N, h->K);
   const Layout lay = layout_for(M, h->K, h->r);
@@ -503,8 +512,7 @@ qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
     maps.l = maps.b;
   }
   if (pl.splits == 1)
-    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B));
+    QW_TRY(make_y_map(&maps.y, y, h->N, M, pl.pair));
   else
     maps.y = maps.a;
   GemmParams p{};
@@ -615,8 +623,7 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
     maps.l = maps.b;
   }
   if (pl.splits == 1)
-    QW_TRY(make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B));
+    QW_TRY(make_y_map(&maps.y, y, h->N, M, pl.pair));
   else
     maps.y = maps.a;
   GemmParams p{};

@@ -69,13 +69,15 @@ struct Cfg {
   static constexpr int CP_WARP0 = NPROD + 1;
   static constexpr int EPI_WARP0 = CP_WARP0 + kCopyWarps;
   static constexpr int THREADS = 32 * (EPI_WARP0 + kEpiWarps);
+  static constexpr int REG_OTHER = 96, REG_EPI = 160;       // per thread after setmaxnreg
   static constexpr int A_BYTES = kBM * ROWB;
   static constexpr int B_BYTES = HB * ROWB;
   static constexpr int SF_BYTES = (1 + NSFB) * SF_BLK;
   static constexpr int STAGE_TX = A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int U_BYTES = kBM * 64;
   static constexpr int L_BYTES = HB * 64;
-  static constexpr int STG_BYTES = 4096;                    // per epilogue warp: 32 rows x 128 B
+  static constexpr int SCOLS = PAIR ? 32 : 64;              // columns of one y store box
+  static constexpr int STG_BYTES = 32 * SCOLS * 2;          // per epilogue warp: 32 rows x SCOLS bf16
   static constexpr int BIAS_BYTES = BN;                     // per epilogue warp: BN / 2 bf16
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -239,6 +241,15 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     return r;
   };
 
+  // Warps [0, EPI_WARP0) are two warpgroups (producers + MMA, copy warps) that
+  // need few registers; the two epilogue warpgroups hold a column half of the
+  // accumulator as packed bf16.  setmaxnreg moves registers between them:
+  // 256 x REG_OTHER + 256 x REG_EPI = 512 x 128, the launch's total.  It is
+  // the first instruction of each branch (warpgroup-wide).
+  static_assert(C::EPI_WARP0 == 8 && C::THREADS == 512, "two warpgroups each side");
+  static_assert(256 * (C::REG_OTHER + C::REG_EPI) <= 512 * 128, "register split");
+  if (warp < C::EPI_WARP0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_OTHER));
   if (warp < C::NPROD) {
     // ------------------------------------------------ producers: warp w issues stages g = w mod NPROD
     if (lane == 0 && warp == 0) {
@@ -401,7 +412,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     }
     __syncwarp();
     cluster_tail();
-  } else if (warp < C::EPI_WARP0) {
+  } else {
     // ------------------------------------------------ scale copies: smem stage -> TMEM slot (rank 0 of a pair)
     const int cw = warp - C::CP_WARP0;
     if (lane == 0 && leader) {
@@ -435,7 +446,9 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     }
     __syncwarp();
     cluster_tail();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_EPI));
     // ------------------------------------------------ epilogue
     const int ew = warp - C::EPI_WARP0;  // 0..7
     const int qd = warp & 3;             // TMEM lane quarter this warp may access
@@ -473,13 +486,16 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         // of TMEM and packed to bf16 pairs in registers first, so the
         // accumulator goes back to the MMA warp before any store is issued
         // (a TMA store can hold its thread while the engine is busy with the
-        // operand loads).  Then the four warps of a column half stage 64
-        // columns of their 128 rows at a time (128B swizzle) and one thread
-        // stores them with one TMA box.  The half's named barrier is reached
-        // by all four warps on every path.
-        constexpr int NH = HC / 64;
+        // operand loads).  Then the four warps of a column half stage SCOLS
+        // columns of their 128 rows at a time (128B swizzle for 64 columns,
+        // 64B for 32) and one thread stores them with one TMA box.  The half's
+        // named barrier is reached by all four warps on every path.
+        constexpr int NH = HC / C::SCOLS, CPR = C::SCOLS / 8;  // store rounds, 16-byte chunks per row
         const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + half * HC;
-        auto chunk = [&](int k) { return reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)); };
+        auto chunk = [&](int k) {
+          const int sw = C::SCOLS == 64 ? (lane & 7) : ((lane >> 1) & 3);
+          return reinterpret_cast<uint4*>(stg + lane * (2 * C::SCOLS) + ((k ^ sw) << 4));
+        };
         // 8 columns (qq * 32 + 8 j ..) of a 32-column TMEM load -> 4 bf16 pairs
         auto convert = [&](const uint32_t* r, int qq, int j) {
           const uint4 bw = bias_s[qq * 4 + j];
@@ -509,11 +525,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
           if (store_issuer) bulk_wait_read<0>();  // the staging blocks are free
           half_sync();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) *chunk(k) = v[8 * hh + k];
+          for (int k = 0; k < CPR; ++k) *chunk(k) = v[CPR * hh + k];
           fence_proxy_async();
           half_sync();
           if (store_issuer && ok) {
-            tma_store_2d(&tmY, stg_half, c0 + hh * 64, tc.m0);
+            tma_store_2d(&tmY, stg_half, c0 + hh * C::SCOLS, tc.m0);
             bulk_commit();
           }
         }

@@ -89,7 +89,7 @@ struct GemmMaps {
   CUtensorMap b;    // codes B [N, K/2] u8, box (ks/2) B x bn rows, same swizzle
   CUtensorMap u;    // branch A [M, r] bf16, box r x 128 rows
   CUtensorMap l;    // branch B [N, r] bf16, box r x bn rows
-  CUtensorMap y;    // output y [M, N] bf16, box 64 x 128 rows, 128B swizzle (bf16 epilogue)
+  CUtensorMap y;    // output y [M, N] bf16 (bf16 epilogue): box 64 x 128 rows, 128B swizzle; on CTA pairs 32 x 128, 64B swizzle
   CUtensorMap sfa;  // A scales viewed as u8 [rows * K / 16 / 256, 256], box 256 x (ks / 32): one stage of 128 rows
   CUtensorMap sfb;  // B scales, same view and box
 };

@@ -289,8 +289,12 @@ __device__ __forceinline__ void write_branch(const PrologueParams& p, const floa
 //   merged : one load (T, P, V, chan) serves the projection and the only Z sweep
 //   nproj  : projection-only loads (T, P), one per chunk
 //   zsweep : sweeps of (T, V, chan) loads over the chunks
+//   rev    : the amax sweep after a projection pass takes the chunks in reverse
+//            order, so its first loads find the chunks the projection read last
+//            still in L2 (a row slab wider than L2 holds is otherwise read twice
+//            from DRAM)
 struct Sched {
-  bool merged;
+  bool merged, rev;
   int nproj, zsweeps, total;
 };
 
@@ -302,6 +306,7 @@ __device__ __forceinline__ Sched schedule(int nch) {
   s.nproj = (proj && !s.merged) ? nch : 0;
   s.zsweeps = (MODE == 0 && nch > 1) ? 2 : 1;
   s.total = s.nproj + s.zsweeps * nch;
+  s.rev = MODE == 1 && s.nproj > 0;
   return s;
 }
 
@@ -326,7 +331,9 @@ __device__ __forceinline__ uint32_t load_bytes(uint32_t kind) {
 
 // chunk index (within this CTA) of load i
 __device__ __forceinline__ int load_chunk(const Sched& s, int i, int nch) {
-  return i < s.nproj ? i : (i - s.nproj) % nch;
+  if (i < s.nproj) return i;
+  const int c = (i - s.nproj) % nch;
+  return s.rev ? nch - 1 - c : c;
 }
 
 template <int R, int MODE, int W>
