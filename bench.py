@@ -17,6 +17,13 @@ The default workload is the action-expert attention projection
 (32 tokens, 1024 -> 1024, rank 32, Hadamard block 128).  Multi-GPU runs are
 independent replicas (the layer needs no exchange between GPUs): weak scaling.
 
+--workload c5action runs one denoising step of the action expert as a set:
+its 300 distinct linears (30 blocks x self q/k/v/o, cross q/k/v/o, ffn.0,
+ffn.2; d 1024, ffn 4096, 32 tokens, cross k/v over the 4096-token context,
+r 32) back to back in one CUDA graph, programmatic dependent launch between
+kernels; one step = the whole set, reported as aggregate GB/s against HBM
+(0.36 GB of distinct weights per step, above L2).
+
 --impl reference times the float64 CPU oracle (oracle/) on the same workload
 and metric, on this host's cores: a deliberately slow correctness reference.
 """
@@ -45,6 +52,19 @@ L2_BYTES = 126 * 10 ** 6
 
 def _c5_like(i, seed):
     return workloads.c5_layer(i, seed)
+
+
+SETS = {
+    "c5action": dict(desc="one denoising step of the action expert: 300 linears (d 1024, ffn 4096, "
+                          "32 tokens; cross k/v over the 4096-token context), r=32, b=128",
+                     unit="GB/s", steps=20, warmup=3),
+}
+
+
+def set_layers(name):
+    """Indices (into the step's 600 linears) of a layer set's members."""
+    specs = workloads.c5_layer_specs(cross_kv_context=True)
+    return [i for i, sp in enumerate(specs) if sp.name.startswith("action.")]
 
 
 WORKLOADS = {
@@ -304,12 +324,228 @@ def config_of(args, wl, shape, instances):
     return cfg
 
 
+def run_set(args, wl):
+    """A layer set (one denoising step of the action expert): every step runs
+    all of its distinct layers once, in model order, from one CUDA graph."""
+    idx = set_layers(args.workload)
+    unit = wl["unit"]
+    specs = workloads.c5_layer_specs(cross_kv_context=True)
+    shapes = [(specs[i].M, specs[i].K, specs[i].N, specs[i].r) for i in idx]
+    set_bytes = sum(layer_bytes(*sh) for sh in shapes)
+    set_flops = sum(layer_flops(*sh) for sh in shapes)
+    cfg = {"workload": f"{args.workload}: {wl['desc']}", "layers": len(idx),
+           "tokens": {"action": 32, "cross_kv_context": 4096}, "d": 1024, "ffn": 4096, "r": 32,
+           "hadamard_block": 128, "parallelism": f"replicas x{args.gpus}"}
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_set_reference(args, wl, idx, shapes, set_bytes, cfg)
+
+    import torch
+    import torch.distributed as dist
+    from bit_w4a4_quantised_b200 import binding as qw
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    steps = args.steps if args.steps is not None else wl["steps"]
+    warmup = max(3, args.warmup if args.warmup is not None else wl["warmup"])
+
+    handles, xs, ys = [], [], []
+    for i in idx:
+        c = workloads.c5_layer(i, args.seed + rank * 100003)
+        handles.append(qw.prepare_weight(torch.from_numpy(c.W).to(dev).to(torch.bfloat16),
+                                         torch.from_numpy(c.s).to(dev),
+                                         torch.from_numpy(c.V).to(dev) if c.r else None,
+                                         torch.from_numpy(c.bias).to(dev).to(torch.bfloat16), c.b))
+        xs.append(torch.from_numpy(c.x).to(dev).to(torch.bfloat16))
+        ys.append(torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev))
+    plans = [qw.plan_info(sh[0], h) for sh, h in zip(shapes, handles)]
+    n_layers = len(idx)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    def run_all(evs=None):
+        for k in range(n_layers):
+            if evs is not None:
+                evs[k][0].record()
+            qw.prologue(xs[k], handles[k])
+            if evs is not None:
+                evs[k][1].record()
+            qw.gemm(shapes[k][0], handles[k], ys[k])
+            if evs is not None:
+                evs[k][2].record()
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            run_all()
+    torch.cuda.synchronize()
+    if qw.device_error():
+        raise RuntimeError("device wait expired during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(n_layers)]
+    g_main, g_prof = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_main, stream=stream):
+        run_all()
+    with torch.cuda.graph(g_prof, stream=stream):
+        run_all(ev)
+    torch.cuda.synchronize()
+
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_uuid) as clk:
+        with torch.cuda.stream(stream):
+            t_start.record()
+            for _ in range(steps):
+                g_main.replay()
+            t_end.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    with torch.cuda.stream(stream):
+        g_prof.replay()
+    torch.cuda.synchronize()
+    if qw.device_error():
+        raise RuntimeError("device wait expired during the timed region")
+    pro_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(n_layers)]
+    gem_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(n_layers)]
+
+    # end to end through the public API: each layer's x in from pinned host
+    # memory, its y back out, every step
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = [torch.empty(y.shape, dtype=torch.bfloat16).pin_memory() for y in ys]
+    dx = [torch.empty_like(x) for x in xs]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    E = max(1, min(steps, 5))
+
+    def e2e_step():
+        for k in range(n_layers):
+            dx[k].copy_(hx[k], non_blocking=True)
+            qw.linear(dx[k], handles[k], ys[k])
+            hy[k].copy_(ys[k], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(E):
+            e2e_step()
+        e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist if world > 1 else None, dev)
+
+    peaks = measured_peaks()
+    value = per_unit(set_bytes * steps * world, ms / 1e3, unit)
+    # dominant kernel over the set: the one with more total device time;
+    # achieved = its algorithmic bytes over the set / its summed durations
+    pro_t, gem_t = sum(pro_ms), sum(gem_ms)
+    dominant = "gemm" if gem_t >= pro_t else "prologue"
+    kb = sum((gemm_bytes if dominant == "gemm" else prologue_bytes)(*sh) for sh in shapes)
+    dur = gem_t if dominant == "gemm" else pro_t
+    achieved = kb / (dur / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "peak_note": f"{peaks['source']} HBM copy bandwidth", "frac": achieved / peaks["hbm_gbs"],
+            "kernel": "fp4_gemm_kernel" if dominant == "gemm" else "prologue_kernel", "traffic": None,
+            "avg_launch_us": dur / n_layers * 1e3,
+            "duration_note": "CUDA events around each kernel of every layer, one replay of the set's graph "
+                             "with event nodes added, right after the timed region",
+            "kernel_share": {"prologue": pro_t / (pro_t + gem_t), "gemm": gem_t / (pro_t + gem_t)},
+            "set_frac": value / world / peaks["hbm_gbs"]}
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3 block-16) GEMM, fp32 accumulate; bf16 in/out; bf16 rank-r branch",
+        "data": "synthetic (seeded; shapes of the Fast-WAM action expert, random-init weights)",
+        "config": dict(cfg, l2=f"{n_layers} distinct layers, "
+                              f"{sum(0.5625 * sh[1] * sh[2] for sh in shapes) / 1e9:.2f} GB of FP4 weights "
+                              f"> 126 MB L2; CUDA graph"),
+        "per_step": {"us": ms / steps * 1e3, "alg_bytes": set_bytes, "alg_flops": set_flops,
+                     "layers_us_median": statistics.median(p + g for p, g in zip(pro_ms, gem_ms)) * 1e3},
+        "roofline": roof,
+        "e2e": {"value": per_unit(set_bytes * E * world, e2e_ms / 1e3, unit), "unit": unit,
+                "h2d_bytes_per_step": sum(2 * sh[0] * sh[1] for sh in shapes),
+                "d2h_bytes_per_step": sum(2 * sh[0] * sh[2] for sh in shapes), "steps": E},
+        "gpu_launches": sum(pl["kernels"] for pl in plans) * steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1:
+        sample = [workloads.c5_layer(idx[k], args.seed) for k in (0, 8)]
+        n, t = time_oracle(sample, args.cpu_budget)
+        sb = sum(layer_bytes(c.M, c.K, c.N, c.r) for c in sample)
+        cores = cores_used()
+        line["cpu_baseline"] = {"value": per_unit(sb / len(sample) * n, t, unit), "unit": unit,
+                                "cores": cores["blas_threads"] or cores["affinity"], "kind": "oracle",
+                                "sample": f"{n} float64 oracle calls ({t:.1f} s) alternating the set's first "
+                                          f"self-attention projection and first ffn.0 (32 tokens); weights "
+                                          f"prepared outside the clock"}
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del g_main, g_prof
+        dist.destroy_process_group()
+    return 0
+
+
+def run_set_reference(args, wl, idx, shapes, set_bytes, cfg):
+    """The oracle on a bounded sample of the set: its layers in order, as many
+    as fit in ~60 s of CPU work, reported in the set's unit."""
+    from oracle import asp
+    unit = wl["unit"]
+    t_budget = 60.0
+    n, t, nbytes = 0, 0.0, 0.0
+    while t < t_budget and n < len(idx):
+        c = workloads.c5_layer(idx[n], args.seed)
+        prep = asp.prepare_weight(c.W, c.s, c.V, c.b)
+        t0 = time.perf_counter()
+        oracle_call(prep, c)
+        t += time.perf_counter() - t0
+        nbytes += layer_bytes(c.M, c.K, c.N, c.r)
+        n += 1
+    value = per_unit(nbytes, t, unit)
+    cores = cores_used()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": 1, "warmup": 0, "ms_per_step": t / n * len(idx) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; shapes of the Fast-WAM action expert)", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores["blas_threads"] or cores["affinity"],
+                         "kind": "oracle",
+                         "sample": f"the first {n} of the set's {len(idx)} layers in model order "
+                                   f"({t:.1f} s of oracle work, bounded to ~60 s), weights prepared outside the "
+                                   f"clock; ms_per_step extrapolates to the whole set"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--workload", default="c2", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="c2", choices=sorted(WORKLOADS) + sorted(SETS))
     ap.add_argument("--impl", default="qwam", choices=["qwam", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
@@ -317,6 +553,8 @@ def main():
                     help="distinct layer instances to rotate over (default: enough to exceed L2)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
+    if args.workload in SETS:
+        return run_set(args, SETS[args.workload])
     wl = WORKLOADS[args.workload]
     probe = wl["make"](0, args.seed)
     shape = (probe.M, probe.K, probe.N, probe.r, probe.b)
