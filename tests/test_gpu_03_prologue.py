@@ -25,6 +25,11 @@ CASES = {
     "m17_r32_b1": lambda: workloads.custom(17, 256, 64, 32, 1, seed=4, n_outliers=2),
     "m64_r32_b2": lambda: workloads.custom(64, 1024, 128, 32, 2, seed=5, n_outliers=4),
     "m1_r32_b128": lambda: workloads.custom(1, 4096, 64, 32, 128, seed=6, n_outliers=8),
+    # the one-launch prologue at <= 32 rows: two chunks per CTA at r = 16,
+    # r = 0 with b = 16, eight chunks per CTA
+    "m32_k2048_r16_b64": lambda: workloads.custom(32, 2048, 96, 16, 64, seed=7, n_outliers=20),
+    "m24_k512_r0_b16": lambda: workloads.custom(24, 512, 64, 0, 16, seed=8, n_outliers=5),
+    "m9_k8192_r32_b128": lambda: workloads.custom(9, 8192, 64, 32, 128, seed=9, n_outliers=40),
 }
 
 

@@ -34,6 +34,9 @@ CASES = {
     # 256 x 256 tiles on CTA pairs (no split-K): ragged M, then ragged M and N
     "m1000_k1024_n2560_r32_b128": lambda: workloads.custom(1000, 1024, 2560, 32, 128, seed=23, n_outliers=10),
     "m1000_k768_n2320_r16_b64": lambda: workloads.custom(1000, 768, 2320, 16, 64, seed=24, n_outliers=8),
+    # 32 rows with two and four prologue chunks per CTA (action-expert FFN shapes)
+    "m32_k2048_n512_r16_b64": lambda: workloads.custom(32, 2048, 512, 16, 64, seed=25, n_outliers=20),
+    "m32_k4096_n1024_r32_b128": lambda: workloads.custom(32, 4096, 1024, 32, 128, seed=26, n_outliers=41),
 }
 
 
