@@ -22,7 +22,9 @@ its 300 distinct linears (30 blocks x self q/k/v/o, cross q/k/v/o, ffn.0,
 ffn.2; d 1024, ffn 4096, 32 tokens, cross k/v over the 4096-token context,
 r 32) back to back in one CUDA graph, programmatic dependent launch between
 kernels; one step = the whole set, reported as aggregate GB/s against HBM
-(0.36 GB of distinct weights per step, above L2).
+(0.28 GB of distinct FP4 weights per step, above L2); --workload c5action32 is the
+same set with the cross k/v projections at 32 tokens (the other reading of the
+config).
 
 --impl reference times the float64 CPU oracle (oracle/) on the same workload
 and metric, on this host's cores: a deliberately slow correctness reference.
@@ -57,14 +59,18 @@ def _c5_like(i, seed):
 SETS = {
     "c5action": dict(desc="one denoising step of the action expert: 300 linears (d 1024, ffn 4096, "
                           "32 tokens; cross k/v over the 4096-token context), r=32, b=128",
-                     unit="GB/s", steps=20, warmup=3),
+                     unit="GB/s", steps=20, warmup=3, cross_kv_context=True),
+    "c5action32": dict(desc="one denoising step of the action expert: 300 linears (d 1024, ffn 4096, "
+                            "every one at 32 tokens, cross k/v included), r=32, b=128",
+                       unit="GB/s", steps=20, warmup=3, cross_kv_context=False),
 }
 
 
-def set_layers(name):
-    """Indices (into the step's 600 linears) of a layer set's members."""
-    specs = workloads.c5_layer_specs(cross_kv_context=True)
-    return [i for i, sp in enumerate(specs) if sp.name.startswith("action.")]
+def set_layers(wl):
+    """The set's layer specs and their indices into the step's 600 linears."""
+    specs = workloads.c5_layer_specs(cross_kv_context=wl["cross_kv_context"])
+    idx = [i for i, sp in enumerate(specs) if sp.name.startswith("action.")]
+    return specs, idx
 
 
 WORKLOADS = {
@@ -327,20 +333,20 @@ def config_of(args, wl, shape, instances):
 def run_set(args, wl):
     """A layer set (one denoising step of the action expert): every step runs
     all of its distinct layers once, in model order, from one CUDA graph."""
-    idx = set_layers(args.workload)
+    specs, idx = set_layers(wl)
     unit = wl["unit"]
-    specs = workloads.c5_layer_specs(cross_kv_context=True)
+    ctx = wl["cross_kv_context"]
     shapes = [(specs[i].M, specs[i].K, specs[i].N, specs[i].r) for i in idx]
     set_bytes = sum(layer_bytes(*sh) for sh in shapes)
     set_flops = sum(layer_flops(*sh) for sh in shapes)
     cfg = {"workload": f"{args.workload}: {wl['desc']}", "layers": len(idx),
-           "tokens": {"action": 32, "cross_kv_context": 4096}, "d": 1024, "ffn": 4096, "r": 32,
+           "tokens": {"action": 32, "cross_kv": 4096 if ctx else 32}, "d": 1024, "ffn": 4096, "r": 32,
            "hadamard_block": 128, "parallelism": f"replicas x{args.gpus}"}
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         if rank != 0:
             return 0
-        return run_set_reference(args, wl, idx, shapes, set_bytes, cfg)
+        return run_set_reference(args, wl, idx, set_bytes, cfg)
 
     import torch
     import torch.distributed as dist
@@ -358,7 +364,7 @@ def run_set(args, wl):
 
     handles, xs, ys = [], [], []
     for i in idx:
-        c = workloads.c5_layer(i, args.seed + rank * 100003)
+        c = workloads.c5_layer(i, args.seed + rank * 100003, cross_kv_context=ctx)
         handles.append(qw.prepare_weight(torch.from_numpy(c.W).to(dev).to(torch.bfloat16),
                                          torch.from_numpy(c.s).to(dev),
                                          torch.from_numpy(c.V).to(dev) if c.r else None,
@@ -488,7 +494,7 @@ def run_set(args, wl):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1:
-        sample = [workloads.c5_layer(idx[k], args.seed) for k in (0, 8)]
+        sample = [workloads.c5_layer(idx[k], args.seed, cross_kv_context=ctx) for k in (0, 8)]
         n, t = time_oracle(sample, args.cpu_budget)
         sb = sum(layer_bytes(c.M, c.K, c.N, c.r) for c in sample)
         cores = cores_used()
@@ -507,7 +513,7 @@ def run_set(args, wl):
     return 0
 
 
-def run_set_reference(args, wl, idx, shapes, set_bytes, cfg):
+def run_set_reference(args, wl, idx, set_bytes, cfg):
     """The oracle on a bounded sample of the set: its layers in order, as many
     as fit in ~60 s of CPU work, reported in the set's unit."""
     from oracle import asp
@@ -515,7 +521,7 @@ def run_set_reference(args, wl, idx, shapes, set_bytes, cfg):
     t_budget = 60.0
     n, t, nbytes = 0, 0.0, 0.0
     while t < t_budget and n < len(idx):
-        c = workloads.c5_layer(idx[n], args.seed)
+        c = workloads.c5_layer(idx[n], args.seed, cross_kv_context=wl["cross_kv_context"])
         prep = asp.prepare_weight(c.W, c.s, c.V, c.b)
         t0 = time.perf_counter()
         oracle_call(prep, c)
