@@ -13,7 +13,7 @@ and the FP4 weight holds W~(I - VV^T).  The branch stays 16-bit (bf16 on the
 card; "16-bit low-rank branch" in the Q-WAM abstract) — in this float64 oracle
 it is exact.
 
-Readings of points the card leaves open (each listed in the design doc):
+Readings of points the card leaves open:
 
 * W~ = W diag(s) H: the card writes W~ = W diag(s) without H, but the branch
   pairs x~V with W~V in the same coordinates, and only with H on both sides

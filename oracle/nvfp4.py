@@ -11,8 +11,7 @@ row "numeric format"; section "Files", row for the NVFP4 checkpoint):
 * scales are stored pre-swizzled into the 128-row x 4-column tile layout that
   FP4 tensor cores consume ("SWIZZLE_32_4_4", section "Files").
 
-What the pages leave open and this oracle fixes (one reading each, listed in
-DESIGN.md):
+What the pages leave open and this oracle fixes (one reading each):
 
 * a fp32 per-tensor scale ``g = amax / (6 * 448)`` over the whole tensor;
 * the quantiser's fp32 operation order (below), with correctly rounded fp32
