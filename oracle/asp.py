@@ -105,6 +105,30 @@ def prepare_weight(W, s, V, b: int, fp4: bool = True) -> dict:
     return out
 
 
+def prepare_weight_shared(W, s, V, b: int, fp4: bool = True) -> dict:
+    """Offline side of the shared-weight arm (model card, section "What ASP
+    is, and what the deflated form means": the cheaper variant "quantises one
+    weight and stores V alone").  Reading: the one quantised weight is W~
+    itself, not deflated, and both paths use it: the FP4 product takes
+    Q(W~), and the branch weight is formed from that stored weight and V,
+    L = deq(Q(W~)) V, so nothing but the FP4 weight and V is stored.  The
+    activation side is the deflated one of the main arm."""
+    Wt = rotate_weight(W, s, b)
+    out = {"Wt": Wt}
+    if fp4:
+        codes, scales, g = nvfp4.quantize(Wt.astype(np.float32))
+        deq = nvfp4.dequantize(codes, scales, g)
+        out.update(codes=codes, scales=scales, g=g, deq=deq)
+    else:
+        deq = Wt
+        out["deq"] = deq
+    if V is None or np.asarray(V).shape[1] == 0:
+        out["L"] = np.zeros((Wt.shape[0], 0))
+    else:
+        out["L"] = deq @ np.asarray(V, dtype=np.float64)
+    return out
+
+
 def activation_prologue(x, s, V, b: int, fp4: bool = True) -> dict:
     """Per-call side: x~, u = x~V, z = x~ - u V^T, and the quantisation of z."""
     xt = rotate_activation(x, s, b)
@@ -124,10 +148,13 @@ def nvfp4_gemm(deq_a, deq_b) -> np.ndarray:
     return np.asarray(deq_a, dtype=np.float64) @ np.asarray(deq_b, dtype=np.float64).T
 
 
-def asp_linear(x, W, s, V, bias, b: int, fp4: bool = True, parts: bool = False):
+def asp_linear(x, W, s, V, bias, b: int, fp4: bool = True, parts: bool = False, variant: str = "deflated"):
     """The whole layer.  ``fp4=False`` replaces both quantisers by the identity
-    (used to pin the formula to x W^T + bias)."""
-    wp = prepare_weight(W, s, V, b, fp4=fp4)
+    (used to pin the formula to x W^T + bias).  ``variant="shared"`` takes the
+    shared-weight arm's weight side (prepare_weight_shared)."""
+    if variant not in ("deflated", "shared"):
+        raise ValueError(variant)
+    wp = (prepare_weight if variant == "deflated" else prepare_weight_shared)(W, s, V, b, fp4=fp4)
     ap = activation_prologue(x, s, V, b, fp4=fp4)
     y_fp4 = nvfp4_gemm(ap["deq"], wp["deq"])
     y_lr = ap["u"] @ wp["L"].T

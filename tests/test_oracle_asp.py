@@ -162,3 +162,68 @@ def test_c1_error_budget():
     ref = case.x.astype(np.float64) @ case.W.astype(np.float64).T + case.bias
     err = asp.rel_fro(y, ref)
     assert 1e-3 < err < 0.2
+
+
+# ---------------------------------------------------------------------------
+# The shared-weight arm (one quantised weight W~, branch weight deq(Q(W~)) V).
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("r", [16, 32])
+@pytest.mark.parametrize("b", [1, 16, 128])
+def test_shared_identity_quantiser_gives_plain_linear(r, b):
+    # z W~^T + u (W~V)^T = x~ W~^T - u V^T W~^T + u V^T W~^T = x W^T
+    rng = np.random.default_rng(100 + r + b)
+    M, K, N = 12, 256, 40
+    x = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K)) * 0.02
+    s = np.exp(rng.uniform(-1, 1, K))
+    V = np.linalg.qr(rng.standard_normal((K, r)))[0]
+    bias = rng.standard_normal(N) * 0.01
+    y = asp.asp_linear(x, W, s, V, bias, b, fp4=False, variant="shared")
+    assert asp.rel_fro(y, x @ W.T + bias) < 1e-12
+
+
+def test_shared_rank0_is_the_deflated_arm():
+    # with no subspace both arms quantise the same W~ and have no branch
+    case = workloads.custom(16, 256, 48, 0, 16, seed=101, n_outliers=2)
+    a = asp.asp_linear(case.x, case.W, case.s, None, case.bias, 16)
+    b_ = asp.asp_linear(case.x, case.W, case.s, None, case.bias, 16, variant="shared")
+    assert np.array_equal(a, b_)
+
+
+def test_shared_weight_codes_are_the_quantised_rotated_weight():
+    case = workloads.custom(8, 256, 32, 32, 16, seed=102, n_outliers=2)
+    wp = asp.prepare_weight_shared(case.W, case.s, case.V, 16)
+    c, sc, g = nvfp4.quantize(asp.rotate_weight(case.W, case.s, 16).astype(np.float32))
+    assert np.array_equal(wp["codes"], c) and np.array_equal(wp["scales"], sc) and wp["g"] == g
+    dp = asp.prepare_weight(case.W, case.s, case.V, 16)
+    assert not np.array_equal(dp["codes"], wp["codes"])      # the deflated arm quantises W_d
+
+
+def test_shared_input_in_span_uses_the_quantised_weight_columns():
+    # exact construction as for the deflated arm (b = 1, 2^k smoothing,
+    # identity-column V): z == 0, and the branch weight is the picked columns of
+    # the dequantised stored weight, so y is an explicit product of those
+    rng = np.random.default_rng(103)
+    M, K, N, r = 16, 64, 32, 8
+    cols = rng.choice(K, r, replace=False)
+    V = np.zeros((K, r))
+    V[cols, np.arange(r)] = 1.0
+    s = 2.0 ** rng.integers(-3, 4, K)
+    xt = np.zeros((M, K))
+    xt[:, cols] = rng.standard_normal((M, r))
+    x = xt * s
+    W = rng.standard_normal((N, K)) * 0.02
+    bias = rng.standard_normal(N) * 0.01
+    y, parts = asp.asp_linear(x, W, s, V, bias, 1, parts=True, variant="shared")
+    assert np.all(parts["act"]["z"] == 0) and np.array_equal(parts["y_fp4"], np.zeros((M, N)))
+    c, sc, g = nvfp4.quantize((W * s).astype(np.float32))
+    deq = nvfp4.dequantize(c, sc, g)
+    want = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            want[m, n] = sum(xt[m, cols[j]] * deq[n, cols[j]] for j in range(r)) + bias[n]
+    assert np.allclose(y, want, rtol=1e-14, atol=1e-15)
+    # the deflated arm's branch uses the exact W~V instead
+    yd = asp.asp_linear(x, W, s, V, bias, 1, variant="deflated")
+    assert np.allclose(yd, xt[:, cols] @ (W * s)[:, cols].T + bias, rtol=1e-14, atol=1e-15)
