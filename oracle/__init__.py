@@ -12,11 +12,16 @@ nvfp4
     E2M1 / E4M3 value tables, round-to-nearest-even encoders by brute-force
     table search, the fp32-exact two-level NVFP4 quantiser, dequantiser, nibble
     packing and the 128x4 scale-tile layout.
+fp8
+    The FP8 W8A8 arm's per-tensor E4M3 quantiser and its dequantisation.
 asp
     Block Hadamard, smoothing, rank-r deflation and the full layer
-    ``y = (x~V)(W~V)^T + NVFP4GEMM((I-VV^T)x~, W~(I-VV^T)) + bias`` in float64.
+    ``y = (x~V)(W~V)^T + NVFP4GEMM((I-VV^T)x~, W~(I-VV^T)) + bias`` in float64;
+    the shared-weight arm's weight side; the FP8 arm (``fmt="fp8"``).
 
-Sources: "FastWAM UR3 3-task — 4-bit quantisations" (Hugging Face model card),
+Sources: "QuantWAMs: Calibrating at the Right Granularity for World Action
+Models" (report), section "During inference" (FP8 W8A8 for the upgraded
+Linears); "FastWAM UR3 3-task — 4-bit quantisations" (Hugging Face model card),
 sections "What ASP is, and what the deflated form means" (the contract) and the
 top comparison table (numeric format), "Files" (scale swizzle), and
 "Verification — NVFP4 deflated ASP" (storage figures); "Q-WAM: 4-Bit Quantization

@@ -32,7 +32,21 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import nvfp4
+from . import fp8, nvfp4
+
+FORMATS = ("nvfp4", "fp8")
+
+
+def _quantise(T32, fmt: str) -> dict:
+    """The chosen 4-bit or 8-bit quantiser on a fp32 tensor, with its float64
+    dequantisation: NVFP4 (codes, block scales, g) or FP8 E4M3 (codes, g)."""
+    if fmt == "nvfp4":
+        codes, scales, g = nvfp4.quantize(T32)
+        return {"codes": codes, "scales": scales, "g": g, "deq": nvfp4.dequantize(codes, scales, g)}
+    if fmt == "fp8":
+        codes, g = fp8.quantize(T32)
+        return {"codes": codes, "g": g, "deq": fp8.dequantize(codes, g)}
+    raise ValueError(fmt)
 
 
 def sylvester(b: int) -> np.ndarray:
@@ -90,16 +104,16 @@ def deflate(T, V):
     return c, T - c @ V.T
 
 
-def prepare_weight(W, s, V, b: int, fp4: bool = True) -> dict:
+def prepare_weight(W, s, V, b: int, fp4: bool = True, fmt: str = "nvfp4") -> dict:
     """Offline side: W~, the exact branch L = W~V, the deflated weight
-    W_d = W~ - L V^T, and its quantisation (codes, scales, g_w)."""
+    W_d = W~ - L V^T, and its quantisation (codes, scales, g_w).  ``fp4=False``
+    replaces the quantiser by the identity; ``fmt="fp8"`` takes the FP8 arm's
+    per-tensor E4M3 quantiser instead of NVFP4."""
     Wt = rotate_weight(W, s, b)
     L, Wd = deflate(Wt, V)
     out = {"Wt": Wt, "L": L, "Wd": Wd}
     if fp4:
-        codes, scales, g = nvfp4.quantize(Wd.astype(np.float32))
-        out.update(codes=codes, scales=scales, g=g,
-                   deq=nvfp4.dequantize(codes, scales, g))
+        out.update(_quantise(Wd.astype(np.float32), fmt))
     else:
         out["deq"] = Wd
     return out
@@ -129,15 +143,14 @@ def prepare_weight_shared(W, s, V, b: int, fp4: bool = True) -> dict:
     return out
 
 
-def activation_prologue(x, s, V, b: int, fp4: bool = True) -> dict:
-    """Per-call side: x~, u = x~V, z = x~ - u V^T, and the quantisation of z."""
+def activation_prologue(x, s, V, b: int, fp4: bool = True, fmt: str = "nvfp4") -> dict:
+    """Per-call side: x~, u = x~V, z = x~ - u V^T, and the quantisation of z
+    (NVFP4, or the FP8 arm's E4M3 with ``fmt="fp8"``)."""
     xt = rotate_activation(x, s, b)
     u, z = deflate(xt, V)
     out = {"xt": xt, "u": u, "z": z}
     if fp4:
-        codes, scales, g = nvfp4.quantize(z.astype(np.float32))
-        out.update(codes=codes, scales=scales, g=g,
-                   deq=nvfp4.dequantize(codes, scales, g))
+        out.update(_quantise(z.astype(np.float32), fmt))
     else:
         out["deq"] = z
     return out
@@ -148,14 +161,22 @@ def nvfp4_gemm(deq_a, deq_b) -> np.ndarray:
     return np.asarray(deq_a, dtype=np.float64) @ np.asarray(deq_b, dtype=np.float64).T
 
 
-def asp_linear(x, W, s, V, bias, b: int, fp4: bool = True, parts: bool = False, variant: str = "deflated"):
+def asp_linear(x, W, s, V, bias, b: int, fp4: bool = True, parts: bool = False, variant: str = "deflated",
+               fmt: str = "nvfp4"):
     """The whole layer.  ``fp4=False`` replaces both quantisers by the identity
     (used to pin the formula to x W^T + bias).  ``variant="shared"`` takes the
-    shared-weight arm's weight side (prepare_weight_shared)."""
+    shared-weight arm's weight side (prepare_weight_shared).  ``fmt="fp8"`` is
+    the FP8 W8A8 arm: the same layer with both quantisers FP8 E4M3 per tensor
+    (oracle.fp8) and the product taken on those operands."""
     if variant not in ("deflated", "shared"):
         raise ValueError(variant)
-    wp = (prepare_weight if variant == "deflated" else prepare_weight_shared)(W, s, V, b, fp4=fp4)
-    ap = activation_prologue(x, s, V, b, fp4=fp4)
+    if fmt not in FORMATS or (fmt != "nvfp4" and variant != "deflated"):
+        raise ValueError(f"format {fmt!r} with variant {variant!r}")
+    if variant == "deflated":
+        wp = prepare_weight(W, s, V, b, fp4=fp4, fmt=fmt)
+    else:
+        wp = prepare_weight_shared(W, s, V, b, fp4=fp4)
+    ap = activation_prologue(x, s, V, b, fp4=fp4, fmt=fmt)
     y_fp4 = nvfp4_gemm(ap["deq"], wp["deq"])
     y_lr = ap["u"] @ wp["L"].T
     y = y_fp4 + y_lr
