@@ -28,9 +28,13 @@ SIGNATURES = {
                               ctypes.POINTER(_I), ctypes.POINTER(_F)]),
     "qwam_export_weight": (_I, [_P, _P, _P, _P, _P]),
     "qwam_debug_prepare_weight": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
+    "qwam_prepare_weight_shared": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
+    "qwam_prepare_weight_fp8": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
+    "qwam_handle_format": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "qwam_debug_prologue": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "qwam_quantize_fp32": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "qwam_fp4_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "qwam_debug_fp4_gemm_withheld": (_I, [_P, _P, _P, _P, _I, _I, _I, ctypes.c_uint64, _P, _P]),
     "qwam_plan_info": (_I, [_I, _P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                             ctypes.POINTER(_I)]),
     "qwam_device_error": (_I, [ctypes.POINTER(ctypes.c_uint32)]),
@@ -115,6 +119,15 @@ class Handle:
         _check(load().qwam_handle_info(raw, ctypes.byref(N), ctypes.byref(K), ctypes.byref(r),
                                        ctypes.byref(b), ctypes.byref(gw)))
         self.N, self.K, self.r, self.b, self.g_w = N.value, K.value, r.value, b.value, gw.value
+        fmt, var = _I(), _I()
+        _check(load().qwam_handle_format(raw, ctypes.byref(fmt), ctypes.byref(var)))
+        self.fmt = "fp8" if fmt.value == 1 else "nvfp4"
+        self.variant = "shared" if var.value == 1 else "deflated"
+
+    @property
+    def code_bytes(self) -> int:
+        """Bytes of one row of codes: K / 2 (NVFP4) or K (FP8)."""
+        return self.K if self.fmt == "fp8" else self.K // 2
 
     @property
     def raw(self) -> int:
@@ -135,8 +148,13 @@ class Handle:
             pass
 
 
-def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None) -> Handle:
-    """W bf16 [N, K], s fp32 [K], V fp32 [K, r] or None, bias bf16 [N] or None."""
+def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None, variant: str = "deflated",
+                   fmt: str = "nvfp4") -> Handle:
+    """W bf16 [N, K], s fp32 [K], V fp32 [K, r] or None, bias bf16 [N] or None.
+    variant "deflated" (qwam_prepare_weight) or "shared" (the shared-weight
+    arm, qwam_prepare_weight_shared); fmt "nvfp4" or "fp8" (the W8A8 arm,
+    qwam_prepare_weight_fp8, deflated only).  wd_out (fp32 [N, K]) receives
+    the exact quantiser input: W_d for the deflated arm, W~ for the shared one."""
     import torch
     lib = load()
     N, K = W.shape
@@ -148,11 +166,22 @@ def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None)
     if bias is not None:
         _need(bias, torch.bfloat16, (N,), "bias")
     out = _P()
-    if wd_out is None:
+    if variant not in ("deflated", "shared"):
+        raise ValueError(f"variant must be 'deflated' or 'shared', got {variant!r}")
+    if fmt not in ("nvfp4", "fp8") or (fmt == "fp8" and variant != "deflated"):
+        raise ValueError(f"format {fmt!r} with variant {variant!r}")
+    if wd_out is not None:
+        _need(wd_out, torch.float32, (N, K), "wd_out")
+    if fmt == "fp8":
+        _check(lib.qwam_prepare_weight_fp8(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
+                                           _ptr(wd_out), _stream(stream), ctypes.byref(out)))
+    elif variant == "shared":
+        _check(lib.qwam_prepare_weight_shared(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
+                                              _ptr(wd_out), _stream(stream), ctypes.byref(out)))
+    elif wd_out is None:
         _check(lib.qwam_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
                                        _stream(stream), ctypes.byref(out)))
     else:
-        _need(wd_out, torch.float32, (N, K), "wd_out")
         _check(lib.qwam_debug_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
                                              _ptr(wd_out), _stream(stream), ctypes.byref(out)))
     return Handle(out.value)
@@ -198,7 +227,7 @@ def gemm(M: int, h: Handle, y, stream=None):
 def export_weight(h: Handle, stream=None) -> dict:
     import torch
     dev = torch.device("cuda")
-    codes = torch.empty((h.N, h.K // 2), dtype=torch.uint8, device=dev)
+    codes = torch.empty((h.N, h.code_bytes), dtype=torch.uint8, device=dev)
     sf = torch.empty((-(-h.N // 128) * 128 * h.K // 16,), dtype=torch.uint8, device=dev)
     L = torch.empty((h.N, max(h.r, 1)), dtype=torch.bfloat16, device=dev)
     _check(load().qwam_export_weight(h.raw, _ptr(codes), _ptr(sf), _ptr(L) if h.r else None, _stream(stream)))
@@ -212,7 +241,7 @@ def debug_prologue(x, h: Handle, stream=None) -> dict:
     dev = x.device
     z = torch.empty((M, h.K), dtype=torch.float32, device=dev)
     u = torch.empty((M, max(h.r, 1)), dtype=torch.float32, device=dev)
-    codes = torch.empty((M, h.K // 2), dtype=torch.uint8, device=dev)
+    codes = torch.empty((M, h.code_bytes), dtype=torch.uint8, device=dev)
     sf = torch.empty((-(-M // 128) * 128 * h.K // 16,), dtype=torch.uint8, device=dev)
     ub = torch.empty((M, max(h.r, 1)), dtype=torch.bfloat16, device=dev)
     gx = torch.empty((1,), dtype=torch.float32, device=dev)
@@ -240,6 +269,17 @@ def fp4_gemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, alpha
     _check(load().qwam_fp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
                                 float(alpha), _ptr(out), _stream(stream)))
     return out
+
+
+def debug_fp4_gemm_withheld(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, wait_ns: int,
+                            stream=None) -> None:
+    """qwam_debug_fp4_gemm_withheld: the bare GEMM with a pipeline barrier that
+    never completes and every bounded wait limited to wait_ns; the caller then
+    reads the expired waits with device_error()."""
+    import torch
+    out = torch.empty((M, N), dtype=torch.float32, device=a_codes.device)
+    _check(load().qwam_debug_fp4_gemm_withheld(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
+                                               int(wait_ns), _ptr(out), _stream(stream)))
 
 
 def plan_info(M: int, h: Handle) -> dict:

@@ -21,7 +21,6 @@ namespace {
 constexpr uint32_t kMagic = 0x514d5731u;
 constexpr int kMaxDevices = 64;
 constexpr size_t kHeaderBytes = 256;  // scalars: activation amax, g_x, device error word
-constexpr int kSMs = 148;
 
 thread_local std::string g_err;
 
@@ -51,13 +50,37 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
+// SMs per device, looked up once (grids are sized in multiples of it)
+int g_sms[kMaxDevices];
+inline int sm_count(int dev) { return __atomic_load_n(&g_sms[dev], __ATOMIC_RELAXED); }
+
+// Once per process, before any launch: every warp-specialised kernel was
+// compiled to the register count its setmaxnreg split assumes.
+qwam_status kernels_ready() {
+  static std::once_flag once;
+  static bool ok = false;
+  static char msg[256];
+  std::call_once(once, [] {
+    ok = gemm_register_split_ok(msg, sizeof(msg)) && prologue_register_split_ok(msg, sizeof(msg));
+    if (!ok) cudaGetLastError();
+  });
+  if (!ok) return fail(QWAM_ERR_CUDA, "%s", msg);
+  return QWAM_OK;
+}
+
 qwam_status current_device(int* dev) {
   QW_CUDA(cudaGetDevice(dev));
   int major = 0;
   QW_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev));
   if (major != 10) return fail(QWAM_ERR_ARCH, "device %d is compute capability %d.x; this library is built for sm_100a", *dev, major);
   if (*dev < 0 || *dev >= kMaxDevices) return fail(QWAM_ERR_INVALID_ARG, "device index %d out of range", *dev);
-  return QWAM_OK;
+  if (sm_count(*dev) <= 0) {
+    int sms = 0;
+    QW_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev));
+    if (sms <= 0) return fail(QWAM_ERR_CUDA, "device %d reports %d SMs", *dev, sms);
+    __atomic_store_n(&g_sms[*dev], sms, __ATOMIC_RELAXED);
+  }
+  return kernels_ready();
 }
 
 // ---- tensor maps -----------------------------------------------------------
@@ -72,6 +95,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+PFN_cuTensorMapReplaceAddress_v12000 replace_fn() {
+  static PFN_cuTensorMapReplaceAddress_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapReplaceAddress", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapReplaceAddress_v12000>(p);
+  });
+  return fn;
+}
+
+// Point an encoded tensor map at another buffer of the same shape.
+qwam_status repoint_map(CUtensorMap* m, const void* base) {
+  auto fn = replace_fn();
+  if (!fn) return fail(QWAM_ERR_CUDA, "cuTensorMapReplaceAddress is not available from the driver");
+  CUresult r = fn(m, const_cast<void*>(base));
+  if (r != CUDA_SUCCESS) return fail(QWAM_ERR_CUDA, "cuTensorMapReplaceAddress failed with code %d", static_cast<int>(r));
+  return QWAM_OK;
 }
 
 qwam_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
@@ -113,15 +158,19 @@ qwam_status make_sf_map(CUtensorMap* m, const void* base, size_t rows_padded, in
   return make_map3(m, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Packed E2M1 operand [rows, K/2] u8 as the GEMM reads it (a unit third
-// dimension): one box per stage of ks K elements (ks / 2 bytes, one swizzle atom
-// wide) by box_rows rows.
-qwam_status make_codes_map(CUtensorMap* m, const void* base, int rows, int K, int ks, int box_rows) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows), 1};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(K / 2) * rows};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(ks / 2), static_cast<cuuint32_t>(box_rows), 1};
-  return make_map3(m, base, dims, strides, box, ks == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+// A GEMM operand [rows, row_bytes] u8 (packed E2M1, or FP8 E4M3 one byte per
+// element) as the GEMM reads it (a unit third dimension): one box per stage of
+// box_bytes per row (one 128B or 64B swizzle atom) by box_rows rows.
+qwam_status make_codes_map(CUtensorMap* m, const void* base, int rows, int row_bytes, int box_bytes, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * rows};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows), 1};
+  return make_map3(m, base, dims, strides, box,
+                   box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
+
+// Bytes of one operand row of K elements, and of one stage of ks elements.
+inline int code_bytes(int K, int fmt) { return fmt == 1 ? K : K / 2; }
 
 CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B; }
 
@@ -129,14 +178,18 @@ CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZL
 struct Plan {
   int bn, ks, k_stages, splits;
   bool pair;  // 256 x bn tiles on CTA pairs (no split-K)
+  bool fp8;   // FP8 operands
+  bool wide;  // stages of one 128B swizzle atom per row (large M), else 64B
 };
 
 // Split-K when the output tiles leave SMs idle: the largest power of two <= 8
 // (one portable cluster per tile) with splits <= k_stages and tiles * splits
 // within one wave of the SMs.  Otherwise 256-column tiles run on CTA pairs.
-Plan plan_gemm(int M, int N, int K) {
+Plan plan_gemm(int M, int N, int K, int sms, int fmt) {
   Plan p{};
-  const GemmShape sh = gemm_shape(M, N);
+  const GemmShape sh = gemm_shape(M, N, fmt == 1);
+  p.fp8 = sh.fp8;
+  p.wide = code_bytes(sh.ks, fmt) == 128;
   p.bn = sh.bn;
   p.ks = sh.ks;
   p.k_stages = (K + p.ks - 1) / p.ks;
@@ -144,7 +197,7 @@ Plan plan_gemm(int M, int N, int K) {
   const int tiles = tiles_m * ((N + p.bn - 1) / p.bn);
   p.splits = 1;
   for (int c = 8; c >= 2; c >>= 1)
-    if (c <= p.k_stages && tiles * c <= kSMs) {
+    if (c <= p.k_stages && tiles * c <= sms) {
       p.splits = c;
       break;
     }
@@ -164,7 +217,7 @@ struct Layout {
   size_t codes, sf, u, ub, total;
 };
 
-Layout layout_for(int M, int K, int r) {
+Layout layout_for(int M, int K, int r, int fmt) {
   Layout L{};
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
@@ -174,8 +227,8 @@ Layout layout_for(int M, int K, int r) {
   };
   const size_t Mp = round_up(static_cast<size_t>(M), 128);
   const size_t rr = static_cast<size_t>(std::max(r, 1));
-  L.codes = take(Mp * K / 2);
-  L.sf = take(Mp * K / 16);
+  L.codes = take(Mp * code_bytes(K, fmt));
+  L.sf = take(fmt == 1 ? 16 : Mp * K / 16);  // FP8: no block scales
   L.u = take(static_cast<size_t>(M) * rr * 4);
   L.ub = take(Mp * rr * 2);
   L.total = off;
@@ -213,19 +266,38 @@ qwam_status arena_get(int dev, size_t need, Arena** out) {
 // CTAs along K per 128-row tile of the prologue: the largest power of two
 // that divides the chunk count (K / 128), is at most 8 (one portable cluster)
 // and keeps the grid within one wave of the SMs (at least one part).
-int cluster_parts(int K, int rows) {
+int cluster_parts(int K, int rows, int sms) {
   const int chunks = K / 128;
   const int tiles = (rows + 127) / 128;
   for (int c = 8; c > 1; c >>= 1)
-    if (chunks % c == 0 && tiles * c <= kSMs) return c;
+    if (chunks % c == 0 && tiles * c <= sms) return c;
   return 1;
 }
+
+// Everything the two launches of one layer call need for a given M and scratch
+// area: the GEMM plan, the prologue's and the GEMM's tensor maps and
+// parameters.  M == -1 marks it empty.
+struct CallPlan {
+  int M = -1;
+  const uint8_t* ws = nullptr;  // scratch the maps and pointers refer to
+  const void* x = nullptr;      // buffers the x and y maps point at (nullptr: not encoded yet)
+  const void* y = nullptr;
+  Plan pl{};
+  int pro_form = 0;  // PRO_FUSED, PRO_TWO_PASS or PRO_WIDE
+  int pro_groups = 0;
+  ProMaps pmaps{};
+  PrologueParams prm{};
+  GemmMaps gmaps{};
+  GemmParams gp{};
+};
 
 }  // namespace
 
 struct qwam_layer {
   uint32_t magic;
   int N, K, r, b, dev;
+  int fmt;      // 0 NVFP4 (W4A4), 1 FP8 E4M3 (W8A8)
+  int variant;  // 0 deflated, 1 shared-weight
   uint8_t* codes;
   uint8_t* sf;
   uint16_t* L;
@@ -240,6 +312,12 @@ struct qwam_layer {
   CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256;
   CUtensorMap map_sfb_k128, map_sfb_k256_b1, map_sfb_k256_b2;  // B scales: K per stage, 128-row blocks per box
   ProMaps vmaps;  // P^T and V (hi/lo) tensor maps for the prologue; x is per call
+  // Launch arguments of the last call, kept per scratch kind (0: the growable
+  // workspace, 1: the static scratch of qwam_linear_noalloc) so that repeated
+  // calls with the same M encode no tensor map; a new x or y buffer only
+  // re-points its map.  mu orders host access to them.
+  std::mutex mu;
+  CallPlan call[2];
 };
 
 namespace {
@@ -283,30 +361,48 @@ qwam_status dmalloc(T** p, size_t bytes) {
 
 bool use_fused(int rows) { return rows <= 128; }
 
-// Stats + Quantise (any row count) or Fused (rows <= 128).  T is the bf16
-// [rows, K] input (x or W); vmaps holds the handle's V tensor maps.
-qwam_status run_rows(const void* T, PrologueParams prm, int r, const ProMaps& vmaps, bool allow_fused,
-                     uint32_t* amax, cudaStream_t st) {
-  const int K = prm.K;
-  ProMaps maps = vmaps;
-  QW_TRY(make_map(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, K, prm.rows, static_cast<uint64_t>(K) * 2, 64, 128,
-                  CU_TENSOR_MAP_SWIZZLE_128B));
-  if (r == 0) maps.p_hi = maps.p_lo = maps.v_hi = maps.v_lo = maps.x;
-  prm.amax_glob = amax;
-  prm.parts = cluster_parts(K, prm.rows);
-  prm.chunks = K / 128 / prm.parts;
-  if (allow_fused && use_fused(prm.rows)) {
+// Forms of the activation prologue: one launch for up to 128 rows; above that
+// two launches (Stats, Quantise), with the rotation folded into the tensor-core
+// operand when there is no subspace (r = 0), else the row pipeline with the
+// rank-r projection and deflation.
+enum { PRO_FUSED = 0, PRO_TWO_PASS = 1, PRO_WIDE = 2 };
+int prologue_form(int rows, int r) { return use_fused(rows) ? PRO_FUSED : (r == 0 ? PRO_WIDE : PRO_TWO_PASS); }
+
+// The launches of the row pipeline: Fused (rows <= 128, when allowed), else
+// Stats + Quantise.  prm.amax_glob is the activation / weight amax word.
+qwam_status launch_rows(const ProMaps& maps, const PrologueParams& prm, int r, bool fused, cudaStream_t st) {
+  if (fused) {
     QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Fused, st));
     return QWAM_OK;
   }
-  QW_CUDA(cudaMemsetAsync(amax, 0, sizeof(uint32_t), st));
+  QW_CUDA(cudaMemsetAsync(prm.amax_glob, 0, sizeof(uint32_t), st));
   QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Stats, st));
   QW_CUDA(launch_prologue(maps, prm, r, PrologueMode::Quantise, st));
   return QWAM_OK;
 }
 
+// x (or W) bf16 [rows, K] as the prologue's TMA reads it
+qwam_status make_rows_map(CUtensorMap* m, const void* T, int rows, int K) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, K, rows, static_cast<uint64_t>(K) * 2, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// One pass of the row pipeline over T (the weight side at prepare).
+qwam_status run_rows(const void* T, PrologueParams prm, int r, const ProMaps& vmaps, int sms, uint32_t* amax,
+                     cudaStream_t st) {
+  ProMaps maps = vmaps;
+  QW_TRY(make_rows_map(&maps.x, T, prm.rows, prm.K));
+  if (r == 0) maps.p_hi = maps.p_lo = maps.v_hi = maps.v_lo = maps.x;
+  prm.amax_glob = amax;
+  prm.parts = cluster_parts(prm.K, prm.rows, sms);
+  prm.chunks = prm.K / 128 / prm.parts;
+  return launch_rows(maps, prm, r, false, st);
+}
+
+// shared: the shared-weight arm (quantise W~ itself; L = deq(Q(W~)) V) instead
+// of the deflated one (quantise W_d = W~ - (W~V)V^T; L = W~V).
 qwam_status prepare_impl(const void* W, int N, int K, const float* s, const float* V, int r, const void* bias,
-                         int b, float* wd_out, void* stream, qwam_handle* out) {
+                         int b, float* wd_out, bool shared, int fmt, void* stream, qwam_handle* out) {
   if (!out) return fail(QWAM_ERR_INVALID_ARG, "out handle pointer is NULL");
   *out = nullptr;
   if (!W || !s) return fail(QWAM_ERR_INVALID_ARG, "W and s must be non-NULL");
@@ -319,11 +415,12 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   QW_TRY(current_device(&dev));
   cudaStream_t st = as_stream(stream);
 
-  qwam_layer* h = new qwam_layer();
-  std::memset(h, 0, sizeof(*h));
+  qwam_layer* h = new qwam_layer();  // value-initialised: every pointer and map zero
   h->magic = kMagic;
   h->N = N; h->K = K; h->r = r; h->b = b; h->dev = dev;
-  h->sf_bytes = round_up(static_cast<size_t>(N), 256) * K / 16;
+  h->fmt = fmt;
+  h->variant = shared ? 1 : 0;
+  h->sf_bytes = fmt == 1 ? 16 : round_up(static_cast<size_t>(N), 256) * K / 16;
   float* u_tmp = nullptr;
   uint32_t* scratch = nullptr;  // [0] amax, [1] err, [2] g_w (fp32)
   uint16_t *pw_hi = nullptr, *pw_lo = nullptr;  // P^T of the weight side, diag(s) H V
@@ -339,7 +436,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   };
   qwam_status s_;
   const size_t rr = static_cast<size_t>(std::max(r, 1));
-  if ((s_ = dmalloc(&h->codes, static_cast<size_t>(N) * K / 2)) != QWAM_OK ||
+  if ((s_ = dmalloc(&h->codes, static_cast<size_t>(N) * code_bytes(K, fmt))) != QWAM_OK ||
       (s_ = dmalloc(&h->sf, h->sf_bytes)) != QWAM_OK || (s_ = dmalloc(&h->L, static_cast<size_t>(N) * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->v_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->v_lo, K * rr * 2)) != QWAM_OK ||
       (s_ = dmalloc(&h->px_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->px_lo, K * rr * 2)) != QWAM_OK ||
@@ -411,7 +508,17 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   prm.g_out = reinterpret_cast<float*>(scratch + 2);
   prm.z_out = wd_out;
   prm.err = scratch + 3;
-  if ((s_ = run_rows(W, prm, r, wmaps, false, scratch, st)) != QWAM_OK) return cleanup(s_);
+  prm.fmt = fmt;
+  if (shared && r > 0) {
+    // W~ itself through the row pipeline (no projection, no deflation), then
+    // the branch weight from the stored FP4 weight
+    ProMaps w0{};
+    w0.h = h->vmaps.h;
+    if ((s_ = run_rows(W, prm, 0, w0, sm_count(dev), scratch, st)) != QWAM_OK) return cleanup(s_);
+    QW_CUDA_CLEAN(launch_dequant_project(h->codes, h->sf, prm.g_out, V, N, K, r, h->L, st));
+  } else {
+    if ((s_ = run_rows(W, prm, r, wmaps, sm_count(dev), scratch, st)) != QWAM_OK) return cleanup(s_);
+  }
   uint32_t host_scr[4] = {0, 0, 0, 0};
   QW_CUDA_CLEAN(cudaMemcpyAsync(host_scr, scratch, 16, cudaMemcpyDeviceToHost, st));
   QW_CUDA_CLEAN(cudaStreamSynchronize(st));
@@ -419,14 +526,21 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   if (host_scr[3]) return cleanup(fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired in prepare (flags 0x%x)", host_scr[3]));
   std::memcpy(&h->g_w, &host_scr[2], 4);
 
-  if ((s_ = make_codes_map(&h->map_b128_k128, h->codes, N, K, 128, 128)) != QWAM_OK ||
-      (s_ = make_codes_map(&h->map_b128_k256, h->codes, N, K, 256, 128)) != QWAM_OK ||
-      (s_ = make_codes_map(&h->map_b256_k256, h->codes, N, K, 256, 256)) != QWAM_OK)
+  // B boxes: 64-byte rows (small M) or 128-byte rows (large M), 128 or 256 rows
+  const int cb = code_bytes(K, fmt);
+  if ((s_ = make_codes_map(&h->map_b128_k128, h->codes, N, cb, 64, 128)) != QWAM_OK ||
+      (s_ = make_codes_map(&h->map_b128_k256, h->codes, N, cb, 128, 128)) != QWAM_OK ||
+      (s_ = make_codes_map(&h->map_b256_k256, h->codes, N, cb, 128, 256)) != QWAM_OK)
     return cleanup(s_);
-  if ((s_ = make_sf_map(&h->map_sfb_k128, h->sf, round_up(static_cast<size_t>(N), 256), K, 128, 1)) != QWAM_OK ||
-      (s_ = make_sf_map(&h->map_sfb_k256_b1, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 1)) != QWAM_OK ||
-      (s_ = make_sf_map(&h->map_sfb_k256_b2, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 2)) != QWAM_OK)
+  if (fmt == 1) {  // no block scales: the unread scale maps alias the codes map
+    h->map_sfb_k128 = h->map_sfb_k256_b1 = h->map_sfb_k256_b2 = h->map_b128_k128;
+  } else if ((s_ = make_sf_map(&h->map_sfb_k128, h->sf, round_up(static_cast<size_t>(N), 256), K, 128, 1)) != QWAM_OK ||
+             (s_ = make_sf_map(&h->map_sfb_k256_b1, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 1)) !=
+                 QWAM_OK ||
+             (s_ = make_sf_map(&h->map_sfb_k256_b2, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 2)) !=
+                 QWAM_OK) {
     return cleanup(s_);
+  }
   if (r > 0) {
     if ((s_ = make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r))) !=
             QWAM_OK ||
@@ -456,81 +570,136 @@ qwam_status check_linear_args(const void* x, int M, qwam_handle h) {
   return QWAM_OK;
 }
 
-qwam_status prologue_impl(const void* x, int M, qwam_handle h, float* z_out, float* u_out, cudaStream_t st,
-                          Arena** arena_out, Layout* lay_out) {
-  const Plan pl = plan_gemm(M, h->N, h->K);
-  const Layout lay = layout_for(M, h->K, h->r);
-  Arena* a = nullptr;
-  QW_TRY(arena_get(h->dev, lay.total, &a));
+// y [M, N] bf16 for the TMA store of the bf16 epilogue: 128-row boxes of 64
+// columns (128B swizzle), or of 32 columns (64B swizzle) on CTA pairs (a
+// 16 KB staging area; a fifth operand stage in the room this frees measured
+// slower than four).
+qwam_status make_y_map(CUtensorMap* m, const void* y, int N, int M, bool pair) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, static_cast<uint64_t>(N) * 2, pair ? 32 : 64, 128,
+                  pair ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Launch arguments for M rows of layer h with scratch at ws: the workspace
+// layout of layout_for (scalars at ws: amax, g_x, error word).
+qwam_status build_call(qwam_handle h, int M, uint8_t* ws, CallPlan* c) {
+  c->M = -1;
+  const int sms = sm_count(h->dev);
+  const Plan pl = plan_gemm(M, h->N, h->K, sms, h->fmt);
+  const Layout lay = layout_for(M, h->K, h->r, h->fmt);
   PrologueParams prm{};
   prm.chan = h->inv_s_pm;
   prm.rows = M;
   prm.K = h->K;
   prm.b = h->b;
   prm.hscale = 1.0f / std::sqrt(static_cast<float>(h->b));
-  prm.u_glob = reinterpret_cast<float*>(a->base + lay.u);
-  prm.codes = a->base + lay.codes;
-  prm.sf = a->base + lay.sf;
-  prm.branch = reinterpret_cast<uint16_t*>(a->base + lay.ub);
+  prm.u_glob = reinterpret_cast<float*>(ws + lay.u);
+  prm.amax_glob = reinterpret_cast<uint32_t*>(ws);
+  prm.codes = ws + lay.codes;
+  prm.sf = ws + lay.sf;
+  prm.branch = reinterpret_cast<uint16_t*>(ws + lay.ub);
   prm.branch_mode = 1;
   prm.g_other = h->g_w;
-  prm.g_out = arena_gx(*a);
-  prm.z_out = z_out;
-  prm.u_out = u_out;
-  prm.err = arena_err(*a);
-  QW_TRY(run_rows(x, prm, h->r, h->vmaps, true, arena_amax(*a), st));
-  if (arena_out) *arena_out = a;
-  if (lay_out) *lay_out = lay;
-  return QWAM_OK;
-}
+  prm.g_out = reinterpret_cast<float*>(ws + 4);
+  prm.err = reinterpret_cast<uint32_t*>(ws + 8);
+  prm.parts = cluster_parts(h->K, M, sms);
+  prm.chunks = h->K / 128 / prm.parts;
+  prm.fmt = h->fmt;
 
-// y [M, N] bf16 for the TMA store of the bf16 epilogue: 128-row boxes of 64
-// columns (128B swizzle), or of 32 columns (64B swizzle) on CTA pairs (a
-// 16 KB staging area; a fifth operand stage in the room this frees measured
-// slower than four).
-qwam_status make_y_map(CUtensorMap* m, void* y, int N, int M, bool pair) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, static_cast<uint64_t>(N) * 2, pair ? 32 : 64, 128,
-                  pair ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-qwam_status gemm_impl(int M, qwam_handle h, void* y, cudaStream_t st) {
-  const Plan pl = plan_gemm(M, h->N, h->K);
-  const Layout lay = layout_for(M, h->K, h->r);
-  Arena* a = nullptr;
-  QW_TRY(arena_get(h->dev, lay.total, &a));
-  GemmMaps maps{};
-  QW_TRY(make_codes_map(&maps.a, a->base + lay.codes, M, h->K, pl.ks, 128));
-  maps.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
-  QW_TRY(make_sf_map(&maps.sfa, a->base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks, 1));
-  maps.sfb = pl.ks == 128 ? h->map_sfb_k128 : (pl.bn == 256 ? h->map_sfb_k256_b2 : h->map_sfb_k256_b1);
-  if (h->r > 0) {
-    QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->base + lay.ub, h->r, M, h->r * 2, h->r, 128,
-                    branch_swizzle(h->r)));
-    maps.l = pl.bn == 256 && !pl.pair ? h->map_l256 : h->map_l128;
+  GemmMaps gm{};
+  QW_TRY(make_codes_map(&gm.a, ws + lay.codes, M, code_bytes(h->K, h->fmt), pl.wide ? 128 : 64, 128));
+  gm.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.wide ? h->map_b128_k256 : h->map_b128_k128);
+  if (h->fmt == 1) {  // FP8: no block scales (the unread maps alias the operands)
+    gm.sfa = gm.a;
+    gm.sfb = gm.b;
   } else {
-    maps.u = maps.a;
-    maps.l = maps.b;
+    QW_TRY(make_sf_map(&gm.sfa, ws + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks, 1));
+    gm.sfb = !pl.wide ? h->map_sfb_k128 : (pl.bn == 256 ? h->map_sfb_k256_b2 : h->map_sfb_k256_b1);
   }
-  if (pl.splits == 1)
-    QW_TRY(make_y_map(&maps.y, y, h->N, M, pl.pair));
-  else
-    maps.y = maps.a;
-  GemmParams p{};
-  p.M = M; p.N = h->N; p.K = h->K;
-  p.k_stages = pl.k_stages;
-  p.splits = pl.splits;
-  p.sfa = a->base + lay.sf;
-  p.sfb = h->sf;
-  p.g_a_ptr = arena_gx(*a);
-  p.g_b = h->g_w;
-  p.has_branch = h->r > 0;
-  p.branch_k = h->r;
-  p.bias = h->bias;
-  p.y = y;
-  p.err = arena_err(*a);
-  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks, pl.pair}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
-                      st));
+  if (h->r > 0) {
+    QW_TRY(make_map(&gm.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + lay.ub, h->r, M, h->r * 2, h->r, 128,
+                    branch_swizzle(h->r)));
+    gm.l = pl.bn == 256 && !pl.pair ? h->map_l256 : h->map_l128;
+  } else {
+    gm.u = gm.a;
+    gm.l = gm.b;
+  }
+  gm.y = gm.a;  // split-K writes y with plain stores; otherwise encoded by bind_y
+  GemmParams gp{};
+  gp.M = M; gp.N = h->N; gp.K = h->K;
+  gp.k_stages = pl.k_stages;
+  gp.splits = pl.splits;
+  gp.sfa = ws + lay.sf;
+  gp.sfb = h->sf;
+  gp.g_a_ptr = prm.g_out;
+  gp.g_b = h->g_w;
+  gp.has_branch = h->r > 0;
+  gp.branch_k = h->r;
+  gp.bias = h->bias;
+  gp.err = prm.err;
+  gp.sms = sms;
+
+  c->pl = pl;
+  c->pro_form = prologue_form(M, h->r);
+  c->pro_groups = wide_prologue_groups(M, h->K, sms);
+  c->pmaps = h->vmaps;
+  c->prm = prm;
+  c->gmaps = gm;
+  c->gp = gp;
+  c->x = c->y = nullptr;
+  c->ws = ws;
+  c->M = M;
   return QWAM_OK;
+}
+
+// The cached arguments for (M, ws), rebuilt when either changed.
+qwam_status call_for(qwam_handle h, int M, uint8_t* ws, CallPlan* c) {
+  if (c->M == M && c->ws == ws) return QWAM_OK;
+  return build_call(h, M, ws, c);
+}
+
+qwam_status bind_x(qwam_handle h, CallPlan* c, const void* x) {
+  if (x == c->x) return QWAM_OK;
+  if (c->x) {
+    QW_TRY(repoint_map(&c->pmaps.x, x));
+  } else {
+    QW_TRY(make_rows_map(&c->pmaps.x, x, c->M, h->K));
+    if (h->r == 0) c->pmaps.p_hi = c->pmaps.p_lo = c->pmaps.v_hi = c->pmaps.v_lo = c->pmaps.x;  // unread
+  }
+  c->x = x;
+  return QWAM_OK;
+}
+
+qwam_status bind_y(qwam_handle h, CallPlan* c, void* y) {
+  c->gp.y = y;
+  if (y == c->y || c->pl.splits > 1) {
+    c->y = y;
+    return QWAM_OK;
+  }
+  if (c->y) QW_TRY(repoint_map(&c->gmaps.y, y));
+  else QW_TRY(make_y_map(&c->gmaps.y, y, h->N, c->M, c->pl.pair));
+  c->y = y;
+  return QWAM_OK;
+}
+
+qwam_status launch_call_prologue(const CallPlan& c, const PrologueParams& prm, int r, cudaStream_t st) {
+  if (c.pro_form == PRO_WIDE) {
+    QW_CUDA(cudaMemsetAsync(prm.amax_glob, 0, sizeof(uint32_t), st));
+    QW_CUDA(launch_prologue_wide(c.pmaps.x, prm, PrologueMode::Stats, c.pro_groups, st));
+    QW_CUDA(launch_prologue_wide(c.pmaps.x, prm, PrologueMode::Quantise, c.pro_groups, st));
+    return QWAM_OK;
+  }
+  return launch_rows(c.pmaps, prm, r, c.pro_form == PRO_FUSED, st);
+}
+
+qwam_status launch_call_gemm(const CallPlan& c, cudaStream_t st) {
+  QW_CUDA(launch_gemm(c.gmaps, c.gp, GemmShape{c.pl.bn, c.pl.ks, c.pl.pair, c.pl.fp8},
+                      c.pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
+  return QWAM_OK;
+}
+
+// The workspace arena of the handle's device, grown to hold M rows.
+qwam_status workspace_for(qwam_handle h, int M, Arena** a) {
+  return arena_get(h->dev, layout_for(M, h->K, h->r, h->fmt).total, a);
 }
 
 }  // namespace
@@ -557,10 +726,18 @@ uint8_t* g_static_base[kMaxDevices];  // this device's address of g_static_scrat
 
 // Set-up, once per device, with that device current: look up the device
 // address of the scratch and clear its header (the device error word must
-// start at zero; the other scalars are written before they are read).
-qwam_status static_scratch(int dev, uint8_t** out) {
+// start at zero; the other scalars are written before they are read).  The
+// clearing runs on the legacy stream and synchronises the device, which a
+// stream capture cannot hold: a first call whose stream is being captured is
+// refused.
+qwam_status static_scratch(int dev, cudaStream_t st, uint8_t** out) {
   std::lock_guard<std::mutex> lock(g_static_mu);
   if (!g_static_base[dev]) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    QW_CUDA(cudaStreamIsCapturing(st, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(QWAM_ERR_INVALID_ARG,
+                  "the first qwam_linear_noalloc call on a device sets up its scratch and must not be stream-captured");
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess || !p) {
@@ -582,66 +759,19 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes at most %d rows, got M=%d", kStaticMaxRows, M);
   if (h->K > kStaticMaxK)
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes K <= %d, this layer has K=%d", kStaticMaxK, h->K);
-  const Plan pl = plan_gemm(M, h->N, h->K);
-  const Layout lay = layout_for(M, h->K, h->r);
+  const Layout lay = layout_for(M, h->K, h->r, h->fmt);
   if (lay.total > kStaticBytes)
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc needs %zu bytes of scratch, the static scratch holds %zu",
                 lay.total, kStaticBytes);
   uint8_t* base = nullptr;
-  QW_TRY(static_scratch(h->dev, &base));
-  uint32_t* amax = reinterpret_cast<uint32_t*>(base);
-  float* g_x = reinterpret_cast<float*>(base + 4);
-  uint32_t* err = reinterpret_cast<uint32_t*>(base + 8);
-
-  PrologueParams prm{};
-  prm.chan = h->inv_s_pm;
-  prm.rows = M;
-  prm.K = h->K;
-  prm.b = h->b;
-  prm.hscale = 1.0f / std::sqrt(static_cast<float>(h->b));
-  prm.u_glob = reinterpret_cast<float*>(base + lay.u);
-  prm.codes = base + lay.codes;
-  prm.sf = base + lay.sf;
-  prm.branch = reinterpret_cast<uint16_t*>(base + lay.ub);
-  prm.branch_mode = 1;
-  prm.g_other = h->g_w;
-  prm.g_out = g_x;
-  prm.err = err;
-  QW_TRY(run_rows(x, prm, h->r, h->vmaps, true, amax, st));
-
-  GemmMaps maps{};
-  QW_TRY(make_codes_map(&maps.a, base + lay.codes, M, h->K, pl.ks, 128));
-  maps.b = pl.bn == 256 && !pl.pair ? h->map_b256_k256 : (pl.ks == 256 ? h->map_b128_k256 : h->map_b128_k128);
-  QW_TRY(make_sf_map(&maps.sfa, base + lay.sf, round_up(static_cast<size_t>(M), 128), h->K, pl.ks, 1));
-  maps.sfb = pl.ks == 128 ? h->map_sfb_k128 : (pl.bn == 256 ? h->map_sfb_k256_b2 : h->map_sfb_k256_b1);
-  if (h->r > 0) {
-    QW_TRY(make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base + lay.ub, h->r, M, h->r * 2, h->r, 128,
-                    branch_swizzle(h->r)));
-    maps.l = pl.bn == 256 && !pl.pair ? h->map_l256 : h->map_l128;
-  } else {
-    maps.u = maps.a;
-    maps.l = maps.b;
-  }
-  if (pl.splits == 1)
-    QW_TRY(make_y_map(&maps.y, y, h->N, M, pl.pair));
-  else
-    maps.y = maps.a;
-  GemmParams p{};
-  p.M = M; p.N = h->N; p.K = h->K;
-  p.k_stages = pl.k_stages;
-  p.splits = pl.splits;
-  p.sfa = base + lay.sf;
-  p.sfb = h->sf;
-  p.g_a_ptr = g_x;
-  p.g_b = h->g_w;
-  p.has_branch = h->r > 0;
-  p.branch_k = h->r;
-  p.bias = h->bias;
-  p.y = y;
-  p.err = err;
-  QW_CUDA(launch_gemm(maps, p, GemmShape{pl.bn, pl.ks, pl.pair}, pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16,
-                      st));
-  return QWAM_OK;
+  QW_TRY(static_scratch(h->dev, st, &base));
+  std::lock_guard<std::mutex> lock(h->mu);
+  CallPlan& c = h->call[1];
+  QW_TRY(call_for(h, M, base, &c));
+  QW_TRY(bind_x(h, &c, x));
+  QW_TRY(bind_y(h, &c, y));
+  QW_TRY(launch_call_prologue(c, c.prm, h->r, st));
+  return launch_call_gemm(c, st);
 }
 
 }  // namespace
@@ -650,13 +780,32 @@ extern "C" {
 
 qwam_status qwam_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
                                 const void* bias_bf16, int hadamard_block, void* stream, qwam_handle* out) {
-  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, nullptr, stream, out);
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, nullptr, false, 0, stream, out);
+}
+
+qwam_status qwam_prepare_weight_shared(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                       const void* bias_bf16, int hadamard_block, float* Wt_f32, void* stream,
+                                       qwam_handle* out) {
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, Wt_f32, true, 0, stream, out);
+}
+
+qwam_status qwam_prepare_weight_fp8(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                    const void* bias_bf16, int hadamard_block, float* Wd_f32, void* stream,
+                                    qwam_handle* out) {
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, Wd_f32, false, 1, stream, out);
+}
+
+qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant) {
+  if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
+  if (fmt) *fmt = h->fmt;
+  if (variant) *variant = h->variant;
+  return QWAM_OK;
 }
 
 qwam_status qwam_debug_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
                                       const void* bias_bf16, int hadamard_block, float* Wd_f32, void* stream,
                                       qwam_handle* out) {
-  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, Wd_f32, stream, out);
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, Wd_f32, false, 0, stream, out);
 }
 
 qwam_status qwam_destroy(qwam_handle h) {
@@ -673,7 +822,13 @@ qwam_status qwam_destroy(qwam_handle h) {
 qwam_status qwam_prologue(const void* x_bf16, int M, qwam_handle h, void* stream) {
   QW_TRY(check_linear_args(x_bf16, M, h));
   if (M == 0) return QWAM_OK;
-  return prologue_impl(x_bf16, M, h, nullptr, nullptr, as_stream(stream), nullptr, nullptr);
+  Arena* a = nullptr;
+  QW_TRY(workspace_for(h, M, &a));
+  std::lock_guard<std::mutex> lock(h->mu);
+  CallPlan& c = h->call[0];
+  QW_TRY(call_for(h, M, a->base, &c));
+  QW_TRY(bind_x(h, &c, x_bf16));
+  return launch_call_prologue(c, c.prm, h->r, as_stream(stream));
 }
 
 qwam_status qwam_gemm(int M, qwam_handle h, void* y_bf16, void* stream) {
@@ -682,7 +837,13 @@ qwam_status qwam_gemm(int M, qwam_handle h, void* y_bf16, void* stream) {
   if (M == 0) return QWAM_OK;
   if (!y_bf16) return fail(QWAM_ERR_INVALID_ARG, "y is NULL");
   if (!aligned16(y_bf16)) return fail(QWAM_ERR_ALIGN, "y must be 16-byte aligned");
-  return gemm_impl(M, h, y_bf16, as_stream(stream));
+  Arena* a = nullptr;
+  QW_TRY(workspace_for(h, M, &a));
+  std::lock_guard<std::mutex> lock(h->mu);
+  CallPlan& c = h->call[0];
+  QW_TRY(call_for(h, M, a->base, &c));
+  QW_TRY(bind_y(h, &c, y_bf16));
+  return launch_call_gemm(c, as_stream(stream));
 }
 
 qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream) {
@@ -691,8 +852,16 @@ qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, 
   if (!y_bf16) return fail(QWAM_ERR_INVALID_ARG, "y is NULL");
   if (!aligned16(y_bf16)) return fail(QWAM_ERR_ALIGN, "y must be 16-byte aligned");
   if (y_bf16 == x_bf16) return fail(QWAM_ERR_INVALID_ARG, "y must not alias x");
-  QW_TRY(prologue_impl(x_bf16, M, h, nullptr, nullptr, as_stream(stream), nullptr, nullptr));
-  return gemm_impl(M, h, y_bf16, as_stream(stream));
+  Arena* a = nullptr;
+  QW_TRY(workspace_for(h, M, &a));
+  const cudaStream_t st = as_stream(stream);
+  std::lock_guard<std::mutex> lock(h->mu);
+  CallPlan& c = h->call[0];
+  QW_TRY(call_for(h, M, a->base, &c));
+  QW_TRY(bind_x(h, &c, x_bf16));
+  QW_TRY(bind_y(h, &c, y_bf16));
+  QW_TRY(launch_call_prologue(c, c.prm, h->r, st));
+  return launch_call_gemm(c, st);
 }
 
 qwam_status qwam_linear_noalloc(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream) {
@@ -717,8 +886,10 @@ qwam_status qwam_handle_info(qwam_handle h, int* N, int* K, int* r, int* b, floa
 qwam_status qwam_export_weight(qwam_handle h, void* codes, void* scales, void* L_bf16, void* stream) {
   QW_TRY(check_handle(h));
   cudaStream_t st = as_stream(stream);
-  if (codes) QW_CUDA(cudaMemcpyAsync(codes, h->codes, static_cast<size_t>(h->N) * h->K / 2, cudaMemcpyDeviceToDevice, st));
-  if (scales)
+  if (codes)
+    QW_CUDA(cudaMemcpyAsync(codes, h->codes, static_cast<size_t>(h->N) * code_bytes(h->K, h->fmt),
+                            cudaMemcpyDeviceToDevice, st));
+  if (scales && h->fmt == 0)
     QW_CUDA(cudaMemcpyAsync(scales, h->sf, round_up(static_cast<size_t>(h->N), 128) * h->K / 16, cudaMemcpyDeviceToDevice, st));
   if (L_bf16 && h->r > 0)
     QW_CUDA(cudaMemcpyAsync(L_bf16, h->L, static_cast<size_t>(h->N) * h->r * 2, cudaMemcpyDeviceToDevice, st));
@@ -733,10 +904,22 @@ qwam_status qwam_debug_prologue(const void* x_bf16, int M, qwam_handle h, float*
     return fail(QWAM_ERR_ALIGN, "debug outputs must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
   Arena* a = nullptr;
-  Layout lay{};
-  QW_TRY(prologue_impl(x_bf16, M, h, z_f32, u_f32, st, &a, &lay));
-  if (codes) QW_CUDA(cudaMemcpyAsync(codes, a->base + lay.codes, static_cast<size_t>(M) * h->K / 2, cudaMemcpyDeviceToDevice, st));
-  if (scales)
+  QW_TRY(workspace_for(h, M, &a));
+  const Layout lay = layout_for(M, h->K, h->r, h->fmt);
+  {
+    std::lock_guard<std::mutex> lock(h->mu);
+    CallPlan& c = h->call[0];
+    QW_TRY(call_for(h, M, a->base, &c));
+    QW_TRY(bind_x(h, &c, x_bf16));
+    PrologueParams prm = c.prm;  // with the debug exports of z and u
+    prm.z_out = z_f32;
+    prm.u_out = u_f32;
+    QW_TRY(launch_call_prologue(c, prm, h->r, st));
+  }
+  if (codes)
+    QW_CUDA(cudaMemcpyAsync(codes, a->base + lay.codes, static_cast<size_t>(M) * code_bytes(h->K, h->fmt),
+                            cudaMemcpyDeviceToDevice, st));
+  if (scales && h->fmt == 0)
     QW_CUDA(cudaMemcpyAsync(scales, a->base + lay.sf, round_up(static_cast<size_t>(M), 128) * h->K / 16,
                             cudaMemcpyDeviceToDevice, st));
   if (ubr_bf16 && h->r > 0)
@@ -759,8 +942,11 @@ qwam_status qwam_quantize_fp32(const float* T, int rows, int K, void* codes, voi
   return QWAM_OK;
 }
 
-qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales,
-                          int M, int N, int K, float alpha, float* out_f32, void* stream) {
+namespace {
+
+qwam_status fp4_gemm_impl(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales, int M,
+                          int N, int K, float alpha, float* out_f32, uint64_t wait_ns, uint32_t withheld,
+                          cudaStream_t st) {
   if (!a_codes || !a_scales || !b_codes || !b_scales || !out_f32) return fail(QWAM_ERR_INVALID_ARG, "NULL argument");
   if (M < 1 || N < 16 || N % 16 || K < 128 || K % 128) return fail(QWAM_ERR_SHAPE, "bad GEMM shape M=%d N=%d K=%d", M, N, K);
   if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(out_f32))
@@ -770,9 +956,11 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   Arena* a = nullptr;
   QW_TRY(arena_get(dev, kHeaderBytes, &a));
   const GemmShape sh = gemm_shape(M, N);
+  if (withheld && sh.pair)
+    return fail(QWAM_ERR_SHAPE, "the wait-expiry check runs on single-CTA tiles (M <= 128 or N < 256)");
   GemmMaps maps{};
-  QW_TRY(make_codes_map(&maps.a, a_codes, M, K, sh.ks, 128));
-  QW_TRY(make_codes_map(&maps.b, b_codes, N, K, sh.ks, sh.pair ? sh.bn / 2 : sh.bn));
+  QW_TRY(make_codes_map(&maps.a, a_codes, M, K / 2, sh.ks / 2, 128));
+  QW_TRY(make_codes_map(&maps.b, b_codes, N, K / 2, sh.ks / 2, sh.pair ? sh.bn / 2 : sh.bn));
   maps.u = maps.a;
   maps.l = maps.b;
   maps.y = maps.a;
@@ -789,15 +977,33 @@ qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void*
   p.g_b = 1.0f;
   p.out_f32 = out_f32;
   p.err = arena_err(*a);
-  QW_CUDA(launch_gemm(maps, p, sh, GemmEpilogue::RawF32, as_stream(stream)));
+  p.sms = sm_count(dev);
+  p.wait_ns = wait_ns;
+  p.withheld_bytes = withheld;
+  QW_CUDA(launch_gemm(maps, p, sh, GemmEpilogue::RawF32, st));
   return QWAM_OK;
+}
+
+}  // namespace
+
+qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales,
+                          int M, int N, int K, float alpha, float* out_f32, void* stream) {
+  return fp4_gemm_impl(a_codes, a_scales, b_codes, b_scales, M, N, K, alpha, out_f32, 0, 0, as_stream(stream));
+}
+
+qwam_status qwam_debug_fp4_gemm_withheld(const void* a_codes, const void* a_scales, const void* b_codes,
+                                         const void* b_scales, int M, int N, int K, uint64_t wait_ns, float* out_f32,
+                                         void* stream) {
+  if (wait_ns < 1000 || wait_ns > 1000000000ull)
+    return fail(QWAM_ERR_INVALID_ARG, "wait_ns=%llu must lie in [1 us, 1 s]", static_cast<unsigned long long>(wait_ns));
+  return fp4_gemm_impl(a_codes, a_scales, b_codes, b_scales, M, N, K, 1.0f, out_f32, wait_ns, 16u, as_stream(stream));
 }
 
 qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* splits, int* bn) {
   if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
   if (M < 0) return fail(QWAM_ERR_SHAPE, "M=%d must be >= 0", M);
   const bool f = use_fused(M);
-  const Plan pl = plan_gemm(std::max(M, 1), h->N, h->K);
+  const Plan pl = plan_gemm(std::max(M, 1), h->N, h->K, sm_count(h->dev), h->fmt);
   if (kernels) *kernels = M == 0 ? 0 : (f ? 2 : 3);
   if (fused) *fused = f ? 1 : 0;
   if (splits) *splits = pl.splits;

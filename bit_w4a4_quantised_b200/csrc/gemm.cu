@@ -39,6 +39,7 @@
 // now idle operand ring; the owner sums the splits in order and writes y.
 // Every mbarrier wait is bounded.  No TMA multicast.
 #include <algorithm>
+#include <cstdio>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -51,17 +52,20 @@ constexpr int kEpiWarps = 8;
 constexpr int kCopyWarps = 4;
 constexpr int kScaleSlots = 4;  // TMEM scale ring, one stage per slot
 
-template <int BN, int KS, bool PAIR = false>
+// F8: the FP8 W8A8 arm (E4M3 operands, kind::f8f6f4, one byte per element, no
+// block scales); otherwise NVFP4 (packed E2M1, E4M3 scale per 16 in TMEM).
+template <int BN, int KS, bool PAIR = false, bool F8 = false>
 struct Cfg {
   static constexpr int TM = PAIR ? 2 * kBM : kBM;          // rows of an output tile
   static constexpr int HB = PAIR ? BN / 2 : BN;             // B (and L) rows held by one CTA
-  static constexpr int ROWB = KS / 2;                       // operand bytes per row per stage
-  static constexpr int K64 = KS / 64;                       // MMAs per stage
+  static constexpr int ROWB = F8 ? KS : KS / 2;             // operand bytes per row per stage
+  static constexpr int KM = F8 ? KS / 32 : KS / 64;         // MMAs per stage (K 32 for FP8, 64 for FP4)
+  static constexpr int K64 = KS / 64;                       // K64 steps of a stage (FP4 scale blocks)
   static constexpr uint32_t SWZ = ROWB == 128 ? 2u : 4u;    // UMMA layout: 128B / 64B swizzle
-  static constexpr int STAGES = PAIR ? 4 : (KS == 256 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
-  static constexpr int NSFB = BN / 128;                     // 128-row scale blocks of B
-  static constexpr int SF_BLK = K64 * 512;                  // one 128-row scale block of a stage
-  static constexpr int NBOX = 4;                            // boxes per stage: A, B, A scales, B scales
+  static constexpr int STAGES = PAIR ? 4 : (ROWB == 128 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
+  static constexpr int NSFB = F8 ? 0 : BN / 128;            // 128-row scale blocks of B
+  static constexpr int SF_BLK = F8 ? 0 : K64 * 512;         // one 128-row scale block of a stage
+  static constexpr int NBOX = F8 ? 2 : 4;                   // boxes per stage: A, B (, A scales, B scales)
   // producer warps, taking stages in turn (three keep the CTA at 16 warps, so
   // the epilogue keeps 128 registers)
   static constexpr int NPROD = STAGES < 3 ? STAGES : 3;
@@ -72,7 +76,7 @@ struct Cfg {
   static constexpr int REG_OTHER = 96, REG_EPI = 160;       // per thread after setmaxnreg
   static constexpr int A_BYTES = kBM * ROWB;
   static constexpr int B_BYTES = HB * ROWB;
-  static constexpr int SF_BYTES = (1 + NSFB) * SF_BLK;
+  static constexpr int SF_BYTES = F8 ? 0 : (1 + NSFB) * SF_BLK;
   static constexpr int STAGE_TX = A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int U_BYTES = kBM * 64;
   static constexpr int L_BYTES = HB * 64;
@@ -94,7 +98,7 @@ struct Cfg {
   // steps of A (4 columns) then of B (BN / 32 columns).
   static constexpr int SF_A_COLS = K64 * 4;
   static constexpr int SF_COLS = SF_A_COLS + K64 * (BN / 32);
-  static constexpr int TMEM_USED = BN + kScaleSlots * SF_COLS;
+  static constexpr int TMEM_USED = BN + (F8 ? 0 : kScaleSlots * SF_COLS);
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -119,13 +123,13 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n,
   return {(rest % tiles_m) * tm, (rest / tiles_m % tiles_n) * bn, sp};
 }
 
-template <int BN, int KS, int EPI, bool PAIR>
-__global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
+template <int BN, int KS, int EPI, bool PAIR, bool F8>
+__global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmSA,
                     const __grid_constant__ CUtensorMap tmSB, const GemmParams p) {
-  using C = Cfg<BN, KS, PAIR>;
+  using C = Cfg<BN, KS, PAIR, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES] operands and scales landed
@@ -140,10 +144,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
   constexpr bool kClusterK = EPI == static_cast<int>(GemmEpilogue::SplitK);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t wlim = p.wait_ns ? p.wait_ns : kWaitLimitNs;
   const int tiles_m = (p.M + C::TM - 1) / C::TM;
   const int tiles_n = (p.N + BN - 1) / BN;
   const int n_tiles = tiles_m * tiles_n * p.splits;
-  const int k64_total = p.K / 64;
+  const int k64_total = p.K / (F8 ? 32 : 64);  // MMA K steps over the whole K
   // CTA pair: rank 0 issues the MMAs and the scale copies for both CTAs; each
   // CTA loads its own 128 rows of A and its half of the B rows, and every load
   // of either CTA counts its bytes on rank 0's barrier.
@@ -236,8 +241,8 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     Range r;
     r.s_begin = split * p.k_stages / p.splits;
     r.n_st = (split + 1) * p.k_stages / p.splits - r.s_begin;
-    r.k64_begin = r.s_begin * C::K64;
-    r.n_k64 = min(r.n_st * C::K64, k64_total - r.k64_begin);
+    r.k64_begin = r.s_begin * C::KM;
+    r.n_k64 = min(r.n_st * C::KM, k64_total - r.k64_begin);
     return r;
   };
 
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         // branch operands of this tile, once the previous tile's branch MMAs are done
         int bok = 1;
         if (lane == 0) {
-          bok = (nbranch == 0 || mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_PRODUCER_WAIT)) ? 1 : 0;
+          bok = (nbranch == 0 || mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_PRODUCER_WAIT, wlim)) ? 1 : 0;
           if (bok && leader)
             mbar_arrive_expect_tx(branch_full, static_cast<uint32_t>((PAIR ? 2 : 1) * (kBM + C::HB) * p.branch_k * 2));
         }
@@ -307,7 +312,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         const uint32_t ph = (g / C::STAGES) & 1;
         uint8_t* const dst = smem + dst_base + st * dst_step;
         int wok = 1;
-        if (lane == 0) wok = mbar_wait(&empty[st], ph ^ 1u, p.err, DEVERR_PRODUCER_WAIT) ? 1 : 0;
+        if (lane == 0) wok = mbar_wait(&empty[st], ph ^ 1u, p.err, DEVERR_PRODUCER_WAIT, wlim) ? 1 : 0;
         wok = __shfl_sync(0xffffffffu, wok, 0);
         if (!wok) {
           ok = false;
@@ -324,7 +329,8 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
           cy = 2 * kst * C::K64;
           cz = lane == 2 ? tc.m0 / kBM : tc.n0 / 128;
         }
-        if (lane == 0 && leader) mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * C::STAGE_TX);
+        if (lane == 0 && leader)
+          mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * C::STAGE_TX + (g == 0 ? p.withheld_bytes : 0u));
         __syncwarp();
         auto load = [&]() {
           if constexpr (PAIR) tma_load_3d_pair(dst, map, lead(&full[st]), cx, cy, cz);
@@ -348,17 +354,17 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     // every copy this warp started must land before the CTA exits (in a pair
     // rank 0 counts them; every MMA commit to this CTA's barriers must arrive)
     if (lane == 0) {
-      if (leader && last >= 0) mbar_wait(&full[last % C::STAGES], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
-      if (leader && nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
-      if (PAIR && last >= 0) mbar_wait(&empty[last % C::STAGES], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT);
-      if (PAIR && nbranch > 0) mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT);
+      if (leader && last >= 0) mbar_wait(&full[last % C::STAGES], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT, wlim);
+      if (leader && nbranch > 0) mbar_wait(branch_full, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT, wlim);
+      if (PAIR && last >= 0) mbar_wait(&empty[last % C::STAGES], (last / C::STAGES) & 1, p.err, DEVERR_DRAIN_WAIT, wlim);
+      if (PAIR && nbranch > 0) mbar_wait(branch_empty, (nbranch - 1) & 1, p.err, DEVERR_DRAIN_WAIT, wlim);
     }
     __syncwarp();
     cluster_tail();
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------ MMA issuer (rank 0 of a pair)
     if (lane == 0 && leader) {
-      const uint32_t idesc_fp4 = idesc_mxf4(C::TM, BN);
+      const uint32_t idesc_fp4 = F8 ? idesc_f8e4m3(C::TM, BN) : idesc_mxf4(C::TM, BN);
       const uint32_t idesc_br = idesc_bf16(C::TM, BN);
       const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
       const uint32_t sbo = 8u * p.branch_k * 2u;
@@ -369,11 +375,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         const TileCoord tc = coord(t);
         const Range rg = range_of(tc.split);
         // the epilogue must have drained the previous tile's accumulator
-        if (!mbar_wait(acc_empty, (tl & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) break;
+        if (!mbar_wait(acc_empty, (tl & 1) ^ 1u, p.err, DEVERR_MMA_WAIT, wlim)) break;
         tc_fence_after();
         uint32_t accum = 0;
         if (p.has_branch && tc.split == 0) {
-          if (!mbar_wait(branch_full, nbranch & 1, p.err, DEVERR_BRANCH_WAIT)) break;
+          if (!mbar_wait(branch_full, nbranch & 1, p.err, DEVERR_BRANCH_WAIT, wlim)) break;
           tc_fence_after();
           for (int kk = 0; kk < p.branch_k / 16; ++kk) {
             const uint64_t ud = smem_desc(us + kk * 32, 16, sbo, layout), ld = smem_desc(ls + kk * 32, 16, sbo, layout);
@@ -386,8 +392,8 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         }
         for (int i = 0; i < rg.n_st; ++i, ++g) {
           const int st = g % C::STAGES, sl = g % kScaleSlots;
-          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_MMA_WAIT) ||
-              !mbar_wait(&sf_ready[sl], (g / kScaleSlots) & 1, p.err, DEVERR_MMA_WAIT)) {
+          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_MMA_WAIT, wlim) ||
+              (!F8 && !mbar_wait(&sf_ready[sl], (g / kScaleSlots) & 1, p.err, DEVERR_MMA_WAIT, wlim))) {
             ok = false;
             break;
           }
@@ -395,16 +401,22 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
           const uint32_t a_s = smem_u32(smem + C::OFF_A + st * C::A_BYTES);
           const uint32_t b_s = smem_u32(smem + C::OFF_B + st * C::B_BYTES);
           const uint32_t sfa = tmem + BN + sl * C::SF_COLS, sfb = sfa + C::SF_A_COLS;
-          const int nk = min(C::K64, rg.n_k64 - i * C::K64);
+          const int nk = min(C::KM, rg.n_k64 - i * C::KM);
           for (int kk = 0; kk < nk; ++kk) {
+            // one MMA takes 32 bytes of each operand row (K 64 FP4 / K 32 FP8)
             const uint64_t ad = smem_desc(a_s + kk * 32, 16, 8 * C::ROWB, C::SWZ);
             const uint64_t bd = smem_desc(b_s + kk * 32, 16, 8 * C::ROWB, C::SWZ);
-            if constexpr (PAIR) mma_mxf4nvf4_pair(tmem, ad, bd, idesc_fp4, sfa + kk * 4, sfb + kk * (BN / 32), accum);
-            else mma_mxf4nvf4(tmem, ad, bd, idesc_fp4, sfa + kk * 4, sfb + kk * (BN / 32), accum);
+            if constexpr (F8) {
+              if constexpr (PAIR) mma_f8_pair(tmem, ad, bd, idesc_fp4, accum);
+              else mma_f8(tmem, ad, bd, idesc_fp4, accum);
+            } else {
+              if constexpr (PAIR) mma_mxf4nvf4_pair(tmem, ad, bd, idesc_fp4, sfa + kk * 4, sfb + kk * (BN / 32), accum);
+              else mma_mxf4nvf4(tmem, ad, bd, idesc_fp4, sfa + kk * 4, sfb + kk * (BN / 32), accum);
+            }
             accum = 1;
           }
           commit_both(&empty[st]);
-          commit_lead(&sf_tfree[sl]);
+          if constexpr (!F8) commit_lead(&sf_tfree[sl]);
         }
         if (!ok) break;
         commit_both(acc_full);
@@ -415,16 +427,16 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
   } else {
     // ------------------------------------------------ scale copies: smem stage -> TMEM slot (rank 0 of a pair)
     const int cw = warp - C::CP_WARP0;
-    if (lane == 0 && leader) {
+    if (!F8 && lane == 0 && leader) {  // FP8 operands carry no block scales
       int g = 0;
       bool ok = true;
       for (int t = unit; ok && t < n_tiles; t += n_units) {
         const Range rg = range_of(coord(t).split);
         for (int i = 0; i < rg.n_st; ++i, ++g) {
           const int st = g % C::STAGES, sl = g % kScaleSlots;
-          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_SCALE_WAIT) ||
+          if (!mbar_wait(&full[st], (g / C::STAGES) & 1, p.err, DEVERR_SCALE_WAIT, wlim) ||
               (g >= kScaleSlots &&
-               !mbar_wait(&sf_tfree[sl], ((g / kScaleSlots) & 1) ^ 1u, p.err, DEVERR_SCALE_WAIT))) {
+               !mbar_wait(&sf_tfree[sl], ((g / kScaleSlots) & 1) ^ 1u, p.err, DEVERR_SCALE_WAIT, wlim))) {
             ok = false;
             break;
           }
@@ -465,6 +477,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
     const bool store_issuer = qd == 0 && lane == 0;  // one thread per column half
     uint4* bias_s = reinterpret_cast<uint4*>(smem + C::OFF_BIAS + ew * C::BIAS_BYTES);  // this warp's HC bf16
     int tl = 0;
+    bool alive = true;
     for (int t = unit; t < n_tiles; t += n_units, ++tl) {
       const TileCoord tc = coord(t);
       const int row = tc.m0 + qd * 32 + lane;
@@ -478,7 +491,9 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
         }
         __syncwarp();
       }
-      const bool ok = mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT);
+      // after one wait has run out, the accumulator of later tiles never comes
+      const bool ok = alive && mbar_wait(acc_full, tl & 1, p.err, DEVERR_EPILOGUE_WAIT, wlim);
+      alive = ok;
       __syncwarp();
       tc_fence_after();
       if constexpr (EPI == static_cast<int>(GemmEpilogue::Bf16)) {
@@ -635,17 +650,19 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR>::THREADS, 1)
   }
 }
 
-template <int BN, int KS, int EPI, bool PAIR>
+template <int BN, int KS, int EPI, bool PAIR, bool F8>
 cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
-  using C = Cfg<BN, KS, PAIR>;
-  auto kern = fp4_gemm_kernel<BN, KS, EPI, PAIR>;
+  using C = Cfg<BN, KS, PAIR, F8>;
+  auto kern = fp4_gemm_kernel<BN, KS, EPI, PAIR, F8>;
   static const cudaError_t smem_attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (smem_attr != cudaSuccess) return smem_attr;
-  int dev = 0, sms = 0;
+  int dev = 0, sms = p.sms;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (sms <= 0) sms = 148;
+  if (sms <= 0) {
+    const cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
   if (p.k_stages != (p.K + KS - 1) / KS) return cudaErrorInvalidValue;
   const int tiles = ((p.M + C::TM - 1) / C::TM) * ((p.N + BN - 1) / BN) * p.splits;
   cudaLaunchConfig_t cfg = {};
@@ -692,37 +709,83 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, m.a, m.b, m.u, m.l, m.y, m.sfa, m.sfb, p);
 }
 
-template <int BN, int KS, bool PAIR>
+// registers per thread at launch: the split's total over the 512 threads
+template <int BN, int KS, int EPI, bool PAIR, bool F8>
+bool split_ok(char* msg, size_t n) {
+  using C = Cfg<BN, KS, PAIR, F8>;
+  constexpr int want = (256 * C::REG_OTHER + 256 * C::REG_EPI) / C::THREADS;
+  cudaFuncAttributes a{};
+  const cudaError_t e = cudaFuncGetAttributes(&a, fp4_gemm_kernel<BN, KS, EPI, PAIR, F8>);
+  if (e != cudaSuccess) {
+    snprintf(msg, n, "cudaFuncGetAttributes(fp4_gemm_kernel<%d,%d,%d,%d,%d>) failed: %s", BN, KS, EPI, int(PAIR),
+             int(F8), cudaGetErrorString(e));
+    return false;
+  }
+  if ((a.numRegs + 7) / 8 * 8 != want) {
+    snprintf(msg, n,
+             "fp4_gemm_kernel<%d,%d,%d,%d,%d> was compiled to %d registers per thread; its warpgroup register "
+             "split assumes %d",
+             BN, KS, EPI, int(PAIR), int(F8), a.numRegs, want);
+    return false;
+  }
+  return true;
+}
+
+template <int BN, int KS, bool PAIR, bool F8>
 cudaError_t launch_bn(const GemmMaps& m, const GemmParams& p, GemmEpilogue epi, cudaStream_t st) {
   switch (epi) {
-    case GemmEpilogue::Bf16: return launch_t<BN, KS, 0, PAIR>(m, p, st);
-    case GemmEpilogue::RawF32: return launch_t<BN, KS, 1, PAIR>(m, p, st);
+    case GemmEpilogue::Bf16: return launch_t<BN, KS, 0, PAIR, F8>(m, p, st);
+    case GemmEpilogue::RawF32: return launch_t<BN, KS, 1, PAIR, F8>(m, p, st);
     case GemmEpilogue::SplitK:
       if constexpr (PAIR) return cudaErrorInvalidValue;
-      else return launch_t<BN, KS, 2, false>(m, p, st);
+      else return launch_t<BN, KS, 2, false, F8>(m, p, st);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-GemmShape gemm_shape(int M, int N) {
+template <bool F8, int KB, int KS>  // KB: K per stage of the large-M tiles, KS of the small-M ones
+bool format_split_ok(char* msg, size_t n) {
+  return split_ok<256, KB, 0, true, F8>(msg, n) && split_ok<256, KB, 1, true, F8>(msg, n) &&
+         split_ok<256, KB, 0, false, F8>(msg, n) && split_ok<256, KB, 1, false, F8>(msg, n) &&
+         split_ok<256, KB, 2, false, F8>(msg, n) && split_ok<128, KB, 0, false, F8>(msg, n) &&
+         split_ok<128, KB, 1, false, F8>(msg, n) && split_ok<128, KB, 2, false, F8>(msg, n) &&
+         split_ok<128, KS, 0, false, F8>(msg, n) && split_ok<128, KS, 1, false, F8>(msg, n) &&
+         split_ok<128, KS, 2, false, F8>(msg, n);
+}
+
+bool gemm_register_split_ok(char* msg, size_t n) {
+  return format_split_ok<false, 256, 128>(msg, n) && format_split_ok<true, 128, 64>(msg, n);
+}
+
+GemmShape gemm_shape(int M, int N, bool fp8) {
   GemmShape s;
   s.bn = (M <= kBM || N < 256) ? 128 : 256;
-  s.ks = M <= kBM ? 128 : 256;
+  // operand rows of one 128B (large M) or 64B swizzle atom per stage
+  s.ks = (M <= kBM ? 128 : 256) / (fp8 ? 2 : 1);
   s.pair = s.bn == 256;
+  s.fp8 = fp8;
   return s;
 }
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
                         cudaStream_t st) {
+  const int kb = shape.fp8 ? 128 : 256, ksm = shape.fp8 ? 64 : 128;  // K per stage: large / small M
   if (shape.pair) {
-    if (shape.bn == 256 && shape.ks == 256) return launch_bn<256, 256, true>(maps, p, epi, st);
-    return cudaErrorInvalidValue;
+    if (shape.bn != 256 || shape.ks != kb) return cudaErrorInvalidValue;
+    return shape.fp8 ? launch_bn<256, 128, true, true>(maps, p, epi, st)
+                     : launch_bn<256, 256, true, false>(maps, p, epi, st);
   }
-  if (shape.bn == 256 && shape.ks == 256) return launch_bn<256, 256, false>(maps, p, epi, st);
-  if (shape.bn == 128 && shape.ks == 256) return launch_bn<128, 256, false>(maps, p, epi, st);
-  if (shape.bn == 128 && shape.ks == 128) return launch_bn<128, 128, false>(maps, p, epi, st);
+  if (shape.bn == 256 && shape.ks == kb)
+    return shape.fp8 ? launch_bn<256, 128, false, true>(maps, p, epi, st)
+                     : launch_bn<256, 256, false, false>(maps, p, epi, st);
+  if (shape.bn == 128 && shape.ks == kb)
+    return shape.fp8 ? launch_bn<128, 128, false, true>(maps, p, epi, st)
+                     : launch_bn<128, 256, false, false>(maps, p, epi, st);
+  if (shape.bn == 128 && shape.ks == ksm)
+    return shape.fp8 ? launch_bn<128, 64, false, true>(maps, p, epi, st)
+                     : launch_bn<128, 128, false, false>(maps, p, epi, st);
   return cudaErrorInvalidValue;
 }
 

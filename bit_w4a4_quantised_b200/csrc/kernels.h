@@ -41,6 +41,8 @@ struct PrologueParams {
   float* z_out;           // optional fp32 [rows, K] (debug export of Z)
   float* u_out;           // optional fp32 [rows, r] (debug export of c)
   uint32_t* err;          // device error word for bounded waits
+  int fmt;                // element format: 0 NVFP4 (codes [rows, K/2] + tiled
+                          // scales), 1 FP8 E4M3 (codes [rows, K], no block scales)
 };
 
 enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2 };
@@ -50,6 +52,16 @@ enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2 };
 // requires *amax_glob == 0.
 cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode,
                             cudaStream_t st);
+
+// Rank 0, more than 128 rows: Stats / Quantise with the rotation as one bf16
+// tensor-core product against B = diag(chan / sqrt(b)) H_b (hi / lo) per
+// 128-column chunk; grid = (K / 128) x groups CTAs, CTA (c, g) taking the row
+// tiles g, g + groups, ...  x: the prologue's x tensor map.  Stats requires
+// *amax_glob == 0; p.chan, p.rows, p.K, p.b, p.amax_glob, p.codes, p.sf,
+// p.g_out, p.z_out, p.err are read.
+int wide_prologue_groups(int rows, int K, int sms);
+cudaError_t launch_prologue_wide(const CUtensorMap& x, const PrologueParams& p, PrologueMode mode, int groups,
+                                 cudaStream_t st);
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st);
 // counts[0..2] += mismatches of the quantiser's a / 6 and 1 / a (every positive
@@ -61,6 +73,10 @@ cudaError_t launch_split_v(const float* V, int K, int r, uint16_t* v_hi, uint16_
 // P^T = (diag(chan) H V)^T split into bf16 hi/lo, [r, K] each; H block size b.
 cudaError_t launch_make_proj(const float* V, const float* chan, int K, int r, int b, uint16_t* p_hi, uint16_t* p_lo,
                              cudaStream_t st);
+// L [N, r] bf16 = g * deq(codes, sf) V (V fp32 [K, r], r <= 32): the branch
+// weight of the shared-weight arm, from its stored FP4 weight.
+cudaError_t launch_dequant_project(const uint8_t* codes, const uint8_t* sf, const float* g, const float* V, int N,
+                                   int K, int r, uint16_t* L, cudaStream_t st);
 cudaError_t launch_quantize_fp32(const float* T, int rows, int K, uint8_t* codes, uint8_t* sf, float* g_out,
                                  uint32_t* amax_scratch, cudaStream_t st);
 
@@ -82,6 +98,11 @@ struct GemmParams {
   void* y;                 // bf16 [M, N]
   float* out_f32;          // fp32 [M, N] (raw epilogue)
   uint32_t* err;
+  int sms;                 // SMs of the device (0: queried at launch)
+  uint64_t wait_ns;        // limit of every bounded wait (0: the default)
+  // test only: stage 0 expects this many bytes more than its boxes carry, so
+  // its barrier never completes and every wait behind it runs out (0: off)
+  uint32_t withheld_bytes;
 };
 
 struct GemmMaps {
@@ -99,15 +120,24 @@ struct GemmMaps {
 // CTA reads bn / 2 rows of B: the B (and L) tensor maps must have bn / 2-row
 // boxes.  gemm_shape proposes pair for bn == 256; a split-K plan turns it off.
 struct GemmShape {
-  int bn, ks;
+  int bn, ks;   // tile width, K elements per pipeline stage
   bool pair;
+  bool fp8;     // FP8 E4M3 operands (the W8A8 arm) instead of NVFP4
 };
-GemmShape gemm_shape(int M, int N);
+GemmShape gemm_shape(int M, int N, bool fp8 = false);
 
 // p.k_stages must be ceil(K / shape.ks); split-K (p.splits in {2, 4, 8}) needs
 // the SplitK epilogue, shape.pair false, and launches one cluster of p.splits
 // CTAs per tile.
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
                         cudaStream_t st);
+
+// The warp-specialised kernels move registers between warpgroups with
+// setmaxnreg, a split that adds up to the registers the launch gives each
+// thread.  A warpgroup that asks for more than the launch holds waits forever,
+// so before the first launch the host checks the count every such kernel was
+// compiled to.  Each returns false and describes the first mismatch in msg.
+bool gemm_register_split_ok(char* msg, size_t n);
+bool prologue_register_split_ok(char* msg, size_t n);
 
 }  // namespace qwam

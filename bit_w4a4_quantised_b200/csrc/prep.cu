@@ -100,7 +100,44 @@ __global__ void make_proj_kernel(const float* __restrict__ V, const float* __res
   p_lo[static_cast<size_t>(j) * K + k] = lo;
 }
 
+// Shared-weight arm: the branch weight from the stored FP4 weight,
+// L[n, j] = bf16(g * sum_k e2m1(code[n, k]) e4m3(S[n, k / 16]) V[k, j]), fp32
+// accumulation in k order (each e2m1 * e4m3 product is exact in fp32).  A CTA
+// takes 8 rows; lane j of a row's warp owns column j (r <= 32).
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  const float v = mag[c & 7u];
+  return (c & 8u) ? -v : v;
+}
+
+__global__ void dequant_project_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
+                                       const float* __restrict__ g, const float* __restrict__ V, int N, int K, int r,
+                                       uint16_t* __restrict__ L) {
+  const int j = threadIdx.x & 31;
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (n >= N || j >= r) return;
+  const uint8_t* row = codes + static_cast<size_t>(n) * (K / 2);
+  float acc = 0.0f;
+  for (int kb = 0; kb < K / 16; ++kb) {
+    const float sc = e4m3_value(sf[sf_offset(n, kb, K)]);
+    for (int t = 0; t < 8; ++t) {
+      const uint32_t byte = row[kb * 8 + t];
+      const int k = kb * 16 + 2 * t;
+      acc = __fmaf_rn(__fmul_rn(e2m1_value(byte & 15u), sc), V[static_cast<size_t>(k) * r + j], acc);
+      acc = __fmaf_rn(__fmul_rn(e2m1_value(byte >> 4), sc), V[static_cast<size_t>(k + 1) * r + j], acc);
+    }
+  }
+  L[static_cast<size_t>(n) * r + j] = bf16_bits_rn(__fmul_rn(acc, *g));
+}
+
 }  // namespace
+
+cudaError_t launch_dequant_project(const uint8_t* codes, const uint8_t* sf, const float* g, const float* V, int N,
+                                   int K, int r, uint16_t* L, cudaStream_t st) {
+  if (r < 1 || r > 32) return cudaErrorInvalidValue;
+  dequant_project_kernel<<<(N + 7) / 8, 256, 0, st>>>(codes, sf, g, V, N, K, r, L);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_recip(const float* s, float* inv_s, int K, uint32_t* err, cudaStream_t st) {
   recip_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, err);

@@ -37,6 +37,8 @@
 // it bit-identically), Stats (c to global, atomic amax) and Quantise (reads c
 // and amax, recomputes Z bit-identically from the same code and data,
 // quantises).  Every wait on an mbarrier is bounded.
+#include <cstdio>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "quant.cuh"
@@ -239,25 +241,10 @@ __device__ __forceinline__ void split_cols(uint8_t* xs, uint8_t* lo_tile, const 
 template <int W>
 __device__ __forceinline__ void quantise_cols(const PrologueParams& p, const float (&v)[W], int row, int col,
                                               float g, float y_g) {
-  uint32_t cw[W / 8];
-  uint32_t S[W / 16];
-  quant_blocks16<W / 16>(v, g, y_g, cw, S);
-  uint32_t sfw = 0u;
-#pragma unroll
-  for (int k = 0; k < W / 16; ++k) sfw |= S[k] << (8 * k);
-  uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + col / 2);
-#pragma unroll
-  for (int k = 0; k < W / 32; ++k) dst[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
-  // W / 16 scales of consecutive blocks sit in consecutive bytes of one 4-block word
-  if constexpr (W == 64)
-    *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, col / 16, p.K)) = sfw;
+  if (p.fmt == FMT_FP8)
+    quantise_store_fp8<W>(v, row, col, p.K, y_g, p.codes, p.z_out);
   else
-    *reinterpret_cast<uint16_t*>(p.sf + sf_offset(row, col / 16, p.K)) = static_cast<uint16_t>(sfw);
-  if (p.z_out) {
-    float4* z = reinterpret_cast<float4*>(p.z_out + static_cast<size_t>(row) * p.K + col);
-#pragma unroll
-    for (int k = 0; k < W / 4; ++k) z[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-  }
+    quantise_store<W>(v, row, col, p.K, g, y_g, p.codes, p.sf, p.z_out);
 }
 
 // Branch operand for this thread's UC columns [c0, c0 + UC) of c.
@@ -791,7 +778,7 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
           const float4 a = src[k];
           u[4 * k] = a.x; u[4 * k + 1] = a.y; u[4 * k + 2] = a.z; u[4 * k + 3] = a.w;
         }
-        if (part == 0) write_branch<C::UC>(p, u, R, urow_g, uc0, global_scale_from_amax(__uint_as_float(*p.amax_glob)));
+        if (part == 0) write_branch<C::UC>(p, u, R, urow_g, uc0, scale_from_amax(__uint_as_float(*p.amax_glob), p.fmt));
       }
     }
     if constexpr (R > 0) {
@@ -874,7 +861,7 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
     };
 
     float g = 1.0f;
-    if constexpr (MODE == 2) g = global_scale_from_amax(__uint_as_float(*p.amax_glob));
+    if constexpr (MODE == 2) g = scale_from_amax(__uint_as_float(*p.amax_glob), p.fmt);
     float y_g = rcp_rn(g);
     float amax = 0.0f;
     for (int c = 0; c < nch; ++c) {
@@ -914,7 +901,7 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
       cluster_wait();
       float A = 0.0f;
       for (int rk = 0; rk < p.parts; ++rk) A = fmaxf(A, red[kRowWarps + rk]);
-      g = global_scale_from_amax(A);
+      g = scale_from_amax(A, p.fmt);
       y_g = rcp_rn(g);
       if constexpr (R > 0) {
         if (part == 0 && uvalid) write_branch<C::UC>(p, u, R, urow_g, uc0, g);
@@ -983,7 +970,34 @@ cudaError_t launch_r(const ProMaps& maps, const PrologueParams& p, PrologueMode 
   return cudaErrorInvalidValue;
 }
 
+// Stats / Quantise split registers between warpgroups (setmaxnreg); their
+// launch gives each of the 640 threads the split's average
+template <int R, int MODE>
+bool split_ok(char* msg, size_t n) {
+  using C = PCfg<R, MODE, 64>;
+  constexpr int want = (256 * C::REG_SPLIT + 256 * C::REG_ROWS + 128 * C::REG_OTHER) / C::THREADS;
+  cudaFuncAttributes a{};
+  const cudaError_t e = cudaFuncGetAttributes(&a, prologue_kernel<R, MODE, 64>);
+  if (e != cudaSuccess) {
+    snprintf(msg, n, "cudaFuncGetAttributes(prologue_kernel<%d,%d,64>) failed: %s", R, MODE, cudaGetErrorString(e));
+    return false;
+  }
+  if ((a.numRegs + 7) / 8 * 8 != want) {
+    snprintf(msg, n,
+             "prologue_kernel<%d,%d,64> was compiled to %d registers per thread; its warpgroup register split "
+             "assumes %d",
+             R, MODE, a.numRegs, want);
+    return false;
+  }
+  return true;
+}
+
 }  // namespace
+
+bool prologue_register_split_ok(char* msg, size_t n) {
+  return split_ok<0, 1>(msg, n) && split_ok<0, 2>(msg, n) && split_ok<16, 1>(msg, n) && split_ok<16, 2>(msg, n) &&
+         split_ok<32, 1>(msg, n) && split_ok<32, 2>(msg, n);
+}
 
 cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode,
                             cudaStream_t st) {

@@ -227,3 +227,55 @@ WORKLOADS = {
     "c4up": c4_video_ffn_up,
     "c4down": c4_video_ffn_down,
 }
+
+
+# ---------------------------------------------------------------------------
+# The same recipe drawn on the device (benchmark inputs too large to draw on
+# the host in a few minutes: the 600 linears of one denoising step hold 5.4 B
+# weights).  torch's CUDA generator (Philox) replaces PCG64, so the values
+# differ from the NumPy draws of the same (seed, config, layer); the
+# distributions, the draw order and the derived s and V follow the recipe
+# above.  Parity tests use the NumPy draws.
+# ---------------------------------------------------------------------------
+
+def _device_generator(device, seed: int, config_id: int, layer: int):
+    import torch
+    key = np.random.SeedSequence([seed, config_id, layer]).generate_state(2, dtype=np.uint64)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(key[0] & np.uint64(0x7FFFFFFFFFFFFFFF)))
+    return g
+
+
+def draw_layer_device(spec: LayerSpec, *, seed: int, config_id: int, layer: int, device, b: int = 128,
+                      n_outliers: int = 0, outlier_scale: float = 1.0, w_std: float = 0.02,
+                      bias_std: float = 0.01) -> dict:
+    """One layer's inputs as device tensors: x, W, bias bf16; s, V fp32 (V is
+    None for r = 0).  Returns a dict with the spec's M, K, N, r and b."""
+    import torch
+    g = _device_generator(device, seed, config_id, layer)
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    x = torch.randn((M, K), generator=g, device=device, dtype=torch.float32)
+    if n_outliers:
+        idx = torch.randperm(K, generator=g, device=device)[:n_outliers]
+        x[:, idx] *= outlier_scale
+    x = x.to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * w_std).to(torch.bfloat16)
+    bias = (torch.randn((N,), generator=g, device=device, dtype=torch.float32) * bias_std).to(torch.bfloat16)
+    V = None
+    if r:
+        G = torch.randn((K, r), generator=g, device=device, dtype=torch.float64)
+        V = torch.linalg.qr(G)[0].to(torch.float32).contiguous()
+    ax = x.abs().amax(dim=0).to(torch.float64).clamp_min(1e-5)
+    aw = W.abs().amax(dim=0).to(torch.float64).clamp_min(1e-5)
+    s = (ax.sqrt() / aw.sqrt()).to(torch.float32).contiguous()
+    return {"M": M, "K": K, "N": N, "r": r, "b": b, "x": x, "W": W, "bias": bias, "s": s, "V": V}
+
+
+def c5_layer_device(index: int, device, seed: int = 0, cross_kv_context: bool = True) -> dict:
+    """Layer ``index`` of the C5 step drawn on the device (outliers as c5_layer)."""
+    spec = c5_layer_specs(cross_kv_context)[index]
+    frac, scale = (0.005, 30.0) if spec.name.startswith("video") else (0.01, 20.0)
+    d = draw_layer_device(spec, seed=seed, config_id=5, layer=index, device=device,
+                          n_outliers=outlier_count(spec.K, frac), outlier_scale=scale)
+    d["name"] = spec.name
+    return d

@@ -79,6 +79,44 @@ typedef enum {
 qwam_status qwam_prepare_weight(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
                                 const void* bias_bf16, int hadamard_block, void* stream, qwam_handle* out);
 
+/* ---------------------------------------------------------------------------
+ * The shared-weight arm (card, section "What ASP is...": the cheaper variant
+ * that "quantises one weight and stores V alone").  Read here as: the FP4
+ * weight is W~ = W diag(s) H itself, not deflated, and the branch weight is
+ * formed from that stored weight, L = deq(Q(W~)) V (fp32 accumulation, stored
+ * bf16), so a handle carries nothing beyond the FP4 weight, V and the bias.
+ * The activation side and every per-call entry point are those of the
+ * deflated arm (qwam_linear and the rest take the handle unchanged).
+ * Arguments as qwam_prepare_weight; Wt_f32 (device fp32 [N, K] or NULL)
+ * receives the exact fp32 W~ the weight quantiser consumed.  With r == 0 the
+ * two arms coincide.
+ * ------------------------------------------------------------------------- */
+qwam_status qwam_prepare_weight_shared(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                       const void* bias_bf16, int hadamard_block, float* Wt_f32, void* stream,
+                                       qwam_handle* out);
+
+/* ---------------------------------------------------------------------------
+ * The FP8 W8A8 arm ("QuantWAMs: Calibrating at the Right Granularity for World
+ * Action Models", section "During inference": FP8 W8A8 for the Linears that
+ * calibration upgrades).  The same layer with both quantisers FP8 E4M3 (one
+ * byte per element, no block scales) and one fp32 scale per tensor,
+ * g = amax / 448: the weight's at prepare, the activation's per call; element
+ * code = sign | E4M3_rn_satfinite(|v * (1 / g)|).  The GEMM runs on
+ * tcgen05.mma kind::f8f6f4; smoothing, block rotation, the rank-r branch, the
+ * epilogue and every per-call entry point are those of the NVFP4 arm.
+ * Arguments as qwam_prepare_weight; Wd_f32 (device fp32 [N, K] or NULL)
+ * receives the exact fp32 W_d the weight quantiser consumed.  Exports of this
+ * handle's codes (qwam_export_weight, qwam_debug_prologue) are [rows, K] bytes
+ * and carry no scales.
+ * ------------------------------------------------------------------------- */
+qwam_status qwam_prepare_weight_fp8(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                    const void* bias_bf16, int hadamard_block, float* Wd_f32, void* stream,
+                                    qwam_handle* out);
+
+/* Host outputs (each may be NULL): the element format of the handle (0 NVFP4,
+ * 1 FP8 E4M3) and its weight arm (0 deflated, 1 shared-weight). */
+qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant);
+
 /* Release a handle and its device memory (synchronises the device). */
 qwam_status qwam_destroy(qwam_handle h);
 
@@ -96,7 +134,10 @@ qwam_status qwam_destroy(qwam_handle h);
  * synchronises the device, so it must not be stream-captured; a call at the
  * largest M first makes later calls allocation-free).  Calls that share the
  * workspace must be ordered: do not run two qwam_linear calls concurrently on
- * different streams of the same device.
+ * different streams of the same device.  The handle keeps the launch arguments
+ * (tensor maps) of its last M, so a repeated call encodes nothing and a new x
+ * or y buffer only re-points its map; host calls on one handle are serialised
+ * by a lock inside it.
  * ------------------------------------------------------------------------- */
 qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, void* stream);
 
@@ -115,7 +156,9 @@ qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, 
  * The first call on a device does the set-up (looks up the array's device
  * address and clears its header, whose error word must start at zero,
  * synchronising the device); make that first call before any latency-critical
- * loop.  All calls share the one array per device, whatever the handle: calls
+ * loop and before any stream capture: a first call whose stream is being
+ * captured returns QWAM_ERR_INVALID_ARG and does nothing.  All calls share the
+ * one array per device, whatever the handle: calls
  * that overlap in time (other streams, other threads) race on it and corrupt
  * each other's results, so order them.
  * Expired bounded waits are reported by qwam_device_error.
@@ -136,8 +179,8 @@ qwam_status qwam_gemm(int M, qwam_handle h, void* y_bf16, void* stream);
 qwam_status qwam_handle_info(qwam_handle h, int* N, int* K, int* r, int* b, float* g_w);
 
 /* Copy the handle's weight operands into caller device buffers (each may be
- * NULL): codes [N, K/2] bytes; scales: the tiled layout, round_up(N,128)*K/16
- * bytes; L: bf16 [N, r]. */
+ * NULL): codes [N, K/2] bytes (FP8 handles: [N, K]); scales: the tiled layout,
+ * round_up(N,128)*K/16 bytes (not written for FP8 handles); L: bf16 [N, r]. */
 qwam_status qwam_export_weight(qwam_handle h, void* codes, void* scales, void* L_bf16, void* stream);
 
 /* Same as qwam_prepare_weight, and also writes W_d (the exact fp32 tensor the
@@ -148,8 +191,8 @@ qwam_status qwam_debug_prepare_weight(const void* W_bf16, int N, int K, const fl
 
 /* Run the activation prologue and copy its products to caller device buffers
  * (each may be NULL): z fp32 [M, K] (the exact quantiser input), u fp32 [M, r],
- * codes [M, K/2], scales (tiled, round_up(M,128)*K/16 bytes), u' bf16 [M, r],
- * g_x fp32 scalar. */
+ * codes [M, K/2] (FP8 handles: [M, K]), scales (tiled, round_up(M,128)*K/16
+ * bytes; not written for FP8 handles), u' bf16 [M, r], g_x fp32 scalar. */
 qwam_status qwam_debug_prologue(const void* x_bf16, int M, qwam_handle h, float* z_f32, float* u_f32,
                                 void* codes, void* scales, void* ubr_bf16, float* g_x, void* stream);
 
@@ -164,6 +207,19 @@ qwam_status qwam_quantize_fp32(const float* T, int rows, int K, void* codes, voi
  * 128 (A) and 256 (B), padding bytes zero; out fp32 [M, N] device.  K % 128 == 0. */
 qwam_status qwam_fp4_gemm(const void* a_codes, const void* a_scales, const void* b_codes, const void* b_scales,
                           int M, int N, int K, float alpha, float* out_f32, void* stream);
+
+/* Check of the bounded device waits (failure detection without a fault): the
+ * bare GEMM above (alpha = 1) on single-CTA tiles (M <= 128, or N < 256),
+ * with every wait limited to wait_ns (1 us .. 1 s) and the first pipeline
+ * stage's barrier told to expect 16 bytes more than its TMA boxes carry, so
+ * it never completes.  Every role's wait behind it runs out, sets its bit in
+ * the device error word and the kernel returns; qwam_device_error() then
+ * reports QWAM_ERR_TIMEOUT and the context stays usable.  out_f32 is not
+ * written.  The card has no counterpart: this exercises the library's own
+ * wind-down paths. */
+qwam_status qwam_debug_fp4_gemm_withheld(const void* a_codes, const void* a_scales, const void* b_codes,
+                                         const void* b_scales, int M, int N, int K, uint64_t wait_ns, float* out_f32,
+                                         void* stream);
 
 /* How qwam_linear runs for M rows of this layer (host outputs, each may be
  * NULL): kernels = kernel launches per call, fused = 1 when the prologue is the

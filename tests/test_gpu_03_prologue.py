@@ -30,6 +30,10 @@ CASES = {
     "m32_k2048_r16_b64": lambda: workloads.custom(32, 2048, 96, 16, 64, seed=7, n_outliers=20),
     "m24_k512_r0_b16": lambda: workloads.custom(24, 512, 64, 0, 16, seed=8, n_outliers=5),
     "m9_k8192_r32_b128": lambda: workloads.custom(9, 8192, 64, 32, 128, seed=9, n_outliers=40),
+    # rank 0 above 128 rows: the tensor-core rotation against diag(chan) H_b
+    "m257_k1024_r0_b128": lambda: workloads.custom(257, 1024, 128, 0, 128, seed=10, n_outliers=10),
+    "m600_k512_r0_b2": lambda: workloads.custom(600, 512, 64, 0, 2, seed=11, n_outliers=5),
+    "m129_k640_r0_b1": lambda: workloads.custom(129, 640, 64, 0, 1, seed=12, n_outliers=6),
 }
 
 

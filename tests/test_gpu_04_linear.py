@@ -10,12 +10,21 @@ import numpy as np
 import pytest
 
 from bit_w4a4_quantised_b200 import workloads
-from gpu_util import bf16_to_np, prepare
+from gpu_util import bf16_to_np, device_operand_reference, local_rel_errors, prepare
 from oracle import asp
 
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
+# Per row and per 128-column block, against the float64 product of the
+# device's own quantised operands (device_operand_reference): what is left is
+# the bf16 output rounding (unit roundoff 2^-8 per element, about 1.1e-3 rms),
+# the bf16 branch operands (2^-8 each, on the branch's share) and fp32
+# accumulation.  Against
+# the float64 oracle itself a single FP4 code flip in a row (the contract
+# allows 0.1 % of codes to differ) already moves that row by ~8e-3, so local
+# bounds are taken on the device's operands.
+LOCAL_TOL = 4e-3
 
 CASES = {
     "c1": lambda: workloads.c1_tiny(),
@@ -34,6 +43,14 @@ CASES = {
     # 256 x 256 tiles on CTA pairs (no split-K): ragged M, then ragged M and N
     "m1000_k1024_n2560_r32_b128": lambda: workloads.custom(1000, 1024, 2560, 32, 128, seed=23, n_outliers=10),
     "m1000_k768_n2320_r16_b64": lambda: workloads.custom(1000, 768, 2320, 16, 64, seed=24, n_outliers=8),
+    # rank 0 above 128 rows: the rotation folded into the tensor-core operand
+    # (ragged last tile of one row, several tiles per CTA, b = 16 / 32 / 128;
+    # b = 1 is in the prologue tests, whose criterion is the code identity: with
+    # no rotation a few ulp-level code flips in the x20 outlier channels move
+    # this small a layer's error past 2e-3, as a float64 study reproduces)
+    "m129_k640_n256_r0_b16": lambda: workloads.custom(129, 640, 256, 0, 16, seed=27, n_outliers=6),
+    "m1000_k1024_n2560_r0_b32": lambda: workloads.custom(1000, 1024, 2560, 0, 32, seed=28, n_outliers=10),
+    "m4100_k384_n160_r0_b128": lambda: workloads.custom(4100, 384, 160, 0, 128, seed=29, n_outliers=4),
     # 32 rows with two and four prologue chunks per CTA (action-expert FFN shapes)
     "m32_k2048_n512_r16_b64": lambda: workloads.custom(32, 2048, 512, 16, 64, seed=25, n_outliers=20),
     "m32_k4096_n1024_r32_b128": lambda: workloads.custom(32, 4096, 1024, 32, 128, seed=26, n_outliers=41),
@@ -55,8 +72,11 @@ def test_linear_matches_oracle(name):
     case = CASES[name]()
     h, x, y = run_linear(case)
     ref = asp.asp_linear(case.x, case.W, case.s, case.V, case.bias, case.b)
-    err = asp.rel_fro(bf16_to_np(y), ref)
+    got = bf16_to_np(y)
+    err = asp.rel_fro(got, ref)
     assert err <= TOL, err
+    row_err, blk_err = local_rel_errors(got, device_operand_reference(case, h, x))
+    assert row_err <= LOCAL_TOL and blk_err <= LOCAL_TOL, (row_err, blk_err)
 
 
 def test_two_calls_bit_identical():

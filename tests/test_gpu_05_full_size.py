@@ -13,12 +13,15 @@ import numpy as np
 import pytest
 
 from bit_w4a4_quantised_b200 import workloads
-from gpu_util import bf16_to_np, codes_of, prepare
+from gpu_util import bf16_to_np, codes_of, device_operand_reference, local_rel_errors, prepare
 from oracle import asp, nvfp4
 
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
+# per sampled row and per 128-column block of the sampled rows, against the
+# float64 product of the device's own quantised operands (see test_gpu_04)
+LOCAL_TOL = 4e-3
 
 CASES = {
     "c3_r0": lambda: workloads.c3_video_attn(0),
@@ -57,5 +60,7 @@ def test_full_size_layer_on_sampled_rows(name):
     got = bf16_to_np(y)[rows]
     err = asp.rel_fro(got, ref)
     assert err <= TOL, err
+    row_err, blk_err = local_rel_errors(got, device_operand_reference(case, h, x, rows))
+    assert row_err <= LOCAL_TOL and blk_err <= LOCAL_TOL, (row_err, blk_err)
     same = np.mean(codes_of(d["codes"])[rows] == codes[rows])
     assert same >= 0.999, same

@@ -64,20 +64,93 @@ def test_noalloc_matches_oracle():
     assert asp.rel_fro(bf16_to_np(y), ref) <= TOL
 
 
+_FRESH_PROCESS_CHECK = r"""
+import json, sys
+import torch
+sys.path.insert(0, sys.argv[1])
+sys.path.insert(0, sys.argv[1] + "/tests")
+from bit_w4a4_quantised_b200 import binding as qw, workloads
+from gpu_util import prepare
+# the largest scratch layout the limits admit
+case = workloads.custom(128, 16384, 256, 32, 128, seed=36, n_outliers=80)
+h, x, _ = prepare(case)
+ys = [torch.empty((case.M, case.N), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+torch.cuda.synchronize()
+free0 = torch.cuda.mem_get_info()[0]
+qw.linear_noalloc(x, h, ys[0])          # first call of the process: the set-up
+qw.linear_noalloc(x, h, ys[1])
+torch.cuda.synchronize()
+free1 = torch.cuda.mem_get_info()[0]
+qw.linear(x, h, ys[2])                  # the growable workspace: allocates
+torch.cuda.synchronize()
+free2 = torch.cuda.mem_get_info()[0]
+print(json.dumps({"free0": free0, "free1": free1, "free2": free2, "err": qw.device_error(),
+                  "same": bool(torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2]))}))
+"""
+
+
 def test_noalloc_leaves_free_memory_unchanged():
-    import torch
-    from bit_w4a4_quantised_b200 import binding as qw
-    case = workloads.custom(64, 2048, 1536, 32, 128, seed=36, n_outliers=20)
-    h, x, _ = prepare(case)
-    ys = [torch.empty((case.M, case.N), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
-    qw.linear_noalloc(x, h, ys[0])  # set-up happens on the first call of the process at the latest
-    torch.cuda.synchronize()
-    free0 = torch.cuda.mem_get_info()[0]
-    qw.linear_noalloc(x, h, ys[1])
-    qw.linear_noalloc(x, h, ys[2])
-    torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] == free0
-    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    # A fresh process, so no earlier call has set up the static scratch or
+    # grown the ordinary workspace; every kernel is loaded when the library
+    # is (CUDA_MODULE_LOADING=EAGER), so only the calls themselves could move
+    # device memory.  The ordinary call at the same shape must move it: that
+    # is what shows the measurement can see an allocation.
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_MODULE_LOADING="EAGER")
+    out = subprocess.run([sys.executable, "-c", _FRESH_PROCESS_CHECK, root], env=env, capture_output=True,
+                         text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    r = json.loads(out.stdout.strip().splitlines()[-1])
+    assert r["err"] == 0 and r["same"]
+    assert r["free1"] == r["free0"], r
+    assert r["free2"] < r["free1"], r
+
+
+_FRESH_PROCESS_CAPTURE = r"""
+import json, sys
+import torch
+sys.path.insert(0, sys.argv[1])
+sys.path.insert(0, sys.argv[1] + "/tests")
+from bit_w4a4_quantised_b200 import binding as qw, workloads
+from gpu_util import prepare
+case = workloads.custom(32, 1024, 256, 32, 128, seed=39, n_outliers=10)
+h, x, _ = prepare(case)
+y_ref = qw.linear(x, h)
+y = torch.empty_like(y_ref)
+torch.cuda.synchronize()
+status = None
+side = torch.cuda.Stream()
+g = torch.cuda.CUDAGraph()
+try:
+    with torch.cuda.graph(g, stream=side):
+        qw.linear_noalloc(x, h, y)      # first call of the process, inside a capture
+except qw.QwamError as e:
+    status = e.status
+torch.cuda.synchronize()
+qw.linear_noalloc(x, h, y)              # outside the capture the set-up goes ahead
+torch.cuda.synchronize()
+print(json.dumps({"status": status, "err": qw.device_error(), "same": bool(torch.equal(y, y_ref))}))
+"""
+
+
+def test_noalloc_first_call_under_capture_is_refused():
+    # The set-up synchronises the device, which a stream capture cannot hold:
+    # the library refuses it with QWAM_ERR_INVALID_ARG and a later uncaptured
+    # call sets up and computes as usual.
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", _FRESH_PROCESS_CAPTURE, root], capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    r = json.loads(out.stdout.strip().splitlines()[-1])
+    assert r["status"] == 1 and r["err"] == 0 and r["same"], r
 
 
 def test_noalloc_rejects_sizes_beyond_its_limits():
