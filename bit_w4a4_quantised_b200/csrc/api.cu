@@ -20,7 +20,11 @@ namespace {
 
 constexpr uint32_t kMagic = 0x514d5731u;
 constexpr int kMaxDevices = 64;
-constexpr size_t kHeaderBytes = 256;  // scalars: activation amax, g_x, device error word
+// Scalars at the start of every workspace: [0] activation amax (fp32 bits),
+// [4] g_x, [12] the one-pass prologue's grid-barrier count (the first 16 bytes
+// are cleared before each such launch), [32] the device error word.
+constexpr size_t kHeaderBytes = 256;
+constexpr size_t kErrOffset = 32;
 
 thread_local std::string g_err;
 
@@ -237,7 +241,7 @@ Layout layout_for(int M, int K, int r, int fmt) {
 
 uint32_t* arena_amax(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base); }
 float* arena_gx(const Arena& a) { return reinterpret_cast<float*>(a.base + 4); }
-uint32_t* arena_err(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base + 8); }
+uint32_t* arena_err(const Arena& a) { return reinterpret_cast<uint32_t*>(a.base + kErrOffset); }
 
 qwam_status arena_get(int dev, size_t need, Arena** out) {
   std::lock_guard<std::mutex> lock(g_arena_mu);
@@ -365,8 +369,12 @@ bool use_fused(int rows) { return rows <= 128; }
 // two launches (Stats, Quantise), with the rotation folded into the tensor-core
 // operand when there is no subspace (r = 0), else the row pipeline with the
 // rank-r projection and deflation.
-enum { PRO_FUSED = 0, PRO_TWO_PASS = 1, PRO_WIDE = 2 };
-int prologue_form(int rows, int r) { return use_fused(rows) ? PRO_FUSED : (r == 0 ? PRO_WIDE : PRO_TWO_PASS); }
+enum { PRO_FUSED = 0, PRO_TWO_PASS = 1, PRO_WIDE = 2, PRO_ONEPASS = 3 };
+int prologue_form(int rows, int r, int K, int sms) {
+  if (use_fused(rows)) return PRO_FUSED;
+  if (r != 0) return PRO_TWO_PASS;
+  return onepass_prologue_fits(rows, K, wide_prologue_groups(rows, K, sms), sms) ? PRO_ONEPASS : PRO_WIDE;
+}
 
 // The launches of the row pipeline: Fused (rows <= 128, when allowed), else
 // Stats + Quantise.  prm.amax_glob is the activation / weight amax word.
@@ -600,7 +608,7 @@ qwam_status build_call(qwam_handle h, int M, uint8_t* ws, CallPlan* c) {
   prm.branch_mode = 1;
   prm.g_other = h->g_w;
   prm.g_out = reinterpret_cast<float*>(ws + 4);
-  prm.err = reinterpret_cast<uint32_t*>(ws + 8);
+  prm.err = reinterpret_cast<uint32_t*>(ws + kErrOffset);
   prm.parts = cluster_parts(h->K, M, sms);
   prm.chunks = h->K / 128 / prm.parts;
   prm.fmt = h->fmt;
@@ -639,7 +647,7 @@ qwam_status build_call(qwam_handle h, int M, uint8_t* ws, CallPlan* c) {
   gp.sms = sms;
 
   c->pl = pl;
-  c->pro_form = prologue_form(M, h->r);
+  c->pro_form = prologue_form(M, h->r, h->K, sms);
   c->pro_groups = wide_prologue_groups(M, h->K, sms);
   c->pmaps = h->vmaps;
   c->prm = prm;
@@ -682,6 +690,11 @@ qwam_status bind_y(qwam_handle h, CallPlan* c, void* y) {
 }
 
 qwam_status launch_call_prologue(const CallPlan& c, const PrologueParams& prm, int r, cudaStream_t st) {
+  if (c.pro_form == PRO_ONEPASS) {
+    QW_CUDA(cudaMemsetAsync(prm.amax_glob, 0, 16, st));  // amax, g_x, grid-barrier count
+    QW_CUDA(launch_prologue_onepass(c.pmaps.x, prm, c.pro_groups, st));
+    return QWAM_OK;
+  }
   if (c.pro_form == PRO_WIDE) {
     QW_CUDA(cudaMemsetAsync(prm.amax_glob, 0, sizeof(uint32_t), st));
     QW_CUDA(launch_prologue_wide(c.pmaps.x, prm, PrologueMode::Stats, c.pro_groups, st));
@@ -1004,7 +1017,8 @@ qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* 
   if (M < 0) return fail(QWAM_ERR_SHAPE, "M=%d must be >= 0", M);
   const bool f = use_fused(M);
   const Plan pl = plan_gemm(std::max(M, 1), h->N, h->K, sm_count(h->dev), h->fmt);
-  if (kernels) *kernels = M == 0 ? 0 : (f ? 2 : 3);
+  const int form = prologue_form(std::max(M, 1), h->r, h->K, sm_count(h->dev));
+  if (kernels) *kernels = M == 0 ? 0 : (form == PRO_FUSED || form == PRO_ONEPASS ? 2 : 3);
   if (fused) *fused = f ? 1 : 0;
   if (splits) *splits = pl.splits;
   if (bn) *bn = pl.bn;
@@ -1041,8 +1055,8 @@ qwam_status qwam_device_error(uint32_t* code) {
   }
   if (sbase) {  // the error word of qwam_linear_noalloc's static scratch
     uint32_t c = 0;
-    QW_CUDA(cudaMemcpy(&c, sbase + 8, 4, cudaMemcpyDeviceToHost));
-    QW_CUDA(cudaMemset(sbase + 8, 0, 4));
+    QW_CUDA(cudaMemcpy(&c, sbase + kErrOffset, 4, cudaMemcpyDeviceToHost));
+    QW_CUDA(cudaMemset(sbase + kErrOffset, 0, 4));
     *code |= c;
   }
   std::lock_guard<std::mutex> lock(g_arena_mu);

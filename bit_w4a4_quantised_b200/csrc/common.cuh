@@ -26,6 +26,7 @@ enum : uint32_t {
   DEVERR_DRAIN_WAIT = 1u << 3,
   DEVERR_BRANCH_WAIT = 1u << 4,
   DEVERR_SCALE_WAIT = 1u << 5,
+  DEVERR_GRID_WAIT = 1u << 6,  // a grid-wide barrier of a cooperative launch
 };
 
 // A bounded wait gives up after this long (device global timer, nanoseconds).

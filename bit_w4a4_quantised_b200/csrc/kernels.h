@@ -60,6 +60,12 @@ cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r,
 // *amax_glob == 0; p.chan, p.rows, p.K, p.b, p.amax_glob, p.codes, p.sf,
 // p.g_out, p.z_out, p.err are read.
 int wide_prologue_groups(int rows, int K, int sms);
+// One launch of the same rotation for up to six row tiles per CTA and every CTA
+// resident (a cooperative launch): x read once, Z kept on chip across one
+// bounded grid-wide barrier for the amax.  Requires the 16 bytes at
+// p.amax_glob (amax, g_x, barrier count) to be zero at launch.
+bool onepass_prologue_fits(int rows, int K, int groups, int sms);
+cudaError_t launch_prologue_onepass(const CUtensorMap& x, const PrologueParams& p, int groups, cudaStream_t st);
 cudaError_t launch_prologue_wide(const CUtensorMap& x, const PrologueParams& p, PrologueMode mode, int groups,
                                  cudaStream_t st);
 

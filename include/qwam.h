@@ -222,9 +222,10 @@ qwam_status qwam_debug_fp4_gemm_withheld(const void* a_codes, const void* a_scal
                                          void* stream);
 
 /* How qwam_linear runs for M rows of this layer (host outputs, each may be
- * NULL): kernels = kernel launches per call, fused = 1 when the prologue is the
- * single-launch (cluster-wide amax) form, splits = K splits of the GEMM,
- * bn = GEMM tile width. */
+ * NULL): kernels = kernel launches per call (2 when the prologue is one launch:
+ * up to 128 rows, or rank 0 with at most six 128-row tiles per CTA; else 3),
+ * fused = 1 when the prologue is the single-launch cluster form for up to 128
+ * rows, splits = K splits of the GEMM, bn = GEMM tile width. */
 qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* splits, int* bn);
 
 /* Synchronise the current device, then return (and clear) the device error

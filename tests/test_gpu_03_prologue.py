@@ -34,6 +34,8 @@ CASES = {
     "m257_k1024_r0_b128": lambda: workloads.custom(257, 1024, 128, 0, 128, seed=10, n_outliers=10),
     "m600_k512_r0_b2": lambda: workloads.custom(600, 512, 64, 0, 2, seed=11, n_outliers=5),
     "m129_k640_r0_b1": lambda: workloads.custom(129, 640, 64, 0, 1, seed=12, n_outliers=6),
+    # one launch with a grid-wide barrier, 4 row tiles per CTA
+    "m1950_k4736_r0_b64": lambda: workloads.custom(1950, 4736, 64, 0, 64, seed=13, n_outliers=24),
 }
 
 

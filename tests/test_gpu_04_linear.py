@@ -51,6 +51,11 @@ CASES = {
     "m129_k640_n256_r0_b16": lambda: workloads.custom(129, 640, 256, 0, 16, seed=27, n_outliers=6),
     "m1000_k1024_n2560_r0_b32": lambda: workloads.custom(1000, 1024, 2560, 0, 32, seed=28, n_outliers=10),
     "m4100_k384_n160_r0_b128": lambda: workloads.custom(4100, 384, 160, 0, 128, seed=29, n_outliers=4),
+    # the one-launch form with 3 and 4 row tiles per CTA (ragged last tiles), and
+    # a layer with 8 tiles per CTA that keeps the two-launch form
+    "m1100_k6272_n256_r0_b128": lambda: workloads.custom(1100, 6272, 256, 0, 128, seed=30, n_outliers=31),
+    "m1950_k4736_n256_r0_b64": lambda: workloads.custom(1950, 4736, 256, 0, 64, seed=31, n_outliers=24),
+    "m1000_k12800_n128_r0_b128": lambda: workloads.custom(1000, 12800, 128, 0, 128, seed=32, n_outliers=64),
     # 32 rows with two and four prologue chunks per CTA (action-expert FFN shapes)
     "m32_k2048_n512_r16_b64": lambda: workloads.custom(32, 2048, 512, 16, 64, seed=25, n_outliers=20),
     "m32_k4096_n1024_r32_b128": lambda: workloads.custom(32, 4096, 1024, 32, 128, seed=26, n_outliers=41),
