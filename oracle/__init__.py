@@ -14,16 +14,22 @@ nvfp4
     packing and the 128x4 scale-tile layout.
 fp8
     The FP8 W8A8 arm's per-tensor E4M3 quantiser and its dequantisation.
+int4
+    The SVDQuant arm's INT4 group-64 quantiser (fp16 scales), its
+    dequantisation and the exact integer group sums of its product.
 asp
     Block Hadamard, smoothing, rank-r deflation and the full layer
     ``y = (x~V)(W~V)^T + NVFP4GEMM((I-VV^T)x~, W~(I-VV^T)) + bias`` in float64;
-    the shared-weight arm's weight side; the FP8 arm (``fmt="fp8"``).
+    the shared-weight arm's weight side; the FP8 arm (``fmt="fp8"``); the
+    SVDQuant arm (``svdquant_linear``: no rotation, activation not deflated,
+    INT4 group 64 on both sides).
 
 Sources: "QuantWAMs: Calibrating at the Right Granularity for World Action
 Models" (report), section "During inference" (FP8 W8A8 for the upgraded
 Linears); "FastWAM UR3 3-task — 4-bit quantisations" (Hugging Face model card),
-sections "What ASP is, and what the deflated form means" (the contract) and the
-top comparison table (numeric format), "Files" (scale swizzle), and
+sections "What ASP is, and what the deflated form means" (the contract), the
+top comparison table (numeric formats of both checkpoints), "Verification —
+INT4 SVDQuant", "Files" (scale swizzle), and
 "Verification — NVFP4 deflated ASP" (storage figures); "Q-WAM: 4-Bit Quantization
 of World Action Models with Action-Subspace Protection", abstract (16-bit
 low-rank branch, both sides as dense matmuls).

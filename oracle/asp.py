@@ -32,9 +32,9 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import fp8, nvfp4
+from . import fp8, int4, nvfp4
 
-FORMATS = ("nvfp4", "fp8")
+FORMATS = ("nvfp4", "fp8", "int4")
 
 
 def _quantise(T32, fmt: str) -> dict:
@@ -46,6 +46,9 @@ def _quantise(T32, fmt: str) -> dict:
     if fmt == "fp8":
         codes, g = fp8.quantize(T32)
         return {"codes": codes, "g": g, "deq": fp8.dequantize(codes, g)}
+    if fmt == "int4":
+        codes, scales = int4.quantize(T32)
+        return {"codes": codes, "scales": scales, "deq": int4.dequantize(codes, scales)}
     raise ValueError(fmt)
 
 
@@ -143,11 +146,14 @@ def prepare_weight_shared(W, s, V, b: int, fp4: bool = True) -> dict:
     return out
 
 
-def activation_prologue(x, s, V, b: int, fp4: bool = True, fmt: str = "nvfp4") -> dict:
+def activation_prologue(x, s, V, b: int, fp4: bool = True, fmt: str = "nvfp4", deflated: bool = True) -> dict:
     """Per-call side: x~, u = x~V, z = x~ - u V^T, and the quantisation of z
-    (NVFP4, or the FP8 arm's E4M3 with ``fmt="fp8"``)."""
+    (NVFP4, or the FP8 arm's E4M3 with ``fmt="fp8"``).  ``deflated=False``
+    (the SVDQuant arm) quantises x~ itself: z = x~."""
     xt = rotate_activation(x, s, b)
     u, z = deflate(xt, V)
+    if not deflated:
+        z = xt.copy()
     out = {"xt": xt, "u": u, "z": z}
     if fp4:
         out.update(_quantise(z.astype(np.float32), fmt))
@@ -167,16 +173,20 @@ def asp_linear(x, W, s, V, bias, b: int, fp4: bool = True, parts: bool = False, 
     (used to pin the formula to x W^T + bias).  ``variant="shared"`` takes the
     shared-weight arm's weight side (prepare_weight_shared).  ``fmt="fp8"`` is
     the FP8 W8A8 arm: the same layer with both quantisers FP8 E4M3 per tensor
-    (oracle.fp8) and the product taken on those operands."""
-    if variant not in ("deflated", "shared"):
+    (oracle.fp8) and the product taken on those operands.  ``variant=
+    "svdquant"`` (with ``fmt="int4"`` and b = 1) is the SVDQuant arm: see
+    ``svdquant_linear``."""
+    if variant not in ("deflated", "shared", "svdquant"):
         raise ValueError(variant)
-    if fmt not in FORMATS or (fmt != "nvfp4" and variant != "deflated"):
+    if fmt not in FORMATS or (fmt == "fp8" and variant != "deflated") or ((fmt == "int4") != (variant == "svdquant")):
         raise ValueError(f"format {fmt!r} with variant {variant!r}")
-    if variant == "deflated":
-        wp = prepare_weight(W, s, V, b, fp4=fp4, fmt=fmt)
-    else:
+    if variant == "svdquant" and b != 1:
+        raise ValueError("the SVDQuant arm has no Hadamard rotation: b = 1")
+    if variant == "shared":
         wp = prepare_weight_shared(W, s, V, b, fp4=fp4)
-    ap = activation_prologue(x, s, V, b, fp4=fp4, fmt=fmt)
+    else:
+        wp = prepare_weight(W, s, V, b, fp4=fp4, fmt=fmt)
+    ap = activation_prologue(x, s, V, b, fp4=fp4, fmt=fmt, deflated=variant != "svdquant")
     y_fp4 = nvfp4_gemm(ap["deq"], wp["deq"])
     y_lr = ap["u"] @ wp["L"].T
     y = y_fp4 + y_lr
@@ -185,6 +195,22 @@ def asp_linear(x, W, s, V, bias, b: int, fp4: bool = True, parts: bool = False, 
     if parts:
         return y, {"act": ap, "wt": wp, "y_fp4": y_fp4, "y_lr": y_lr}
     return y
+
+
+def svdquant_linear(x, W, s, V, bias, fp4: bool = True, parts: bool = False):
+    """The SVDQuant W4A4 arm (model card, top table, SVDQuant column; "Verification
+    — INT4 SVDQuant"), in this oracle's terms: smoothing x^ = x / s and
+    W^ = W diag(s) with no rotation (b = 1); the low-rank branch from the
+    rank-r basis V, L = W^ V, so that L V^T is the rank-r truncated SVD of W^
+    when V holds its top right singular vectors (calibrating V is out of
+    scope: V is an input, as on the ASP arm); the residual R = W^ - L V^T
+    quantised INT4 group 64, and the activation x^ itself (not deflated)
+    quantised the same way:
+
+        y = deq(Q(x^)) deq(Q(R))^T + (x^ V) L^T + bias
+
+    Without quantisation the two paths add up to x^ W^T^ + bias = x W^T + bias."""
+    return asp_linear(x, W, s, V, bias, 1, fp4=fp4, parts=parts, variant="svdquant", fmt="int4")
 
 
 def rel_fro(a, ref) -> float:
