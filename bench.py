@@ -23,9 +23,11 @@ dominant kernel group.
 
 With the default workload on one GPU the line also carries per_config: the
 single layers (c2 action attention 32 x 1024 -> 1024, c3 video attention
-4096 x 3072 -> 3072 at r = 32 and r = 0, c4 video FFN up and down) and the
-action-expert half of the step (c5action), each with its own roofline,
-cpu_baseline and e2e.  --workload <name> runs one of those alone.
+4096 x 3072 -> 3072 at r = 32 and r = 0, c4 video FFN up and down), the
+action-expert half of the step (c5action), and the boundary's other arms on
+the same layers (c3r0fp8 / c2fp8: the FP8 W8A8 arm, against the FP8 peak;
+c2shared: the shared-weight arm), each with its own roofline, cpu_baseline and
+e2e.  --workload <name> runs one of those alone.
 
 Timing: CUDA events around K steps replayed from a CUDA graph (one untimed
 replay first), barrier + synchronize on both sides, max over ranks.  Multi-GPU
@@ -57,6 +59,7 @@ from bit_w4a4_quantised_b200 import workloads  # noqa: E402
 METRIC = "ASP-NVFP4 linear TFLOP/s and GB/s per layer, % of FP4/HBM roofline"
 L2_BYTES = 126 * 10 ** 6
 DTYPE = "nvfp4 (e2m1 x e4m3 block-16) GEMM, fp32 accumulate; bf16 in/out; bf16 rank-r branch"
+DTYPE_FP8 = "fp8 e4m3 (per-tensor scales) GEMM, fp32 accumulate; bf16 in/out; bf16 rank-r branch"
 
 STEP = dict(desc="one denoising step of the 2-expert model: 600 linears (video d 3072, ffn 14336, 4096 tokens, "
                  "r=0; action d 1024, ffn 4096, 32 tokens, cross k/v over the 4096-token context, r=32), b=128",
@@ -91,11 +94,22 @@ WORKLOADS = {
     "c4down": dict(make=lambda i, seed: workloads.c4_video_ffn_down(seed=seed + i),
                    desc="video-expert FFN down, 4096 tokens, 14336->3072, r=32, b=128",
                    unit="TFLOP/s", steps=500, warmup=5),
+    # the other arms of the boundary on the same layers
+    "c3r0fp8": dict(make=lambda i, seed: workloads.c3_video_attn(0, seed=seed, layer=i), fmt="fp8",
+                    desc="FP8 W8A8 arm: video-expert attention projection, 4096 tokens, 3072->3072, r=0, b=128",
+                    unit="TFLOP/s", steps=2000, warmup=10),
+    "c2fp8": dict(make=lambda i, seed: workloads.c2_action_attn(seed=seed, layer=i), fmt="fp8",
+                  desc="FP8 W8A8 arm: action-expert attention projection, 32 tokens, 1024->1024, r=32, b=128",
+                  unit="GB/s", steps=200000, warmup=50),
+    "c2shared": dict(make=lambda i, seed: workloads.c2_action_attn(seed=seed, layer=i), variant="shared",
+                     desc="shared-weight arm: action-expert attention projection, 32 tokens, 1024->1024, r=32, "
+                          "b=128", unit="GB/s", steps=200000, warmup=50),
 }
 
 # per_config entries of the default run: (steps, warm-up, seconds of oracle work)
 PER_CONFIG = {"c2": (20000, 50, 8.0), "c3": (400, 10, 8.0), "c3r0": (400, 10, 8.0), "c4up": (100, 5, 8.0),
-              "c4down": (100, 5, 8.0), "c5action": (10, 3, 8.0)}
+              "c4down": (100, 5, 8.0), "c5action": (10, 3, 8.0), "c3r0fp8": (400, 10, 6.0),
+              "c2fp8": (20000, 50, 6.0), "c2shared": (20000, 50, 6.0)}
 
 
 def set_layers(wl):
@@ -116,24 +130,28 @@ def step_kinds(specs):
 # ---------------------------------------------------------------------------
 # Algorithmic work per layer (minimal bytes / flops of the method itself).
 # ---------------------------------------------------------------------------
-def layer_bytes(M, K, N, r):
-    """x (bf16) + packed W_d with E4M3 scales (0.5625 B/weight) + L (bf16) +
-    V (fp32) + s (fp32) + bias (bf16) + y (bf16)."""
-    return 2 * M * K + 0.5625 * N * K + 2 * N * r + 4 * K * r + 4 * K + 2 * N + 2 * M * N
+def layer_bytes(M, K, N, r, fmt="nvfp4"):
+    """x (bf16) + packed W_d with E4M3 scales (0.5625 B/weight; FP8 arm: 1 B) +
+    L (bf16) + V (fp32) + s (fp32) + bias (bf16) + y (bf16)."""
+    wb = 1.0 if fmt == "fp8" else 0.5625
+    return 2 * M * K + wb * N * K + 2 * N * r + 4 * K * r + 4 * K + 2 * N + 2 * M * N
 
 
 def layer_flops(M, K, N, r):
     return 2 * M * N * K + 2 * M * N * r + 4 * M * K * r
 
 
-def prologue_bytes(M, K, N, r):
-    """Reads x, V, s; writes FP4 codes + scales (0.5625 B/element) and u'."""
-    return 2 * M * K + 4 * K * r + 4 * K + 0.5625 * M * K + 2 * M * r
+def prologue_bytes(M, K, N, r, fmt="nvfp4"):
+    """Reads x, V, s; writes FP4 codes + scales (0.5625 B/element; FP8: 1 B)
+    and u'."""
+    eb = 1.0 if fmt == "fp8" else 0.5625
+    return 2 * M * K + 4 * K * r + 4 * K + eb * M * K + 2 * M * r
 
 
-def gemm_bytes(M, K, N, r):
-    """Reads FP4 activations + scales, W_d + scales, L, u', bias; writes y."""
-    return 0.5625 * M * K + 0.5625 * N * K + 2 * N * r + 2 * M * r + 2 * N + 2 * M * N
+def gemm_bytes(M, K, N, r, fmt="nvfp4"):
+    """Reads FP4 (FP8) activations + scales, W_d + scales, L, u', bias; writes y."""
+    eb = 1.0 if fmt == "fp8" else 0.5625
+    return eb * M * K + eb * N * K + 2 * N * r + 2 * M * r + 2 * N + 2 * M * N
 
 
 def gemm_flops(M, K, N, r):
@@ -152,6 +170,15 @@ def measured_peaks():
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
                 "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def fp8_peak(peaks, timed_alone):
+    """Dense FP8 peak = 2 x the bf16 peak (nominal 4.5 / 2.25 PFLOP/s)."""
+    burst, sust = 2.0 * peaks["bf16_tflops"], 2.0 * peaks["bf16_tflops_sustained"]
+    which = "burst" if timed_alone else "sustained"
+    note = (f"dense FP8 = 2 x {peaks['source']} {which} cuBLAS bf16 (nominal ratio 4.5/2.25 PFLOP/s); "
+            f"the other fraction against 2 x the {'sustained' if timed_alone else 'burst'} figure")
+    return (burst, sust, note) if timed_alone else (sust, burst, note)
 
 
 def fp4_peak(peaks, timed_alone):
@@ -257,25 +284,31 @@ def blas_threads():
         return None
 
 
-def oracle_call(prep, case):
+def oracle_call(prep, case, fmt="nvfp4"):
     """The per-call work of the layer in the float64 oracle: activation side,
-    FP4 product on dequantised operands, low-rank branch, bias."""
+    FP4 (FP8) product on dequantised operands, low-rank branch, bias."""
     from oracle import asp
-    act = asp.activation_prologue(case.x, case.s, case.V, case.b)
+    act = asp.activation_prologue(case.x, case.s, case.V, case.b, fmt=fmt)
     y = asp.nvfp4_gemm(act["deq"], prep["deq"]) + act["u"] @ prep["L"].T + case.bias.astype("float64")[None, :]
     return y
 
 
-def time_oracle(cases, budget_s):
+def oracle_prepare(c, fmt="nvfp4", variant="deflated"):
+    from oracle import asp
+    if variant == "shared":
+        return asp.prepare_weight_shared(c.W, c.s, c.V, c.b)
+    return asp.prepare_weight(c.W, c.s, c.V, c.b, fmt=fmt)
+
+
+def time_oracle(cases, budget_s, fmt="nvfp4", variant="deflated"):
     """Run oracle calls over the given cases (weights prepared outside the
     clock) until budget_s of CPU work has elapsed; returns (calls, seconds)."""
-    from oracle import asp
-    preps = [asp.prepare_weight(c.W, c.s, c.V, c.b) for c in cases]
+    preps = [oracle_prepare(c, fmt, variant) for c in cases]
     n, t = 0, 0.0
     while True:
         c, p = cases[n % len(cases)], preps[n % len(cases)]
         t0 = time.perf_counter()
-        oracle_call(p, c)
+        oracle_call(p, c, fmt)
         t += time.perf_counter() - t0
         n += 1
         if t >= budget_s:
@@ -398,9 +431,9 @@ def hbm_roof(kernel, nbytes, dur_ms, peaks):
             "kernel": kernel}
 
 
-def tensor_roof(kernel, flops, dur_ms, peaks, timed_alone):
+def tensor_roof(kernel, flops, dur_ms, peaks, timed_alone, fmt="nvfp4"):
     achieved = flops / (dur_ms / 1e3) / 1e12
-    peak, other, note = fp4_peak(peaks, timed_alone)
+    peak, other, note = (fp8_peak if fmt == "fp8" else fp4_peak)(peaks, timed_alone)
     r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "peak_note": note,
          "frac": achieved / peak, "kernel": kernel}
     r["frac_sustained" if timed_alone else "frac_burst"] = achieved / other
@@ -413,6 +446,7 @@ def tensor_roof(kernel, flops, dur_ms, peaks, timed_alone):
 def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     torch, qw = ctx.torch, ctx.qw
     wl = WORKLOADS[name]
+    fmt, variant = wl.get("fmt", "nvfp4"), wl.get("variant", "deflated")
     probe = wl["make"](0, args.seed)
     M, K, N, r, hb = probe.M, probe.K, probe.N, probe.r, probe.b
     warmup = max(3, warmup)
@@ -426,7 +460,7 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
         s = torch.from_numpy(c.s).to(ctx.dev)
         V = torch.from_numpy(c.V).to(ctx.dev) if c.r else None
         bias = torch.from_numpy(c.bias).to(ctx.dev).to(torch.bfloat16)
-        handles.append(qw.prepare_weight(W, s, V, bias, c.b))
+        handles.append(qw.prepare_weight(W, s, V, bias, c.b, variant=variant, fmt=fmt))
         xs.append(torch.from_numpy(c.x).to(ctx.dev).to(torch.bfloat16))
         ys.append(torch.empty((M, N), dtype=torch.bfloat16, device=ctx.dev))
         del W, s, V, bias
@@ -509,18 +543,18 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     ms, e2e_ms = ctx.max_ranks([ms, e2e_ms])
 
     unit = wl["unit"]
-    lb, lf = layer_bytes(M, K, N, r), layer_flops(M, K, N, r)
+    lb, lf = layer_bytes(M, K, N, r, fmt), layer_flops(M, K, N, r)
     units = lb if unit == "GB/s" else lf
     value = per_unit(units * steps * ctx.world, ms / 1e3, unit)
     peaks = measured_peaks()
     pro_avg, gem_avg = sum(pro_ms) / G, sum(gem_ms) / G
     dominant = "gemm" if gem_avg >= pro_avg else "prologue"
     if dominant == "gemm" and unit == "TFLOP/s":
-        roof = tensor_roof("fp4_gemm_kernel", gemm_flops(M, K, N, r), gem_avg, peaks, timed_alone=True)
+        roof = tensor_roof("fp4_gemm_kernel", gemm_flops(M, K, N, r), gem_avg, peaks, timed_alone=True, fmt=fmt)
     elif dominant == "gemm":
-        roof = hbm_roof("fp4_gemm_kernel", gemm_bytes(M, K, N, r), gem_avg, peaks)
+        roof = hbm_roof("fp4_gemm_kernel", gemm_bytes(M, K, N, r, fmt), gem_avg, peaks)
     else:
-        roof = hbm_roof("prologue_kernel", prologue_bytes(M, K, N, r), pro_avg, peaks)
+        roof = hbm_roof("prologue_kernel", prologue_bytes(M, K, N, r, fmt), pro_avg, peaks)
     roof["traffic"] = recorded_traffic(name, roof["kernel"])
     roof["avg_launch_us"] = (gem_avg if dominant == "gemm" else pro_avg) * 1e3
     roof["duration_note"] = ("CUDA events around each kernel in replays of the timed graph with event nodes "
@@ -531,7 +565,8 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": ctx.world, "steps": steps, "warmup": warmup,
         "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": DTYPE, "data": "synthetic (seeded; shapes of the Fast-WAM experts, random-init weights)",
+        "dtype": DTYPE_FP8 if fmt == "fp8" else DTYPE,
+        "data": "synthetic (seeded; shapes of the Fast-WAM experts, random-init weights)",
         "config": {"workload": f"{name}: {wl['desc']}", "M": M, "K": K, "N": N, "r": r, "hadamard_block": hb,
                    "parallelism": f"replicas x{ctx.world}",
                    "l2": f"rotating {P} distinct layer instances, {working_set / 1e6:.0f} MB > 126 MB L2; "
@@ -548,7 +583,7 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     }
     if ctx.rank == 0 and ctx.world == 1:
         cases = [probe] + [wl["make"](i, args.seed) for i in range(1, 3 if M <= 128 else 1)]
-        n, t = time_oracle(cases, cpu_budget)
+        n, t = time_oracle(cases, cpu_budget, fmt, variant)
         cores = cores_used()
         line["cpu_baseline"] = {"value": per_unit(units * n, t, unit), "unit": unit,
                                 "cores": cores["blas_threads"] or cores["affinity"], "kind": "oracle",
@@ -883,19 +918,21 @@ def run_reference(args):
         from oracle import asp
         wl = WORKLOADS[args.workload]
         unit = wl["unit"]
+        fmt, variant = wl.get("fmt", "nvfp4"), wl.get("variant", "deflated")
         cases = [wl["make"](i, args.seed) for i in range(2)]
         c0 = cases[0]
-        units_per_step = (layer_bytes if unit == "GB/s" else layer_flops)(c0.M, c0.K, c0.N, c0.r)
-        preps = [asp.prepare_weight(c.W, c.s, c.V, c.b) for c in cases]
-        oracle_call(preps[0], cases[0])  # warm-up
+        units_per_step = (layer_bytes(c0.M, c0.K, c0.N, c0.r, fmt) if unit == "GB/s"
+                          else layer_flops(c0.M, c0.K, c0.N, c0.r))
+        preps = [oracle_prepare(c, fmt, variant) for c in cases]
+        oracle_call(preps[0], cases[0], fmt)  # warm-up
         t0 = time.perf_counter()
-        oracle_call(preps[0], cases[0])
+        oracle_call(preps[0], cases[0], fmt)
         first = time.perf_counter() - t0
         K_req = args.steps if args.steps is not None else wl["steps"]
         steps = max(1, min(K_req, int(60.0 / max(first, 1e-6))))
         t0 = time.perf_counter()
         for i in range(steps):
-            oracle_call(preps[i % 2], cases[i % 2])
+            oracle_call(preps[i % 2], cases[i % 2], fmt)
         dt = time.perf_counter() - t0
         value = per_unit(units_per_step * steps, dt, unit)
         line.update(value=value, unit=unit, steps=steps, warmup=1, ms_per_step=dt / steps * 1e3,

@@ -31,6 +31,9 @@ SIGNATURES = {
     "qwam_prepare_weight_shared": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     "qwam_prepare_weight_fp8": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     "qwam_handle_format": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "qwam_image_size": (_I, [_P, ctypes.POINTER(ctypes.c_size_t)]),
+    "qwam_save_image": (_I, [_P, _P, ctypes.c_size_t, _P]),
+    "qwam_load_image": (_I, [_P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "qwam_debug_prologue": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "qwam_quantize_fp32": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "qwam_fp4_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
@@ -45,7 +48,8 @@ SIGNATURES = {
 }
 
 STATUS = {0: "QWAM_OK", 1: "QWAM_ERR_INVALID_ARG", 2: "QWAM_ERR_SHAPE", 3: "QWAM_ERR_ALIGN",
-          4: "QWAM_ERR_ARCH", 5: "QWAM_ERR_OOM", 6: "QWAM_ERR_CUDA", 7: "QWAM_ERR_TIMEOUT"}
+          4: "QWAM_ERR_ARCH", 5: "QWAM_ERR_OOM", 6: "QWAM_ERR_CUDA", 7: "QWAM_ERR_TIMEOUT",
+          8: "QWAM_ERR_FORMAT"}
 
 
 class QwamError(RuntimeError):
@@ -135,6 +139,14 @@ class Handle:
             raise ValueError("handle already destroyed")
         return self._raw
 
+    def save_image(self, stream=None) -> bytes:
+        """The layer image (qwam_save_image): header, operands, checksum."""
+        n = ctypes.c_size_t()
+        _check(load().qwam_image_size(self.raw, ctypes.byref(n)))
+        buf = ctypes.create_string_buffer(n.value)
+        _check(load().qwam_save_image(self.raw, buf, n.value, _stream(stream)))
+        return buf.raw
+
     def destroy(self) -> None:
         if self._raw:
             _check(load().qwam_destroy(self._raw))
@@ -184,6 +196,13 @@ def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None,
     else:
         _check(lib.qwam_debug_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
                                              _ptr(wd_out), _stream(stream), ctypes.byref(out)))
+    return Handle(out.value)
+
+
+def load_image(image: bytes, stream=None) -> Handle:
+    """A handle on the current device from a layer image (qwam_load_image)."""
+    out = _P()
+    _check(load().qwam_load_image(image, len(image), _stream(stream), ctypes.byref(out)))
     return Handle(out.value)
 
 

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -409,6 +410,86 @@ qwam_status run_rows(const void* T, PrologueParams prm, int r, const ProMaps& vm
 
 // shared: the shared-weight arm (quantise W~ itself; L = deq(Q(W~)) V) instead
 // of the deflated one (quantise W_d = W~ - (W~V)V^T; L = W~V).
+// The device arrays a layer owns, sized from its shape (r = 0 keeps
+// one-column placeholders for the rank-r arrays, which nothing reads).
+size_t layer_code_bytes(const qwam_layer* h) { return static_cast<size_t>(h->N) * code_bytes(h->K, h->fmt); }
+size_t layer_branch_bytes(const qwam_layer* h) { return static_cast<size_t>(h->N) * std::max(h->r, 1) * 2; }
+size_t layer_v_bytes(const qwam_layer* h) { return static_cast<size_t>(h->K) * std::max(h->r, 1) * 2; }
+
+qwam_status alloc_layer(qwam_layer* h, bool with_bias) {
+  h->sf_bytes = h->fmt == 1 ? 16 : round_up(static_cast<size_t>(h->N), 256) * h->K / 16;
+  const size_t K = static_cast<size_t>(h->K);
+  QW_TRY(dmalloc(&h->codes, layer_code_bytes(h)));
+  QW_TRY(dmalloc(&h->sf, h->sf_bytes));
+  QW_TRY(dmalloc(&h->L, layer_branch_bytes(h)));
+  QW_TRY(dmalloc(&h->v_hi, layer_v_bytes(h)));
+  QW_TRY(dmalloc(&h->v_lo, layer_v_bytes(h)));
+  QW_TRY(dmalloc(&h->px_hi, layer_v_bytes(h)));
+  QW_TRY(dmalloc(&h->px_lo, layer_v_bytes(h)));
+  QW_TRY(dmalloc(&h->inv_s, K * 4));
+  QW_TRY(dmalloc(&h->inv_s_pm, K * 8));
+  QW_TRY(dmalloc(&h->hmat, 128 * 128 * 2));
+  if (with_bias) QW_TRY(dmalloc(&h->bias, static_cast<size_t>(h->N) * 2));
+  return QWAM_OK;
+}
+
+// Everything of a layer that follows from its shape and its device addresses:
+// the bf16 H_b blocks of one 128-column chunk and every tensor map the calls
+// read.  A map encodes an address, not data, so this may run before the
+// arrays are filled.  The H_b upload is ordered on st (a pageable source is
+// staged before the call returns, so the host vector may go).
+qwam_status finish_layer(qwam_layer* h, cudaStream_t st) {
+  const int N = h->N, K = h->K, r = h->r, b = h->b;
+  // H_b restricted to one 128-column chunk, in Sylvester order: +-1 where row and
+  // column lie in the same b-block, 0 elsewhere (1/sqrt(b) is in the channel
+  // vector); the B operand of the prologue's tensor-core rotation.
+  std::vector<uint16_t> hm(128 * 128);
+  for (int n = 0; n < 128; ++n)
+    for (int k = 0; k < 128; ++k)
+      hm[n * 128 + k] = (n ^ k) >= b ? 0 : ((__builtin_popcount(n & k & (b - 1)) & 1) ? 0xBF80u : 0x3F80u);
+  QW_CUDA(cudaMemcpyAsync(h->hmat, hm.data(), hm.size() * 2, cudaMemcpyHostToDevice, st));
+  QW_TRY(make_map(&h->vmaps.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->hmat, 128, 128, 256, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B));
+  if (r > 0) {
+    QW_TRY(make_map(&h->vmaps.p_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->px_hi, K, r, static_cast<uint64_t>(K) * 2, 64,
+                    r, CU_TENSOR_MAP_SWIZZLE_128B));
+    QW_TRY(make_map(&h->vmaps.p_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->px_lo, K, r, static_cast<uint64_t>(K) * 2, 64,
+                    r, CU_TENSOR_MAP_SWIZZLE_128B));
+    QW_TRY(make_map(&h->vmaps.v_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_hi, r, K, r * 2, r, 128, branch_swizzle(r)));
+    QW_TRY(make_map(&h->vmaps.v_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_lo, r, K, r * 2, r, 128, branch_swizzle(r)));
+  }
+  // B boxes: 64-byte rows (small M) or 128-byte rows (large M), 128 or 256 rows
+  const int cb = code_bytes(K, h->fmt);
+  QW_TRY(make_codes_map(&h->map_b128_k128, h->codes, N, cb, 64, 128));
+  QW_TRY(make_codes_map(&h->map_b128_k256, h->codes, N, cb, 128, 128));
+  QW_TRY(make_codes_map(&h->map_b256_k256, h->codes, N, cb, 128, 256));
+  if (h->fmt == 1) {  // no block scales: the unread scale maps alias the codes map
+    h->map_sfb_k128 = h->map_sfb_k256_b1 = h->map_sfb_k256_b2 = h->map_b128_k128;
+  } else {
+    const size_t rows = round_up(static_cast<size_t>(N), 256);
+    QW_TRY(make_sf_map(&h->map_sfb_k128, h->sf, rows, K, 128, 1));
+    QW_TRY(make_sf_map(&h->map_sfb_k256_b1, h->sf, rows, K, 256, 1));
+    QW_TRY(make_sf_map(&h->map_sfb_k256_b2, h->sf, rows, K, 256, 2));
+  }
+  if (r > 0) {
+    QW_TRY(make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r)));
+    QW_TRY(make_map(&h->map_l256, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 256, branch_swizzle(r)));
+  } else {
+    h->map_l128 = h->map_b128_k128;
+    h->map_l256 = h->map_b256_k256;
+  }
+  return QWAM_OK;
+}
+
+qwam_layer* new_layer(int N, int K, int r, int b, int dev, int fmt, int variant) {
+  qwam_layer* h = new qwam_layer();  // value-initialised: every pointer and map zero
+  h->magic = kMagic;
+  h->N = N; h->K = K; h->r = r; h->b = b; h->dev = dev;
+  h->fmt = fmt;
+  h->variant = variant;
+  return h;
+}
+
 qwam_status prepare_impl(const void* W, int N, int K, const float* s, const float* V, int r, const void* bias,
                          int b, float* wd_out, bool shared, int fmt, void* stream, qwam_handle* out) {
   if (!out) return fail(QWAM_ERR_INVALID_ARG, "out handle pointer is NULL");
@@ -423,12 +504,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   QW_TRY(current_device(&dev));
   cudaStream_t st = as_stream(stream);
 
-  qwam_layer* h = new qwam_layer();  // value-initialised: every pointer and map zero
-  h->magic = kMagic;
-  h->N = N; h->K = K; h->r = r; h->b = b; h->dev = dev;
-  h->fmt = fmt;
-  h->variant = shared ? 1 : 0;
-  h->sf_bytes = fmt == 1 ? 16 : round_up(static_cast<size_t>(N), 256) * K / 16;
+  qwam_layer* h = new_layer(N, K, r, b, dev, fmt, shared ? 1 : 0);
   float* u_tmp = nullptr;
   uint32_t* scratch = nullptr;  // [0] amax, [1] err, [2] g_w (fp32)
   uint16_t *pw_hi = nullptr, *pw_lo = nullptr;  // P^T of the weight side, diag(s) H V
@@ -444,17 +520,11 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   };
   qwam_status s_;
   const size_t rr = static_cast<size_t>(std::max(r, 1));
-  if ((s_ = dmalloc(&h->codes, static_cast<size_t>(N) * code_bytes(K, fmt))) != QWAM_OK ||
-      (s_ = dmalloc(&h->sf, h->sf_bytes)) != QWAM_OK || (s_ = dmalloc(&h->L, static_cast<size_t>(N) * rr * 2)) != QWAM_OK ||
-      (s_ = dmalloc(&h->v_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->v_lo, K * rr * 2)) != QWAM_OK ||
-      (s_ = dmalloc(&h->px_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&h->px_lo, K * rr * 2)) != QWAM_OK ||
-      (s_ = dmalloc(&pw_hi, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&pw_lo, K * rr * 2)) != QWAM_OK ||
-      (s_ = dmalloc(&h->inv_s, static_cast<size_t>(K) * 4)) != QWAM_OK ||
-      (s_ = dmalloc(&h->inv_s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK || (s_ = dmalloc(&s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK ||
-      (s_ = dmalloc(&h->hmat, 128 * 128 * 2)) != QWAM_OK ||
-      (s_ = dmalloc(&u_tmp, static_cast<size_t>(N) * rr * 4)) != QWAM_OK || (s_ = dmalloc(&scratch, 64)) != QWAM_OK)
+  if ((s_ = alloc_layer(h, bias != nullptr)) != QWAM_OK || (s_ = dmalloc(&pw_hi, K * rr * 2)) != QWAM_OK ||
+      (s_ = dmalloc(&pw_lo, K * rr * 2)) != QWAM_OK || (s_ = dmalloc(&s_pm, static_cast<size_t>(K) * 8)) != QWAM_OK ||
+      (s_ = dmalloc(&u_tmp, static_cast<size_t>(N) * rr * 4)) != QWAM_OK || (s_ = dmalloc(&scratch, 64)) != QWAM_OK ||
+      (s_ = finish_layer(h, st)) != QWAM_OK)
     return cleanup(s_);
-  if (bias && (s_ = dmalloc(&h->bias, static_cast<size_t>(N) * 2)) != QWAM_OK) return cleanup(s_);
 
 #define QW_CUDA_CLEAN(call)                                                                                      \
   do {                                                                                                           \
@@ -469,36 +539,17 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   const float hscale = 1.0f / std::sqrt(static_cast<float>(b));
   QW_CUDA_CLEAN(launch_chan_pm(h->inv_s, hscale, K, h->inv_s_pm, st));
   QW_CUDA_CLEAN(launch_chan_pm(s, hscale, K, s_pm, st));
-  // H_b restricted to one 128-column chunk, in Sylvester order: +-1 where row and
-  // column lie in the same b-block, 0 elsewhere (1/sqrt(b) is in the channel
-  // vector); the B operand of the prologue's tensor-core rotation.
-  {
-    std::vector<uint16_t> hm(128 * 128);
-    for (int n = 0; n < 128; ++n)
-      for (int k = 0; k < 128; ++k)
-        hm[n * 128 + k] = (n ^ k) >= b ? 0 : ((__builtin_popcount(n & k & (b - 1)) & 1) ? 0xBF80u : 0x3F80u);
-    QW_CUDA_CLEAN(cudaMemcpy(h->hmat, hm.data(), hm.size() * 2, cudaMemcpyHostToDevice));
-    if ((s_ = make_map(&h->vmaps.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->hmat, 128, 128, 256, 64, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != QWAM_OK)
-      return cleanup(s_);
-  }
   ProMaps wmaps{};  // the weight pass uses P of the weight side
   wmaps.h = h->vmaps.h;
   if (r > 0) {
     QW_CUDA_CLEAN(launch_split_v(V, K, r, h->v_hi, h->v_lo, st));
     QW_CUDA_CLEAN(launch_make_proj(V, s, K, r, b, pw_hi, pw_lo, st));
     QW_CUDA_CLEAN(launch_make_proj(V, h->inv_s, K, r, b, h->px_hi, h->px_lo, st));
+    wmaps = h->vmaps;
     auto pmap = [&](CUtensorMap* m, const uint16_t* base) {
       return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, K, r, static_cast<uint64_t>(K) * 2, 64, r,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     };
-    if ((s_ = pmap(&h->vmaps.p_hi, h->px_hi)) != QWAM_OK || (s_ = pmap(&h->vmaps.p_lo, h->px_lo)) != QWAM_OK ||
-        (s_ = make_map(&h->vmaps.v_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_hi, r, K, r * 2, r, 128,
-                       branch_swizzle(r))) != QWAM_OK ||
-        (s_ = make_map(&h->vmaps.v_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->v_lo, r, K, r * 2, r, 128,
-                       branch_swizzle(r))) != QWAM_OK)
-      return cleanup(s_);
-    wmaps = h->vmaps;
     if ((s_ = pmap(&wmaps.p_hi, pw_hi)) != QWAM_OK || (s_ = pmap(&wmaps.p_lo, pw_lo)) != QWAM_OK) return cleanup(s_);
   }
   PrologueParams prm{};
@@ -534,31 +585,6 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   if (host_scr[3]) return cleanup(fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired in prepare (flags 0x%x)", host_scr[3]));
   std::memcpy(&h->g_w, &host_scr[2], 4);
 
-  // B boxes: 64-byte rows (small M) or 128-byte rows (large M), 128 or 256 rows
-  const int cb = code_bytes(K, fmt);
-  if ((s_ = make_codes_map(&h->map_b128_k128, h->codes, N, cb, 64, 128)) != QWAM_OK ||
-      (s_ = make_codes_map(&h->map_b128_k256, h->codes, N, cb, 128, 128)) != QWAM_OK ||
-      (s_ = make_codes_map(&h->map_b256_k256, h->codes, N, cb, 128, 256)) != QWAM_OK)
-    return cleanup(s_);
-  if (fmt == 1) {  // no block scales: the unread scale maps alias the codes map
-    h->map_sfb_k128 = h->map_sfb_k256_b1 = h->map_sfb_k256_b2 = h->map_b128_k128;
-  } else if ((s_ = make_sf_map(&h->map_sfb_k128, h->sf, round_up(static_cast<size_t>(N), 256), K, 128, 1)) != QWAM_OK ||
-             (s_ = make_sf_map(&h->map_sfb_k256_b1, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 1)) !=
-                 QWAM_OK ||
-             (s_ = make_sf_map(&h->map_sfb_k256_b2, h->sf, round_up(static_cast<size_t>(N), 256), K, 256, 2)) !=
-                 QWAM_OK) {
-    return cleanup(s_);
-  }
-  if (r > 0) {
-    if ((s_ = make_map(&h->map_l128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 128, branch_swizzle(r))) !=
-            QWAM_OK ||
-        (s_ = make_map(&h->map_l256, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L, r, N, r * 2, r, 256, branch_swizzle(r))) !=
-            QWAM_OK)
-      return cleanup(s_);
-  } else {
-    h->map_l128 = h->map_b128_k128;
-    h->map_l256 = h->map_b256_k256;
-  }
   cudaFree(s_pm);
   cudaFree(u_tmp);
   cudaFree(scratch);
@@ -715,6 +741,77 @@ qwam_status workspace_for(qwam_handle h, int M, Arena** a) {
   return arena_get(h->dev, layout_for(M, h->K, h->r, h->fmt).total, a);
 }
 
+// ---------------------------------------------------------------------------
+// Layer images: a prepared layer as one host byte string.  A 64-byte header
+// (little-endian), then the arrays the calls read, each padded to 16 bytes:
+// codes, block scales (NVFP4 only), L, V hi/lo and P^T hi/lo (r > 0 only),
+// 1/s, bias (when present).  What follows from these (the row-pipeline form of
+// 1/s, the H_b blocks and every tensor map) is rebuilt on load.  The checksum
+// is FNV-1a 64 (Fowler, Noll and Vo) over the whole image with its own field
+// taken as zero.
+constexpr char kImageMagic[8] = {'Q', 'W', 'A', 'M', 'I', 'M', 'G', '\0'};
+constexpr uint32_t kImageVersion = 1;
+
+struct ImageHeader {
+  char magic[8];
+  uint32_t version, header_bytes;
+  int32_t N, K, r, b, fmt, variant;
+  uint32_t flags;  // bit 0: bias present
+  float g_w;
+  uint64_t total_bytes, checksum;
+};
+static_assert(sizeof(ImageHeader) == 64, "image header is 64 bytes");
+
+struct ImageSection {
+  void* dev;
+  size_t bytes;
+};
+
+size_t pad16(size_t n) { return (n + 15) & ~static_cast<size_t>(15); }
+
+// The sections of a layer in image order; returns their count (at most 9).
+int image_sections(const qwam_layer* h, bool with_bias, ImageSection* out) {
+  int n = 0;
+  out[n++] = {h->codes, layer_code_bytes(h)};
+  if (h->fmt == 0) out[n++] = {h->sf, h->sf_bytes};
+  if (h->r > 0) {
+    const size_t vb = static_cast<size_t>(h->K) * h->r * 2;
+    out[n++] = {h->L, static_cast<size_t>(h->N) * h->r * 2};
+    out[n++] = {h->v_hi, vb};
+    out[n++] = {h->v_lo, vb};
+    out[n++] = {h->px_hi, vb};
+    out[n++] = {h->px_lo, vb};
+  }
+  out[n++] = {h->inv_s, static_cast<size_t>(h->K) * 4};
+  if (with_bias) out[n++] = {h->bias, static_cast<size_t>(h->N) * 2};
+  return n;
+}
+
+size_t image_bytes(const qwam_layer* h, bool with_bias) {
+  ImageSection sec[9];
+  const int n = image_sections(h, with_bias, sec);
+  size_t total = sizeof(ImageHeader);
+  for (int i = 0; i < n; ++i) total += pad16(sec[i].bytes);
+  return total;
+}
+
+uint64_t fnv1a64(const uint8_t* p, size_t n, uint64_t h = 0xcbf29ce484222325ull) {
+  for (size_t i = 0; i < n; ++i) {
+    h ^= p[i];
+    h *= 0x100000001b3ull;
+  }
+  return h;
+}
+
+uint64_t image_checksum(const uint8_t* img, size_t total) {
+  ImageHeader hd;
+  std::memcpy(&hd, img, sizeof hd);
+  hd.checksum = 0;
+  const uint64_t h = fnv1a64(reinterpret_cast<const uint8_t*>(&hd), sizeof hd);
+  return fnv1a64(img + sizeof hd, total - sizeof hd, h);
+}
+
+
 }  // namespace
 
 // ---- allocation-free variant of the layer call -----------------------------
@@ -812,6 +909,101 @@ qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant) {
   if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
   if (fmt) *fmt = h->fmt;
   if (variant) *variant = h->variant;
+  return QWAM_OK;
+}
+
+qwam_status qwam_image_size(qwam_handle h, size_t* bytes) {
+  if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
+  if (!bytes) return fail(QWAM_ERR_INVALID_ARG, "bytes pointer is NULL");
+  *bytes = image_bytes(h, h->bias != nullptr);
+  return QWAM_OK;
+}
+
+qwam_status qwam_save_image(qwam_handle h, void* host_buf, size_t buf_bytes, void* stream) {
+  QW_TRY(check_handle(h));
+  if (!host_buf) return fail(QWAM_ERR_INVALID_ARG, "host buffer is NULL");
+  const bool with_bias = h->bias != nullptr;
+  const size_t total = image_bytes(h, with_bias);
+  if (buf_bytes < total) return fail(QWAM_ERR_INVALID_ARG, "host buffer holds %zu bytes, the image needs %zu", buf_bytes, total);
+  uint8_t* img = static_cast<uint8_t*>(host_buf);
+  cudaStream_t st = as_stream(stream);
+  std::memset(img, 0, total);
+  ImageSection sec[9];
+  const int n = image_sections(h, with_bias, sec);
+  size_t off = sizeof(ImageHeader);
+  for (int i = 0; i < n; ++i) {
+    QW_CUDA(cudaMemcpyAsync(img + off, sec[i].dev, sec[i].bytes, cudaMemcpyDeviceToHost, st));
+    off += pad16(sec[i].bytes);
+  }
+  QW_CUDA(cudaStreamSynchronize(st));
+  ImageHeader hd{};
+  std::memcpy(hd.magic, kImageMagic, 8);
+  hd.version = kImageVersion;
+  hd.header_bytes = sizeof(ImageHeader);
+  hd.N = h->N; hd.K = h->K; hd.r = h->r; hd.b = h->b;
+  hd.fmt = h->fmt;
+  hd.variant = h->variant;
+  hd.flags = with_bias ? 1u : 0u;
+  hd.g_w = h->g_w;
+  hd.total_bytes = total;
+  std::memcpy(img, &hd, sizeof hd);
+  hd.checksum = image_checksum(img, total);
+  std::memcpy(img, &hd, sizeof hd);
+  return QWAM_OK;
+}
+
+qwam_status qwam_load_image(const void* host_buf, size_t buf_bytes, void* stream, qwam_handle* out) {
+  if (!out) return fail(QWAM_ERR_INVALID_ARG, "out handle pointer is NULL");
+  *out = nullptr;
+  if (!host_buf) return fail(QWAM_ERR_INVALID_ARG, "host buffer is NULL");
+  const uint8_t* img = static_cast<const uint8_t*>(host_buf);
+  ImageHeader hd;
+  if (buf_bytes < sizeof hd) return fail(QWAM_ERR_FORMAT, "image of %zu bytes is shorter than its header", buf_bytes);
+  std::memcpy(&hd, img, sizeof hd);
+  if (std::memcmp(hd.magic, kImageMagic, 8) != 0) return fail(QWAM_ERR_FORMAT, "not a layer image (bad magic)");
+  if (hd.version != kImageVersion || hd.header_bytes != sizeof hd)
+    return fail(QWAM_ERR_FORMAT, "image version %u / header %u bytes is not %u / %zu", hd.version, hd.header_bytes,
+                kImageVersion, sizeof hd);
+  if (check_layer_shape(hd.N, hd.K, hd.r, hd.b) != QWAM_OK)
+    return fail(QWAM_ERR_FORMAT, "image shape N=%d K=%d r=%d b=%d is not a valid layer", hd.N, hd.K, hd.r, hd.b);
+  if ((hd.fmt != 0 && hd.fmt != 1) || (hd.variant != 0 && hd.variant != 1) || (hd.fmt == 1 && hd.variant != 0) ||
+      (hd.flags & ~1u) || !(std::isfinite(hd.g_w) && hd.g_w > 0.0f))
+    return fail(QWAM_ERR_FORMAT, "image header fields are out of range (fmt %d, variant %d, flags 0x%x)", hd.fmt,
+                hd.variant, hd.flags);
+  qwam_layer shape{};
+  shape.N = hd.N; shape.K = hd.K; shape.r = hd.r; shape.fmt = hd.fmt;
+  shape.sf_bytes = hd.fmt == 1 ? 16 : round_up(static_cast<size_t>(hd.N), 256) * hd.K / 16;
+  const bool with_bias = hd.flags & 1u;
+  const size_t total = image_bytes(&shape, with_bias);
+  if (hd.total_bytes != total || buf_bytes < total)
+    return fail(QWAM_ERR_FORMAT, "image says %llu bytes, its shape needs %zu, the buffer holds %zu",
+                static_cast<unsigned long long>(hd.total_bytes), total, buf_bytes);
+  if (image_checksum(img, total) != hd.checksum) return fail(QWAM_ERR_FORMAT, "image checksum does not match");
+
+  int dev = 0;
+  QW_TRY(current_device(&dev));
+  cudaStream_t st = as_stream(stream);
+  qwam_layer* h = new_layer(hd.N, hd.K, hd.r, hd.b, dev, hd.fmt, hd.variant);
+  h->g_w = hd.g_w;
+  auto cleanup = [&](qwam_status s) {
+    free_layer(h);
+    return s;
+  };
+  qwam_status s_;
+  if ((s_ = alloc_layer(h, with_bias)) != QWAM_OK || (s_ = finish_layer(h, st)) != QWAM_OK) return cleanup(s_);
+  ImageSection sec[9];
+  const int n = image_sections(h, with_bias, sec);
+  size_t off = sizeof(ImageHeader);
+  cudaError_t e = cudaSuccess;
+  if (hd.fmt == 1) e = cudaMemsetAsync(h->sf, 0, h->sf_bytes, st);
+  for (int i = 0; i < n && e == cudaSuccess; ++i) {
+    e = cudaMemcpyAsync(sec[i].dev, img + off, sec[i].bytes, cudaMemcpyHostToDevice, st);
+    off += pad16(sec[i].bytes);
+  }
+  if (e == cudaSuccess) e = launch_chan_pm(h->inv_s, 1.0f / std::sqrt(static_cast<float>(hd.b)), hd.K, h->inv_s_pm, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cleanup(fail(QWAM_ERR_CUDA, "loading the image failed: %s", cudaGetErrorString(e)));
+  *out = h;
   return QWAM_OK;
 }
 
@@ -1083,6 +1275,7 @@ const char* qwam_status_string(qwam_status s) {
     case QWAM_ERR_OOM: return "QWAM_ERR_OOM";
     case QWAM_ERR_CUDA: return "QWAM_ERR_CUDA";
     case QWAM_ERR_TIMEOUT: return "QWAM_ERR_TIMEOUT";
+    case QWAM_ERR_FORMAT: return "QWAM_ERR_FORMAT";
   }
   return "QWAM_UNKNOWN";
 }

@@ -41,33 +41,60 @@ constexpr int kXBytes = kTile * kTile * 2;       // two 64-column boxes, 128B sw
 constexpr int kOffB = 0;                         // B_hi, then B_lo: the x tile's layout, rows = n
 constexpr int kOffX = kOffB + 2 * kXBytes;
 constexpr int kOffBar = kOffX + kSlots * kXBytes;
-constexpr int kSmem = kOffBar + 256 + 1024;
+constexpr int kOffStage = kOffBar + 256;           // 128 staged channel words for building B
+constexpr int kSmem = kOffStage + 512 + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 
 // B = diag(chan / sqrt(b)) H_b of chunk c, split into bf16 hi / lo, in the
 // K-major 128B-swizzled layout of the x tile (row n, 16-byte chunk j of the
 // 64-column half kb): hi at dst, lo at dst + kXBytes.  p.chan holds chan /
 // sqrt(b) (a layer constant, so this may run before the wait on the previous
-// kernel).  Threads [tid0 of nthreads] share the work.
-__device__ __forceinline__ void build_rotation_operand(uint8_t* dst, const PrologueParams& p, int c, int tid,
-                                                       int nthreads) {
-  const float* ch = p.chan + static_cast<size_t>(c) * 2 * kTile;
+// kernel).  The chunk's 128 values and their hi / lo parts are staged first
+// (stage: 128 words, hi in bits 0..15, lo in 16..31); an entry of B is then
+// one of them with both signs flipped (bf16 rounding is sign-symmetric, so
+// -c splits into -hi, -lo) or zero.  Called by the nthreads builder threads
+// (tid 0 .. nthreads - 1, whole warps, nthreads >= 128), which synchronise on
+// named barrier kBuildBar.
+constexpr int kBuildBar = 2;
+constexpr int kBuildWarp0 = 2;  // warps 2 .. end build B; 0 (loads) and 1 (MMA) do not wait for it
+constexpr int kBuilders = kThreads - 32 * kBuildWarp0;
+__device__ __forceinline__ void build_rotation_operand(uint8_t* dst, uint32_t* stage, const PrologueParams& p, int c,
+                                                       int tid, int nthreads) {
+  if (tid < kTile) {
+    const float v = p.chan[static_cast<size_t>(c) * 2 * kTile + tid];
+    const uint32_t hi = bf16_bits_rn(v);
+    const uint32_t lo = bf16_bits_rn(__fsub_rn(v, __uint_as_float(hi << 16)));
+    stage[tid] = hi | (lo << 16);
+  }
+  named_bar(kBuildBar, nthreads);
+  // An item is the 16-byte chunk of row n holding k = k0 .. k0 + 7 (k0 = 64 kb +
+  // 8 j).  The Sylvester sign (-1)^popcount(n & k) over those k is the sign at
+  // k0 times the parity pattern of (n & 7) & e, e = 0 .. 7 (bit e of kPar[n & 7]);
+  // b-blocks of 8 or more columns hold all 8 entries or none.
+  constexpr uint32_t kPar[8] = {0x00u, 0xAAu, 0xCCu, 0x66u, 0xF0u, 0x5Au, 0x3Cu, 0x96u};
+  const uint32_t bmask = static_cast<uint32_t>(p.b - 1);
   for (int idx = tid; idx < 2 * kTile * 8; idx += nthreads) {
     const int kb = idx >> 10, n = (idx >> 3) & 127, j = idx & 7;
+    const int k0 = kb * 64 + 8 * j;
+    const uint32_t s0 = (__popc(static_cast<uint32_t>(n & k0) & bmask) & 1u) ? 0xFFu : 0u;
+    const uint32_t negs = s0 ^ kPar[n & 7];
+    const uint4 st0 = *reinterpret_cast<const uint4*>(stage + k0);
+    const uint4 st1 = *reinterpret_cast<const uint4*>(stage + k0 + 4);
+    const uint32_t sw[8] = {st0.x, st0.y, st0.z, st0.w, st1.x, st1.y, st1.z, st1.w};
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
-      float v[2];
+      uint32_t w[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int k = kb * 64 + 8 * j + e + h;
-        const bool in_block = (n ^ k) < p.b;
-        const bool neg = (__popc(n & k & (p.b - 1)) & 1) != 0;
-        v[h] = in_block ? (neg ? -ch[k] : ch[k]) : 0.0f;
+        const int k = k0 + e + h;
+        // within H's b-block of k?  (for b < 8 the block bits of e matter too)
+        const bool in_block = ((static_cast<uint32_t>(n ^ k)) & ~bmask) == 0u;
+        const uint32_t sgn = (p.b >= 8 ? (negs >> (e + h)) : (__popc(static_cast<uint32_t>(n & k) & bmask))) & 1u;
+        w[h] = in_block ? (sw[e + h] ^ (sgn ? 0x80008000u : 0u)) : 0u;
       }
-      hw[e / 2] = bf16x2_rn(v[0], v[1]);
-      lw[e / 2] = bf16x2_rn(__fsub_rn(v[0], __uint_as_float(hw[e / 2] << 16)),
-                            __fsub_rn(v[1], __uint_as_float(hw[e / 2] & 0xffff0000u)));
+      hw[e / 2] = (w[0] & 0xffffu) | (w[1] << 16);
+      lw[e / 2] = (w[0] >> 16) | (w[1] & 0xffff0000u);
     }
     const int off = kb * 16384 + n * 128 + ((j ^ (n & 7)) << 4);
     *reinterpret_cast<uint4*>(dst + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -101,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + kSlots;       // [kSlots] MMAs done with the slot
   uint64_t* zfull = bars + 2 * kSlots;   // [2] Z of a tile in TMEM buffer d
   uint64_t* zfree = zfull + 2;           // [2] row warps read buffer d
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zfree + 2);
+  uint64_t* b_ready = zfree + 2;         // the builder warps wrote B
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_ready + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunks = p.K / kTile;
@@ -119,18 +147,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&zfull[i], 1);
       mbar_init(&zfree[i], kRowWarps);
     }
+    mbar_init(b_ready, kBuilders / 32);
     fence_barrier_init();
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
-  build_rotation_operand(smem + kOffB, p, c, threadIdx.x, kThreads);
-  fence_proxy_async();  // B is read by the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // B is built while the first x tiles are in flight; the MMA warp waits for it
+  if (warp >= kBuildWarp0) {
+    build_rotation_operand(smem + kOffB, reinterpret_cast<uint32_t*>(smem + kOffStage), p, c,
+                           threadIdx.x - 32 * kBuildWarp0, kBuilders);
+    fence_proxy_async();  // B is read by the tensor core
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_ready);
+  }
   // Stats reads x, which the kernel before it may write: wait for it, then let
   // Quantise start (Quantise therefore sees final x without waiting itself).
   if constexpr (MODE == 1) griddep_wait();
@@ -166,7 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t bs = smem_u32(smem + kOffB);
       int i = 0;
-      for (int t = g0; t < tiles; t += groups, ++i) {
+      const bool bok = mbar_wait(b_ready, 0, p.err, DEVERR_MMA_WAIT);
+      for (int t = g0; bok && t < tiles; t += groups, ++i) {
         const int slot = i % kSlots, d = i & 1;
         if (!mbar_wait(&full[slot], (i / kSlots) & 1, p.err, DEVERR_MMA_WAIT)) break;
         if (!mbar_wait(&zfree[d], ((i >> 1) & 1) ^ 1u, p.err, DEVERR_MMA_WAIT)) break;
@@ -250,7 +286,8 @@ constexpr int kOnePassMaxTiles = 6;
 constexpr int kOffRing = kOffB + 2 * kXBytes;     // ring slots 0, 1 (tiles 0, 1, then 2)
 constexpr int kOffKeep = kOffRing + 2 * kXBytes;  // x of tiles 3, 4, 5, kept for phase 2
 constexpr int kOffBar1 = kOffKeep + 3 * kXBytes;
-constexpr int kSmem1 = kOffBar1 + 256 + 1024;
+constexpr int kOffStage1 = kOffBar1 + 256;
+constexpr int kSmem1 = kOffStage1 + 512 + 1024;
 static_assert(kSmem1 <= 227 * 1024, "shared memory budget");
 constexpr int kBarCountOffset = 12;               // bytes after the amax word
 
@@ -271,8 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ring_free = bars + 6;        // MMAs of tile 0 done with ring slot 0
   uint64_t* zfull = bars + 7;            // [4] Z of a tile in TMEM buffer d
   uint64_t* zfree = bars + 11;           // [4] row warps done with buffer d
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
-  int* grid_ok = reinterpret_cast<int*>(bars + 16);
+  uint64_t* b_ready = bars + 15;         // the builder warps wrote B
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  int* grid_ok = reinterpret_cast<int*>(bars + 17);
   uint32_t* bar_count = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.amax_glob) + kBarCountOffset);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -292,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&zfull[i], 1);
       mbar_init(&zfree[i], kRowWarps);
     }
+    mbar_init(b_ready, kBuilders / 32);
     *grid_ok = 1;
     fence_barrier_init();
   }
@@ -299,12 +338,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  build_rotation_operand(smem + kOffB, p, c, threadIdx.x, kThreads);
-  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // B is built while the first x tiles are in flight; the MMA warp waits for it
+  if (warp >= kBuildWarp0) {
+    build_rotation_operand(smem + kOffB, reinterpret_cast<uint32_t*>(smem + kOffStage1), p, c,
+                           threadIdx.x - 32 * kBuildWarp0, kBuilders);
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_ready);
+  }
   griddep_wait();
   griddep_launch_dependents();
 
@@ -335,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t bs = smem_u32(smem + kOffB);
       int n3 = 0;  // MMAs issued into buffer 3 so far
-      bool ok = true;
+      bool ok = mbar_wait(b_ready, 0, p.err, DEVERR_MMA_WAIT);
       for (int k = 0; ok && k < kOnePassMaxTiles; ++k) {  // phase 1
         const int i = onepass_order(k);
         if (i >= n) continue;
@@ -403,18 +448,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     named_bar(1, 32 * kRowWarps);  // every row warp of this CTA published
     if (rw == 0 && lane == 0) {
+      // the CTA's maxima (ordered before this by the named barrier) are made
+      // visible device-wide by a full fence before the arrival; then poll with
+      // acquire order until every CTA has arrived
       __threadfence();
       atomicAdd(bar_count, 1u);
       const uint64_t t0 = global_timer_ns();
-      while (*reinterpret_cast<volatile uint32_t*>(bar_count) < gridDim.x) {
+      for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar_count) : "memory");
+        if (v >= gridDim.x) break;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
           atomicOr(p.err, DEVERR_GRID_WAIT);
           *grid_ok = 0;
           break;
         }
-        __nanosleep(128);
       }
-      __threadfence();
     }
     __syncwarp();  // the named barrier is warp-aligned: lane 0 rejoins first
     named_bar(1, 32 * kRowWarps);

@@ -56,7 +56,8 @@ typedef enum {
   QWAM_ERR_ARCH = 4,        /* current device is not compute capability 10.x */
   QWAM_ERR_OOM = 5,         /* device allocation failed */
   QWAM_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed */
-  QWAM_ERR_TIMEOUT = 7      /* a bounded device wait expired (qwam_device_error) */
+  QWAM_ERR_TIMEOUT = 7,     /* a bounded device wait expired (qwam_device_error) */
+  QWAM_ERR_FORMAT = 8       /* a layer image is malformed or fails its checksum */
 } qwam_status;
 
 /* ---------------------------------------------------------------------------
@@ -116,6 +117,39 @@ qwam_status qwam_prepare_weight_fp8(const void* W_bf16, int N, int K, const floa
 /* Host outputs (each may be NULL): the element format of the handle (0 NVFP4,
  * 1 FP8 E4M3) and its weight arm (0 deflated, 1 shared-weight). */
 qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant);
+
+/* ---------------------------------------------------------------------------
+ * Layer images (card "FastWAM UR3 3-task -- 4-bit quantisations", section
+ * "Files": the NVFP4 deflated-ASP checkpoint stores packed E2M1 weights and
+ * E4M3 block scales already in the tensor-core tile layout, and is
+ * self-contained).  A prepared layer as one host byte string, so that a
+ * checkpoint is quantised once and loaded without the bf16 weight.
+ *
+ * Layout (little-endian): a 64-byte header {char magic[8] = "QWAMIMG\0";
+ * uint32 version = 1; uint32 header_bytes = 64; int32 N, K, r, b, fmt,
+ * variant; uint32 flags (bit 0: bias present); float g_w; uint64
+ * total_bytes; uint64 checksum}, then these arrays, each zero-padded to a
+ * multiple of 16 bytes: codes (N * K/2 bytes; FP8: N * K), block scales
+ * (NVFP4 only: round_up(N,256) * K/16 bytes, tiled as on the device), and
+ * when r > 0: L bf16 [N, r], V hi and lo bf16 [K, r] each, P^T hi and lo
+ * bf16 [r, K] each; then 1/s fp32 [K]; then bias bf16 [N] when flag bit 0
+ * is set.  checksum = FNV-1a 64 (offset basis 0xcbf29ce484222325, prime
+ * 0x100000001b3) over all total_bytes with the checksum field read as zero.
+ *
+ * qwam_image_size: *bytes = the image length of h (host call, no device work).
+ * qwam_save_image: writes the image of h into host_buf (host memory, pageable
+ *   or pinned, at least qwam_image_size bytes; QWAM_ERR_INVALID_ARG if
+ *   shorter).  Copies on `stream` and synchronises it.
+ * qwam_load_image: checks the image on the host first (magic, version, a
+ *   valid shape and format, total_bytes against the shape and buf_bytes, the
+ *   checksum: QWAM_ERR_FORMAT on any mismatch, with nothing allocated), then
+ *   makes a new handle on the current device whose calls return exactly what
+ *   the saved handle's calls return.  The caller keeps host_buf; the call
+ *   synchronises `stream`.
+ * ------------------------------------------------------------------------- */
+qwam_status qwam_image_size(qwam_handle h, size_t* bytes);
+qwam_status qwam_save_image(qwam_handle h, void* host_buf, size_t buf_bytes, void* stream);
+qwam_status qwam_load_image(const void* host_buf, size_t buf_bytes, void* stream, qwam_handle* out);
 
 /* Release a handle and its device memory (synchronises the device). */
 qwam_status qwam_destroy(qwam_handle h);
