@@ -26,8 +26,9 @@ single layers (c2 action attention 32 x 1024 -> 1024, c3 video attention
 4096 x 3072 -> 3072 at r = 32 and r = 0, c4 video FFN up and down), the
 action-expert half of the step (c5action), and the boundary's other arms on
 the same layers (c3r0fp8 / c2fp8: the FP8 W8A8 arm, against the FP8 peak;
-c2shared: the shared-weight arm), each with its own roofline, cpu_baseline and
-e2e.  --workload <name> runs one of those alone.
+c2shared: the shared-weight arm; c3int4 / c2int4: the SVDQuant INT4 arm,
+whose products run on the FP8 tensor-core kind), each with its own roofline,
+cpu_baseline and e2e.  --workload <name> runs one of those alone.
 
 Timing: CUDA events around K steps replayed from a CUDA graph (one untimed
 replay first), barrier + synchronize on both sides, max over ranks.  Multi-GPU
@@ -60,6 +61,9 @@ METRIC = "ASP-NVFP4 linear TFLOP/s and GB/s per layer, % of FP4/HBM roofline"
 L2_BYTES = 126 * 10 ** 6
 DTYPE = "nvfp4 (e2m1 x e4m3 block-16) GEMM, fp32 accumulate; bf16 in/out; bf16 rank-r branch"
 DTYPE_FP8 = "fp8 e4m3 (per-tensor scales) GEMM, fp32 accumulate; bf16 in/out; bf16 rank-r branch"
+DTYPE_INT4 = ("int4 group-64 (fp16 scales) levels as e4m3 on f8f6f4 tensor cores, exact group sums, fp32 "
+              "rescale per group; bf16 in/out; bf16 rank-r branch")
+DTYPES = {"nvfp4": DTYPE, "fp8": DTYPE_FP8, "int4": DTYPE_INT4}
 
 STEP = dict(desc="one denoising step of the 2-expert model: 600 linears (video d 3072, ffn 14336, 4096 tokens, "
                  "r=0; action d 1024, ffn 4096, 32 tokens, cross k/v over the 4096-token context, r=32), b=128",
@@ -104,12 +108,21 @@ WORKLOADS = {
     "c2shared": dict(make=lambda i, seed: workloads.c2_action_attn(seed=seed, layer=i), variant="shared",
                      desc="shared-weight arm: action-expert attention projection, 32 tokens, 1024->1024, r=32, "
                           "b=128", unit="GB/s", steps=200000, warmup=50),
+    "c3int4": dict(make=lambda i, seed: workloads.c3_video_attn_int4(seed=seed, layer=i), fmt="int4",
+                   variant="svdquant",
+                   desc="SVDQuant INT4 arm: video-expert attention projection, 4096 tokens, 3072->3072, r=32, "
+                        "no rotation", unit="TFLOP/s", steps=2000, warmup=10),
+    "c2int4": dict(make=lambda i, seed: workloads.c2_action_attn_int4(seed=seed, layer=i), fmt="int4",
+                   variant="svdquant",
+                   desc="SVDQuant INT4 arm: action-expert attention projection, 32 tokens, 1024->1024, r=32, "
+                        "no rotation", unit="GB/s", steps=200000, warmup=50),
 }
 
 # per_config entries of the default run: (steps, warm-up, seconds of oracle work)
 PER_CONFIG = {"c2": (20000, 50, 8.0), "c3": (400, 10, 8.0), "c3r0": (400, 10, 8.0), "c4up": (100, 5, 8.0),
               "c4down": (100, 5, 8.0), "c5action": (10, 3, 8.0), "c3r0fp8": (400, 10, 6.0),
-              "c2fp8": (20000, 50, 6.0), "c2shared": (20000, 50, 6.0)}
+              "c2fp8": (20000, 50, 6.0), "c2shared": (20000, 50, 6.0), "c3int4": (400, 10, 6.0),
+              "c2int4": (20000, 50, 6.0)}
 
 
 def set_layers(wl):
@@ -130,10 +143,18 @@ def step_kinds(specs):
 # ---------------------------------------------------------------------------
 # Algorithmic work per layer (minimal bytes / flops of the method itself).
 # ---------------------------------------------------------------------------
+def elem_bytes(fmt):
+    """Bytes of one quantised element with its share of the scales, as the
+    format stores it: NVFP4 0.5 + 1/16 (E4M3 per 16), FP8 1, INT4 0.5 + 2/64
+    (fp16 per 64; the device holds the levels as bytes, which the algorithmic
+    count does not credit)."""
+    return {"nvfp4": 0.5625, "fp8": 1.0, "int4": 0.53125}[fmt]
+
+
 def layer_bytes(M, K, N, r, fmt="nvfp4"):
-    """x (bf16) + packed W_d with E4M3 scales (0.5625 B/weight; FP8 arm: 1 B) +
-    L (bf16) + V (fp32) + s (fp32) + bias (bf16) + y (bf16)."""
-    wb = 1.0 if fmt == "fp8" else 0.5625
+    """x (bf16) + the quantised weight with its scales (elem_bytes) + L (bf16)
+    + V (fp32) + s (fp32) + bias (bf16) + y (bf16)."""
+    wb = elem_bytes(fmt)
     return 2 * M * K + wb * N * K + 2 * N * r + 4 * K * r + 4 * K + 2 * N + 2 * M * N
 
 
@@ -142,15 +163,15 @@ def layer_flops(M, K, N, r):
 
 
 def prologue_bytes(M, K, N, r, fmt="nvfp4"):
-    """Reads x, V, s; writes FP4 codes + scales (0.5625 B/element; FP8: 1 B)
-    and u'."""
-    eb = 1.0 if fmt == "fp8" else 0.5625
+    """Reads x, V, s; writes the quantised activation (elem_bytes) and u'."""
+    eb = elem_bytes(fmt)
     return 2 * M * K + 4 * K * r + 4 * K + eb * M * K + 2 * M * r
 
 
 def gemm_bytes(M, K, N, r, fmt="nvfp4"):
-    """Reads FP4 (FP8) activations + scales, W_d + scales, L, u', bias; writes y."""
-    eb = 1.0 if fmt == "fp8" else 0.5625
+    """Reads the quantised activations and weights (elem_bytes), L, u', bias;
+    writes y."""
+    eb = elem_bytes(fmt)
     return eb * M * K + eb * N * K + 2 * N * r + 2 * M * r + 2 * N + 2 * M * N
 
 
@@ -288,7 +309,7 @@ def oracle_call(prep, case, fmt="nvfp4"):
     """The per-call work of the layer in the float64 oracle: activation side,
     FP4 (FP8) product on dequantised operands, low-rank branch, bias."""
     from oracle import asp
-    act = asp.activation_prologue(case.x, case.s, case.V, case.b, fmt=fmt)
+    act = asp.activation_prologue(case.x, case.s, case.V, case.b, fmt=fmt, deflated=fmt != "int4")
     y = asp.nvfp4_gemm(act["deq"], prep["deq"]) + act["u"] @ prep["L"].T + case.bias.astype("float64")[None, :]
     return y
 
@@ -433,7 +454,8 @@ def hbm_roof(kernel, nbytes, dur_ms, peaks):
 
 def tensor_roof(kernel, flops, dur_ms, peaks, timed_alone, fmt="nvfp4"):
     achieved = flops / (dur_ms / 1e3) / 1e12
-    peak, other, note = (fp8_peak if fmt == "fp8" else fp4_peak)(peaks, timed_alone)
+    # the INT4 arm's products run on kind::f8f6f4: the FP8 peak
+    peak, other, note = (fp4_peak if fmt == "nvfp4" else fp8_peak)(peaks, timed_alone)
     r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "peak_note": note,
          "frac": achieved / peak, "kernel": kernel}
     r["frac_sustained" if timed_alone else "frac_burst"] = achieved / other
@@ -450,7 +472,8 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     probe = wl["make"](0, args.seed)
     M, K, N, r, hb = probe.M, probe.K, probe.N, probe.r, probe.b
     warmup = max(3, warmup)
-    per_inst = (N * K / 2 + N * K / 16 + 2 * N * max(r, 1) + 8 * K * max(r, 1) + 4 * K + 2 * N
+    wdev = {"nvfp4": 0.5625, "fp8": 1.0, "int4": 1.0625}[fmt]  # device bytes per weight
+    per_inst = (wdev * N * K + 2 * N * max(r, 1) + 8 * K * max(r, 1) + 4 * K + 2 * N
                 + 2 * M * K + 2 * M * N)
     P = args.instances or max(1, min(256, math.ceil(1.5 * L2_BYTES / per_inst)))
     handles, xs, ys = [], [], []
@@ -549,10 +572,11 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     peaks = measured_peaks()
     pro_avg, gem_avg = sum(pro_ms) / G, sum(gem_ms) / G
     dominant = "gemm" if gem_avg >= pro_avg else "prologue"
+    gemm_kernel = "group_gemm_kernel" if fmt == "int4" else "fp4_gemm_kernel"
     if dominant == "gemm" and unit == "TFLOP/s":
-        roof = tensor_roof("fp4_gemm_kernel", gemm_flops(M, K, N, r), gem_avg, peaks, timed_alone=True, fmt=fmt)
+        roof = tensor_roof(gemm_kernel, gemm_flops(M, K, N, r), gem_avg, peaks, timed_alone=True, fmt=fmt)
     elif dominant == "gemm":
-        roof = hbm_roof("fp4_gemm_kernel", gemm_bytes(M, K, N, r, fmt), gem_avg, peaks)
+        roof = hbm_roof(gemm_kernel, gemm_bytes(M, K, N, r, fmt), gem_avg, peaks)
     else:
         roof = hbm_roof("prologue_kernel", prologue_bytes(M, K, N, r, fmt), pro_avg, peaks)
     roof["traffic"] = recorded_traffic(name, roof["kernel"])
@@ -565,7 +589,7 @@ def bench_layer(ctx, args, name, steps, warmup, cpu_budget):
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": ctx.world, "steps": steps, "warmup": warmup,
         "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": DTYPE_FP8 if fmt == "fp8" else DTYPE,
+        "dtype": DTYPES[fmt],
         "data": "synthetic (seeded; shapes of the Fast-WAM experts, random-init weights)",
         "config": {"workload": f"{name}: {wl['desc']}", "M": M, "K": K, "N": N, "r": r, "hadamard_block": hb,
                    "parallelism": f"replicas x{ctx.world}",

@@ -30,6 +30,8 @@ SIGNATURES = {
     "qwam_debug_prepare_weight": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     "qwam_prepare_weight_shared": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     "qwam_prepare_weight_fp8": (_I, [_P, _I, _I, _P, _P, _I, _P, _I, _P, _P, ctypes.POINTER(_P)]),
+    "qwam_prepare_weight_int4": (_I, [_P, _I, _I, _P, _P, _I, _P, _P, _P, ctypes.POINTER(_P)]),
+    "qwam_int4_gemm": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "qwam_handle_format": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "qwam_image_size": (_I, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "qwam_save_image": (_I, [_P, _P, ctypes.c_size_t, _P]),
@@ -125,13 +127,13 @@ class Handle:
         self.N, self.K, self.r, self.b, self.g_w = N.value, K.value, r.value, b.value, gw.value
         fmt, var = _I(), _I()
         _check(load().qwam_handle_format(raw, ctypes.byref(fmt), ctypes.byref(var)))
-        self.fmt = "fp8" if fmt.value == 1 else "nvfp4"
-        self.variant = "shared" if var.value == 1 else "deflated"
+        self.fmt = {0: "nvfp4", 1: "fp8", 2: "int4"}[fmt.value]
+        self.variant = {0: "deflated", 1: "shared", 2: "svdquant"}[var.value]
 
     @property
     def code_bytes(self) -> int:
-        """Bytes of one row of codes: K / 2 (NVFP4) or K (FP8)."""
-        return self.K if self.fmt == "fp8" else self.K // 2
+        """Bytes of one row of codes: K / 2 (NVFP4) or K (FP8; INT4 levels as E4M3 bytes)."""
+        return self.K // 2 if self.fmt == "nvfp4" else self.K
 
     @property
     def raw(self) -> int:
@@ -165,8 +167,10 @@ def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None,
     """W bf16 [N, K], s fp32 [K], V fp32 [K, r] or None, bias bf16 [N] or None.
     variant "deflated" (qwam_prepare_weight) or "shared" (the shared-weight
     arm, qwam_prepare_weight_shared); fmt "nvfp4" or "fp8" (the W8A8 arm,
-    qwam_prepare_weight_fp8, deflated only).  wd_out (fp32 [N, K]) receives
-    the exact quantiser input: W_d for the deflated arm, W~ for the shared one."""
+    qwam_prepare_weight_fp8, deflated only); fmt "int4" with variant
+    "svdquant" (the SVDQuant arm, qwam_prepare_weight_int4, hadamard_block 1).
+    wd_out (fp32 [N, K]) receives the exact quantiser input: W_d for the
+    deflated arm, W~ for the shared one, the residual R for SVDQuant."""
     import torch
     lib = load()
     N, K = W.shape
@@ -178,13 +182,17 @@ def prepare_weight(W, s, V, bias, hadamard_block: int, stream=None, wd_out=None,
     if bias is not None:
         _need(bias, torch.bfloat16, (N,), "bias")
     out = _P()
-    if variant not in ("deflated", "shared"):
-        raise ValueError(f"variant must be 'deflated' or 'shared', got {variant!r}")
-    if fmt not in ("nvfp4", "fp8") or (fmt == "fp8" and variant != "deflated"):
-        raise ValueError(f"format {fmt!r} with variant {variant!r}")
+    if variant not in ("deflated", "shared", "svdquant"):
+        raise ValueError(f"variant must be 'deflated', 'shared' or 'svdquant', got {variant!r}")
+    if (fmt not in ("nvfp4", "fp8", "int4") or (fmt == "fp8" and variant != "deflated")
+            or ((fmt == "int4") != (variant == "svdquant")) or (fmt == "int4" and hadamard_block != 1)):
+        raise ValueError(f"format {fmt!r} with variant {variant!r} and block {hadamard_block}")
     if wd_out is not None:
         _need(wd_out, torch.float32, (N, K), "wd_out")
-    if fmt == "fp8":
+    if fmt == "int4":
+        _check(lib.qwam_prepare_weight_int4(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), _ptr(wd_out),
+                                            _stream(stream), ctypes.byref(out)))
+    elif fmt == "fp8":
         _check(lib.qwam_prepare_weight_fp8(_ptr(W), N, K, _ptr(s), _ptr(V), r, _ptr(bias), hadamard_block,
                                            _ptr(wd_out), _stream(stream), ctypes.byref(out)))
     elif variant == "shared":
@@ -267,6 +275,22 @@ def debug_prologue(x, h: Handle, stream=None) -> dict:
     _check(load().qwam_debug_prologue(_ptr(x), M, h.raw, _ptr(z), _ptr(u) if h.r else None, _ptr(codes),
                                       _ptr(sf), _ptr(ub) if h.r else None, _ptr(gx), _stream(stream)))
     return {"z": z, "u": u[:, :h.r], "codes": codes, "scales": sf, "ub": ub[:, :h.r], "g_x": gx}
+
+
+def int4_gemm(a_levels, a_scales, b_levels, b_scales, stream=None):
+    """qwam_int4_gemm: a_levels u8 [M, K], a_scales fp32 [K/64, M], b_levels
+    u8 [N, K], b_scales fp32 [K/64, N] (device) -> fp32 [M, N]."""
+    import torch
+    M, K = a_levels.shape
+    N = b_levels.shape[0]
+    _need(a_levels, torch.uint8, (M, K), "a_levels")
+    _need(b_levels, torch.uint8, (N, K), "b_levels")
+    _need(a_scales, torch.float32, (K // 64, M), "a_scales")
+    _need(b_scales, torch.float32, (K // 64, N), "b_scales")
+    out = torch.empty((M, N), dtype=torch.float32, device=a_levels.device)
+    _check(load().qwam_int4_gemm(_ptr(a_levels), _ptr(a_scales), _ptr(b_levels), _ptr(b_scales), M, N, K, _ptr(out),
+                                 _stream(stream)))
+    return out
 
 
 def quantize_fp32(T, stream=None):

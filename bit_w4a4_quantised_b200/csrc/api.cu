@@ -175,7 +175,8 @@ qwam_status make_codes_map(CUtensorMap* m, const void* base, int rows, int row_b
 }
 
 // Bytes of one operand row of K elements, and of one stage of ks elements.
-inline int code_bytes(int K, int fmt) { return fmt == 1 ? K : K / 2; }
+// (FP8 E4M3 and the INT4 arm's levels as E4M3 bytes: one byte per element)
+inline int code_bytes(int K, int fmt) { return fmt == 1 || fmt == 2 ? K : K / 2; }
 
 CUtensorMapSwizzle branch_swizzle(int r) { return r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B; }
 
@@ -210,6 +211,17 @@ Plan plan_gemm(int M, int N, int K, int sms, int fmt) {
   return p;
 }
 
+// INT4 arm: K splits of the group GEMM when its 128 x 128 output tiles leave
+// SMs idle: the largest count up to 16 with tiles * splits within one wave and
+// at least one stage (K 128) per split.
+int group_splits(int M, int N, int K, int sms) {
+  const int tiles = ((M + 127) / 128) * ((N + 127) / 128);
+  const int k_stages = K / 128;
+  int s = 1;
+  while (s * 2 <= 16 && s * 2 <= k_stages && tiles * s * 2 <= sms) s *= 2;
+  return s;
+}
+
 // ---- per-device workspace --------------------------------------------------
 struct Arena {
   uint8_t* base = nullptr;
@@ -219,10 +231,13 @@ std::mutex g_arena_mu;
 Arena g_arena[kMaxDevices];
 
 struct Layout {
-  size_t codes, sf, u, ub, total;
+  size_t codes, sf, u, ub, part, total;
 };
 
-Layout layout_for(int M, int K, int r, int fmt) {
+// part_bytes: the INT4 arm's split-K partial tiles (0 otherwise).  Its
+// activation scales are fp32 [K / 64][round_up(M, 128)], the same bytes as the
+// NVFP4 tiles.
+Layout layout_for(int M, int K, int r, int fmt, size_t part_bytes = 0) {
   Layout L{};
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
@@ -236,6 +251,7 @@ Layout layout_for(int M, int K, int r, int fmt) {
   L.sf = take(fmt == 1 ? 16 : Mp * K / 16);  // FP8: no block scales
   L.u = take(static_cast<size_t>(M) * rr * 4);
   L.ub = take(Mp * rr * 2);
+  L.part = take(part_bytes);
   L.total = off;
   return L;
 }
@@ -294,6 +310,8 @@ struct CallPlan {
   PrologueParams prm{};
   GemmMaps gmaps{};
   GemmParams gp{};
+  GroupGemmMaps ggmaps{};  // INT4 arm
+  GroupGemmParams ggp{};
 };
 
 }  // namespace
@@ -301,8 +319,8 @@ struct CallPlan {
 struct qwam_layer {
   uint32_t magic;
   int N, K, r, b, dev;
-  int fmt;      // 0 NVFP4 (W4A4), 1 FP8 E4M3 (W8A8)
-  int variant;  // 0 deflated, 1 shared-weight
+  int fmt;      // 0 NVFP4 (W4A4), 1 FP8 E4M3 (W8A8), 2 INT4 group 64 (the SVDQuant arm)
+  int variant;  // 0 deflated, 1 shared-weight, 2 SVDQuant
   uint8_t* codes;
   uint8_t* sf;
   uint16_t* L;
@@ -316,6 +334,7 @@ struct qwam_layer {
   size_t sf_bytes;
   CUtensorMap map_b128_k128, map_b128_k256, map_b256_k256, map_l128, map_l256;
   CUtensorMap map_sfb_k128, map_sfb_k256_b1, map_sfb_k256_b2;  // B scales: K per stage, 128-row blocks per box
+  CUtensorMap map_sgb;  // INT4: B scales fp32 [K / 64][N], box 128 columns x 2 groups
   ProMaps vmaps;  // P^T and V (hi/lo) tensor maps for the prologue; x is per call
   // Launch arguments of the last call, kept per scratch kind (0: the growable
   // workspace, 1: the static scratch of qwam_linear_noalloc) so that repeated
@@ -370,7 +389,7 @@ bool use_fused(int rows) { return rows <= 128; }
 // two launches (Stats, Quantise), with the rotation folded into the tensor-core
 // operand when there is no subspace (r = 0), else the row pipeline with the
 // rank-r projection and deflation.
-enum { PRO_FUSED = 0, PRO_TWO_PASS = 1, PRO_WIDE = 2, PRO_ONEPASS = 3 };
+enum { PRO_FUSED = 0, PRO_TWO_PASS = 1, PRO_WIDE = 2, PRO_ONEPASS = 3, PRO_LOCAL = 4 };
 int prologue_form(int rows, int r, int K, int sms) {
   if (use_fused(rows)) return PRO_FUSED;
   if (r != 0) return PRO_TWO_PASS;
@@ -405,7 +424,9 @@ qwam_status run_rows(const void* T, PrologueParams prm, int r, const ProMaps& vm
   prm.amax_glob = amax;
   prm.parts = cluster_parts(prm.K, prm.rows, sms);
   prm.chunks = prm.K / 128 / prm.parts;
-  return launch_rows(maps, prm, r, false, st);
+  // INT4 (local group scales): the one-launch form at any row count, whose
+  // CUDA-core scaling gives W~ = RN(W * s) exactly (b = 1)
+  return launch_rows(maps, prm, r, prm.fmt == 2, st);
 }
 
 // shared: the shared-weight arm (quantise W~ itself; L = deq(Q(W~)) V) instead
@@ -416,8 +437,16 @@ size_t layer_code_bytes(const qwam_layer* h) { return static_cast<size_t>(h->N) 
 size_t layer_branch_bytes(const qwam_layer* h) { return static_cast<size_t>(h->N) * std::max(h->r, 1) * 2; }
 size_t layer_v_bytes(const qwam_layer* h) { return static_cast<size_t>(h->K) * std::max(h->r, 1) * 2; }
 
+// Bytes of the weight scales: NVFP4 tiles (rows padded to 256), none for FP8
+// (a 16-byte placeholder), fp32 [K / 64][N] for INT4.
+size_t layer_sf_bytes(int N, int K, int fmt) {
+  if (fmt == 1) return 16;
+  if (fmt == 2) return static_cast<size_t>(N) * K / 16;
+  return round_up(static_cast<size_t>(N), 256) * K / 16;
+}
+
 qwam_status alloc_layer(qwam_layer* h, bool with_bias) {
-  h->sf_bytes = h->fmt == 1 ? 16 : round_up(static_cast<size_t>(h->N), 256) * h->K / 16;
+  h->sf_bytes = layer_sf_bytes(h->N, h->K, h->fmt);
   const size_t K = static_cast<size_t>(h->K);
   QW_TRY(dmalloc(&h->codes, layer_code_bytes(h)));
   QW_TRY(dmalloc(&h->sf, h->sf_bytes));
@@ -463,7 +492,11 @@ qwam_status finish_layer(qwam_layer* h, cudaStream_t st) {
   QW_TRY(make_codes_map(&h->map_b128_k128, h->codes, N, cb, 64, 128));
   QW_TRY(make_codes_map(&h->map_b128_k256, h->codes, N, cb, 128, 128));
   QW_TRY(make_codes_map(&h->map_b256_k256, h->codes, N, cb, 128, 256));
-  if (h->fmt == 1) {  // no block scales: the unread scale maps alias the codes map
+  h->map_sgb = h->map_b128_k128;  // unread unless INT4
+  if (h->fmt == 2)
+    QW_TRY(make_map(&h->map_sgb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, h->sf, N, K / 64, static_cast<uint64_t>(N) * 4, 128,
+                    2, CU_TENSOR_MAP_SWIZZLE_NONE));
+  if (h->fmt != 0) {  // no NVFP4 block scales: the unread scale maps alias the codes map
     h->map_sfb_k128 = h->map_sfb_k256_b1 = h->map_sfb_k256_b2 = h->map_b128_k128;
   } else {
     const size_t rows = round_up(static_cast<size_t>(N), 256);
@@ -504,7 +537,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   QW_TRY(current_device(&dev));
   cudaStream_t st = as_stream(stream);
 
-  qwam_layer* h = new_layer(N, K, r, b, dev, fmt, shared ? 1 : 0);
+  qwam_layer* h = new_layer(N, K, r, b, dev, fmt, fmt == 2 ? 2 : (shared ? 1 : 0));
   float* u_tmp = nullptr;
   uint32_t* scratch = nullptr;  // [0] amax, [1] err, [2] g_w (fp32)
   uint16_t *pw_hi = nullptr, *pw_lo = nullptr;  // P^T of the weight side, diag(s) H V
@@ -568,6 +601,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   prm.z_out = wd_out;
   prm.err = scratch + 3;
   prm.fmt = fmt;
+  prm.sf_pitch = N;  // INT4 weight scales [K / 64][N]
   if (shared && r > 0) {
     // W~ itself through the row pipeline (no projection, no deflation), then
     // the branch weight from the stored FP4 weight
@@ -584,6 +618,7 @@ qwam_status prepare_impl(const void* W, int N, int K, const float* s, const floa
   if (host_scr[1]) return cleanup(fail(QWAM_ERR_INVALID_ARG, "smoothing vector s has an entry that is <= 0 or not finite"));
   if (host_scr[3]) return cleanup(fail(QWAM_ERR_TIMEOUT, "a bounded device wait expired in prepare (flags 0x%x)", host_scr[3]));
   std::memcpy(&h->g_w, &host_scr[2], 4);
+  if (fmt == 2) h->g_w = 1.0f;  // INT4: every scale is a group scale
 
   cudaFree(s_pm);
   cudaFree(u_tmp);
@@ -613,13 +648,23 @@ qwam_status make_y_map(CUtensorMap* m, const void* y, int N, int M, bool pair) {
                   pair ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// The workspace layout of an M-row call of layer h.
+Layout layout_of(const qwam_layer* h, int M) {
+  size_t part = 0;
+  if (h->fmt == 2) {
+    const int sp = group_splits(std::max(M, 1), h->N, h->K, sm_count(h->dev));
+    if (sp > 1) part = static_cast<size_t>(sp) * M * h->N * 4;
+  }
+  return layout_for(M, h->K, h->r, h->fmt, part);
+}
+
 // Launch arguments for M rows of layer h with scratch at ws: the workspace
-// layout of layout_for (scalars at ws: amax, g_x, error word).
+// layout of layout_of (scalars at ws: amax, g_x, error word).
 qwam_status build_call(qwam_handle h, int M, uint8_t* ws, CallPlan* c) {
   c->M = -1;
   const int sms = sm_count(h->dev);
   const Plan pl = plan_gemm(M, h->N, h->K, sms, h->fmt);
-  const Layout lay = layout_for(M, h->K, h->r, h->fmt);
+  const Layout lay = layout_of(h, M);
   PrologueParams prm{};
   prm.chan = h->inv_s_pm;
   prm.rows = M;
@@ -638,6 +683,46 @@ qwam_status build_call(qwam_handle h, int M, uint8_t* ws, CallPlan* c) {
   prm.parts = cluster_parts(h->K, M, sms);
   prm.chunks = h->K / 128 / prm.parts;
   prm.fmt = h->fmt;
+
+  if (h->fmt == 2) {
+    // SVDQuant arm: the Local prologue (b = 1, INT4 quantised as read, bf16(c)
+    // for the branch) and the group GEMM (+ the split-K sum)
+    const int Mp = static_cast<int>(round_up(static_cast<size_t>(M), 128));
+    prm.branch_mode = 0;
+    prm.sf_pitch = Mp;
+    GroupGemmMaps gg{};
+    QW_TRY(make_codes_map(&gg.a, ws + lay.codes, M, h->K, 128, 128));
+    gg.b = h->map_b128_k256;
+    QW_TRY(make_map(&gg.sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws + lay.sf, M, h->K / 64, static_cast<uint64_t>(Mp) * 4,
+                    128, 2, CU_TENSOR_MAP_SWIZZLE_NONE));
+    gg.sb = h->map_sgb;
+    if (h->r > 0) {
+      QW_TRY(make_map(&gg.u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + lay.ub, h->r, M, h->r * 2, h->r, 128,
+                      branch_swizzle(h->r)));
+      gg.l = h->map_l128;
+    } else {
+      gg.u = gg.sa;  // unread
+      gg.l = gg.sb;
+    }
+    GroupGemmParams gq{};
+    gq.M = M; gq.N = h->N; gq.K = h->K;
+    gq.splits = group_splits(M, h->N, h->K, sms);
+    gq.branch_k = h->r;
+    gq.bias = h->bias;
+    gq.partial = gq.splits > 1 ? reinterpret_cast<float*>(ws + lay.part) : nullptr;
+    gq.err = prm.err;
+    c->pl = pl;
+    c->pro_form = PRO_LOCAL;
+    c->pro_groups = 0;
+    c->pmaps = h->vmaps;
+    c->prm = prm;
+    c->ggmaps = gg;
+    c->ggp = gq;
+    c->x = c->y = nullptr;
+    c->ws = ws;
+    c->M = M;
+    return QWAM_OK;
+  }
 
   GemmMaps gm{};
   QW_TRY(make_codes_map(&gm.a, ws + lay.codes, M, code_bytes(h->K, h->fmt), pl.wide ? 128 : 64, 128));
@@ -704,6 +789,11 @@ qwam_status bind_x(qwam_handle h, CallPlan* c, const void* x) {
 }
 
 qwam_status bind_y(qwam_handle h, CallPlan* c, void* y) {
+  if (h->fmt == 2) {  // plain stores; with split K the final sum writes y
+    c->ggp.y = c->ggp.splits == 1 ? y : nullptr;
+    c->y = y;
+    return QWAM_OK;
+  }
   c->gp.y = y;
   if (y == c->y || c->pl.splits > 1) {
     c->y = y;
@@ -716,6 +806,10 @@ qwam_status bind_y(qwam_handle h, CallPlan* c, void* y) {
 }
 
 qwam_status launch_call_prologue(const CallPlan& c, const PrologueParams& prm, int r, cudaStream_t st) {
+  if (c.pro_form == PRO_LOCAL) {
+    QW_CUDA(launch_prologue(c.pmaps, prm, r, PrologueMode::Local, st));
+    return QWAM_OK;
+  }
   if (c.pro_form == PRO_ONEPASS) {
     QW_CUDA(cudaMemsetAsync(prm.amax_glob, 0, 16, st));  // amax, g_x, grid-barrier count
     QW_CUDA(launch_prologue_onepass(c.pmaps.x, prm, c.pro_groups, st));
@@ -731,6 +825,12 @@ qwam_status launch_call_prologue(const CallPlan& c, const PrologueParams& prm, i
 }
 
 qwam_status launch_call_gemm(const CallPlan& c, cudaStream_t st) {
+  if (c.pro_form == PRO_LOCAL) {
+    QW_CUDA(launch_group_gemm(c.ggmaps, c.ggp, st));
+    if (c.ggp.splits > 1)
+      QW_CUDA(launch_splitk_finalize(c.ggp.partial, c.ggp.splits, c.M, c.ggp.N, c.ggp.bias, const_cast<void*>(c.y), st));
+    return QWAM_OK;
+  }
   QW_CUDA(launch_gemm(c.gmaps, c.gp, GemmShape{c.pl.bn, c.pl.ks, c.pl.pair, c.pl.fp8},
                       c.pl.splits > 1 ? GemmEpilogue::SplitK : GemmEpilogue::Bf16, st));
   return QWAM_OK;
@@ -738,14 +838,17 @@ qwam_status launch_call_gemm(const CallPlan& c, cudaStream_t st) {
 
 // The workspace arena of the handle's device, grown to hold M rows.
 qwam_status workspace_for(qwam_handle h, int M, Arena** a) {
-  return arena_get(h->dev, layout_for(M, h->K, h->r, h->fmt).total, a);
+  return arena_get(h->dev, layout_of(h, M).total, a);
 }
 
 // ---------------------------------------------------------------------------
 // Layer images: a prepared layer as one host byte string.  A 64-byte header
 // (little-endian), then the arrays the calls read, each padded to 16 bytes:
-// codes, block scales (NVFP4 only), L, V hi/lo and P^T hi/lo (r > 0 only),
-// 1/s, bias (when present).  What follows from these (the row-pipeline form of
+// codes, block scales (NVFP4 and INT4), L, V hi/lo and P^T hi/lo (r > 0 only),
+// 1/s, bias (when present).  INT4 levels are stored 4-bit (two's complement,
+// two per byte, the even element in the low nibble) and their scales as
+// fp16, as the checkpoint format keeps them; the device holds E4M3 bytes and
+// fp32.  What follows from these (the row-pipeline form of
 // 1/s, the H_b blocks and every tensor map) is rebuilt on load.  The checksum
 // is FNV-1a 64 (Fowler, Noll and Vo) over the whole image with its own field
 // taken as zero.
@@ -764,26 +867,70 @@ static_assert(sizeof(ImageHeader) == 64, "image header is 64 bytes");
 
 struct ImageSection {
   void* dev;
-  size_t bytes;
+  size_t bytes;  // in the image
+  int kind;      // 0 as on the device; 1 INT4 levels (packed 4-bit); 2 INT4 scales (fp16)
 };
+
+// E4M3 byte of an INT4 level (-8..7, all exact in E4M3) and back.
+uint8_t e4m3_of_level(int v) {
+  if (v == 0) return 0;
+  const int a = v < 0 ? -v : v;
+  int e = 0;
+  while ((a >> (e + 1)) != 0) ++e;
+  const int m = ((a << 3) >> e) & 7;  // three mantissa bits of a / 2^e
+  return static_cast<uint8_t>((v < 0 ? 0x80 : 0) | ((e + 7) << 3) | m);
+}
+bool level_of_e4m3(uint8_t b, int* v) {
+  for (int l = -8; l <= 7; ++l)
+    if (e4m3_of_level(l) == b || (l == 0 && b == 0x80)) {
+      *v = l;
+      return true;
+    }
+  return false;
+}
+// fp16 bits of an fp32 value that fp16 holds exactly (false otherwise), and back.
+bool half_bits_exact(float f, uint16_t* out) {
+  if (!(f >= 0.0f) || f > 65504.0f) return false;
+  if (f == 0.0f) {
+    *out = 0;
+    return true;
+  }
+  int ex = 0;
+  std::frexp(f, &ex);  // f = fr 2^ex, fr in [0.5, 1)
+  const int e = ex - 1;
+  const double q = e >= -14 ? std::ldexp(static_cast<double>(f), 10 - e) - 1024.0 : std::ldexp(static_cast<double>(f), 24);
+  if (q != std::floor(q) || q < 0 || q > 1023) return false;
+  *out = static_cast<uint16_t>(e >= -14 ? ((e + 15) << 10) | static_cast<int>(q) : static_cast<int>(q));
+  return true;
+}
+float float_of_half_bits(uint16_t hb) {
+  const int e = (hb >> 10) & 31, m = hb & 1023;
+  const float v = e == 0 ? std::ldexp(static_cast<float>(m), -24) : std::ldexp(static_cast<float>(1024 + m), e - 25);
+  return (hb & 0x8000) ? -v : v;
+}
 
 size_t pad16(size_t n) { return (n + 15) & ~static_cast<size_t>(15); }
 
 // The sections of a layer in image order; returns their count (at most 9).
 int image_sections(const qwam_layer* h, bool with_bias, ImageSection* out) {
   int n = 0;
-  out[n++] = {h->codes, layer_code_bytes(h)};
-  if (h->fmt == 0) out[n++] = {h->sf, h->sf_bytes};
+  if (h->fmt == 2) {
+    out[n++] = {h->codes, layer_code_bytes(h) / 2, 1};
+    out[n++] = {h->sf, h->sf_bytes / 2, 2};
+  } else {
+    out[n++] = {h->codes, layer_code_bytes(h), 0};
+    if (h->fmt == 0) out[n++] = {h->sf, h->sf_bytes, 0};
+  }
   if (h->r > 0) {
     const size_t vb = static_cast<size_t>(h->K) * h->r * 2;
-    out[n++] = {h->L, static_cast<size_t>(h->N) * h->r * 2};
-    out[n++] = {h->v_hi, vb};
-    out[n++] = {h->v_lo, vb};
-    out[n++] = {h->px_hi, vb};
-    out[n++] = {h->px_lo, vb};
+    out[n++] = {h->L, static_cast<size_t>(h->N) * h->r * 2, 0};
+    out[n++] = {h->v_hi, vb, 0};
+    out[n++] = {h->v_lo, vb, 0};
+    out[n++] = {h->px_hi, vb, 0};
+    out[n++] = {h->px_lo, vb, 0};
   }
-  out[n++] = {h->inv_s, static_cast<size_t>(h->K) * 4};
-  if (with_bias) out[n++] = {h->bias, static_cast<size_t>(h->N) * 2};
+  out[n++] = {h->inv_s, static_cast<size_t>(h->K) * 4, 0};
+  if (with_bias) out[n++] = {h->bias, static_cast<size_t>(h->N) * 2, 0};
   return n;
 }
 
@@ -869,7 +1016,7 @@ qwam_status linear_noalloc_impl(const void* x, int M, qwam_handle h, void* y, cu
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes at most %d rows, got M=%d", kStaticMaxRows, M);
   if (h->K > kStaticMaxK)
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc takes K <= %d, this layer has K=%d", kStaticMaxK, h->K);
-  const Layout lay = layout_for(M, h->K, h->r, h->fmt);
+  const Layout lay = layout_of(h, M);
   if (lay.total > kStaticBytes)
     return fail(QWAM_ERR_SHAPE, "qwam_linear_noalloc needs %zu bytes of scratch, the static scratch holds %zu",
                 lay.total, kStaticBytes);
@@ -905,6 +1052,40 @@ qwam_status qwam_prepare_weight_fp8(const void* W_bf16, int N, int K, const floa
   return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, hadamard_block, Wd_f32, false, 1, stream, out);
 }
 
+qwam_status qwam_prepare_weight_int4(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                     const void* bias_bf16, float* Wd_f32, void* stream, qwam_handle* out) {
+  return prepare_impl(W_bf16, N, K, s, V, r, bias_bf16, 1, Wd_f32, false, 2, stream, out);
+}
+
+qwam_status qwam_int4_gemm(const void* a_levels, const float* a_scales, const void* b_levels, const float* b_scales,
+                           int M, int N, int K, float* out_f32, void* stream) {
+  if (!a_levels || !a_scales || !b_levels || !b_scales || !out_f32) return fail(QWAM_ERR_INVALID_ARG, "NULL argument");
+  if (M < 4 || M % 4 || N < 16 || N % 16 || K < 128 || K % 128)
+    return fail(QWAM_ERR_SHAPE, "M a positive multiple of 4, N of 16 and K of 128 required (M=%d N=%d K=%d)", M, N, K);
+  if (!aligned16(a_levels) || !aligned16(a_scales) || !aligned16(b_levels) || !aligned16(b_scales) || !aligned16(out_f32))
+    return fail(QWAM_ERR_ALIGN, "device pointers must be 16-byte aligned");
+  int dev = 0;
+  QW_TRY(current_device(&dev));
+  Arena* ar = nullptr;
+  QW_TRY(arena_get(dev, kHeaderBytes, &ar));
+  GroupGemmMaps m{};
+  QW_TRY(make_codes_map(&m.a, a_levels, M, K, 128, 128));
+  QW_TRY(make_codes_map(&m.b, b_levels, N, K, 128, 128));
+  QW_TRY(make_map(&m.sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a_scales, M, K / 64, static_cast<uint64_t>(M) * 4, 128, 2,
+                  CU_TENSOR_MAP_SWIZZLE_NONE));
+  QW_TRY(make_map(&m.sb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, b_scales, N, K / 64, static_cast<uint64_t>(N) * 4, 128, 2,
+                  CU_TENSOR_MAP_SWIZZLE_NONE));
+  m.u = m.sa;  // no branch: unread
+  m.l = m.sb;
+  GroupGemmParams p{};
+  p.M = M; p.N = N; p.K = K;
+  p.splits = 1;
+  p.partial = out_f32;
+  p.err = arena_err(*ar);
+  QW_CUDA(launch_group_gemm(m, p, as_stream(stream)));
+  return QWAM_OK;
+}
+
 qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant) {
   if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
   if (fmt) *fmt = h->fmt;
@@ -931,11 +1112,39 @@ qwam_status qwam_save_image(qwam_handle h, void* host_buf, size_t buf_bytes, voi
   ImageSection sec[9];
   const int n = image_sections(h, with_bias, sec);
   size_t off = sizeof(ImageHeader);
+  std::vector<uint8_t> tmp[2];  // INT4 levels and scales as the device holds them
   for (int i = 0; i < n; ++i) {
-    QW_CUDA(cudaMemcpyAsync(img + off, sec[i].dev, sec[i].bytes, cudaMemcpyDeviceToHost, st));
+    if (sec[i].kind == 0) {
+      QW_CUDA(cudaMemcpyAsync(img + off, sec[i].dev, sec[i].bytes, cudaMemcpyDeviceToHost, st));
+    } else {
+      std::vector<uint8_t>& v = tmp[sec[i].kind - 1];
+      v.resize(2 * sec[i].bytes);
+      QW_CUDA(cudaMemcpyAsync(v.data(), sec[i].dev, v.size(), cudaMemcpyDeviceToHost, st));
+    }
     off += pad16(sec[i].bytes);
   }
   QW_CUDA(cudaStreamSynchronize(st));
+  off = sizeof(ImageHeader);
+  for (int i = 0; i < n; ++i) {
+    uint8_t* dst = img + off;
+    if (sec[i].kind == 1) {
+      const std::vector<uint8_t>& v = tmp[0];
+      for (size_t j = 0; j < sec[i].bytes; ++j) {
+        int lo = 0, hi = 0;
+        if (!level_of_e4m3(v[2 * j], &lo) || !level_of_e4m3(v[2 * j + 1], &hi))
+          return fail(QWAM_ERR_FORMAT, "the handle holds a code that is no INT4 level");
+        dst[j] = static_cast<uint8_t>((lo & 15) | ((hi & 15) << 4));
+      }
+    } else if (sec[i].kind == 2) {
+      const float* f = reinterpret_cast<const float*>(tmp[1].data());
+      for (size_t j = 0; j < sec[i].bytes / 2; ++j) {
+        uint16_t hb = 0;
+        if (!half_bits_exact(f[j], &hb)) return fail(QWAM_ERR_FORMAT, "the handle holds a scale that is no fp16 value");
+        std::memcpy(dst + 2 * j, &hb, 2);
+      }
+    }
+    off += pad16(sec[i].bytes);
+  }
   ImageHeader hd{};
   std::memcpy(hd.magic, kImageMagic, 8);
   hd.version = kImageVersion;
@@ -966,13 +1175,14 @@ qwam_status qwam_load_image(const void* host_buf, size_t buf_bytes, void* stream
                 kImageVersion, sizeof hd);
   if (check_layer_shape(hd.N, hd.K, hd.r, hd.b) != QWAM_OK)
     return fail(QWAM_ERR_FORMAT, "image shape N=%d K=%d r=%d b=%d is not a valid layer", hd.N, hd.K, hd.r, hd.b);
-  if ((hd.fmt != 0 && hd.fmt != 1) || (hd.variant != 0 && hd.variant != 1) || (hd.fmt == 1 && hd.variant != 0) ||
-      (hd.flags & ~1u) || !(std::isfinite(hd.g_w) && hd.g_w > 0.0f))
+  if (hd.fmt < 0 || hd.fmt > 2 || hd.variant < 0 || hd.variant > 2 || (hd.fmt == 1 && hd.variant != 0) ||
+      ((hd.fmt == 2) != (hd.variant == 2)) || (hd.fmt == 2 && hd.b != 1) || (hd.flags & ~1u) ||
+      !(std::isfinite(hd.g_w) && hd.g_w > 0.0f))
     return fail(QWAM_ERR_FORMAT, "image header fields are out of range (fmt %d, variant %d, flags 0x%x)", hd.fmt,
                 hd.variant, hd.flags);
   qwam_layer shape{};
   shape.N = hd.N; shape.K = hd.K; shape.r = hd.r; shape.fmt = hd.fmt;
-  shape.sf_bytes = hd.fmt == 1 ? 16 : round_up(static_cast<size_t>(hd.N), 256) * hd.K / 16;
+  shape.sf_bytes = layer_sf_bytes(hd.N, hd.K, hd.fmt);
   const bool with_bias = hd.flags & 1u;
   const size_t total = image_bytes(&shape, with_bias);
   if (hd.total_bytes != total || buf_bytes < total)
@@ -996,8 +1206,30 @@ qwam_status qwam_load_image(const void* host_buf, size_t buf_bytes, void* stream
   size_t off = sizeof(ImageHeader);
   cudaError_t e = cudaSuccess;
   if (hd.fmt == 1) e = cudaMemsetAsync(h->sf, 0, h->sf_bytes, st);
+  std::vector<uint8_t> tmp[2];  // INT4 levels and scales in the device's form
   for (int i = 0; i < n && e == cudaSuccess; ++i) {
-    e = cudaMemcpyAsync(sec[i].dev, img + off, sec[i].bytes, cudaMemcpyHostToDevice, st);
+    const uint8_t* src = img + off;
+    if (sec[i].kind == 0) {
+      e = cudaMemcpyAsync(sec[i].dev, src, sec[i].bytes, cudaMemcpyHostToDevice, st);
+    } else {
+      std::vector<uint8_t>& v = tmp[sec[i].kind - 1];
+      v.resize(2 * sec[i].bytes);
+      if (sec[i].kind == 1) {
+        for (size_t j = 0; j < sec[i].bytes; ++j) {
+          const int lo = src[j] & 15, hi = src[j] >> 4;
+          v[2 * j] = e4m3_of_level(lo >= 8 ? lo - 16 : lo);
+          v[2 * j + 1] = e4m3_of_level(hi >= 8 ? hi - 16 : hi);
+        }
+      } else {
+        float* f = reinterpret_cast<float*>(v.data());
+        for (size_t j = 0; j < sec[i].bytes / 2; ++j) {
+          uint16_t hb;
+          std::memcpy(&hb, src + 2 * j, 2);
+          f[j] = float_of_half_bits(hb);
+        }
+      }
+      e = cudaMemcpyAsync(sec[i].dev, v.data(), v.size(), cudaMemcpyHostToDevice, st);
+    }
     off += pad16(sec[i].bytes);
   }
   if (e == cudaSuccess) e = launch_chan_pm(h->inv_s, 1.0f / std::sqrt(static_cast<float>(hd.b)), hd.K, h->inv_s_pm, st);
@@ -1096,6 +1328,7 @@ qwam_status qwam_export_weight(qwam_handle h, void* codes, void* scales, void* L
                             cudaMemcpyDeviceToDevice, st));
   if (scales && h->fmt == 0)
     QW_CUDA(cudaMemcpyAsync(scales, h->sf, round_up(static_cast<size_t>(h->N), 128) * h->K / 16, cudaMemcpyDeviceToDevice, st));
+  if (scales && h->fmt == 2) QW_CUDA(cudaMemcpyAsync(scales, h->sf, h->sf_bytes, cudaMemcpyDeviceToDevice, st));
   if (L_bf16 && h->r > 0)
     QW_CUDA(cudaMemcpyAsync(L_bf16, h->L, static_cast<size_t>(h->N) * h->r * 2, cudaMemcpyDeviceToDevice, st));
   return QWAM_OK;
@@ -1110,7 +1343,7 @@ qwam_status qwam_debug_prologue(const void* x_bf16, int M, qwam_handle h, float*
   cudaStream_t st = as_stream(stream);
   Arena* a = nullptr;
   QW_TRY(workspace_for(h, M, &a));
-  const Layout lay = layout_for(M, h->K, h->r, h->fmt);
+  const Layout lay = layout_of(h, M);
   {
     std::lock_guard<std::mutex> lock(h->mu);
     CallPlan& c = h->call[0];
@@ -1124,12 +1357,16 @@ qwam_status qwam_debug_prologue(const void* x_bf16, int M, qwam_handle h, float*
   if (codes)
     QW_CUDA(cudaMemcpyAsync(codes, a->base + lay.codes, static_cast<size_t>(M) * code_bytes(h->K, h->fmt),
                             cudaMemcpyDeviceToDevice, st));
-  if (scales && h->fmt == 0)
+  if (scales && h->fmt != 1)  // NVFP4 tiles, or INT4 fp32 [K / 64][round_up(M, 128)]: the same bytes
     QW_CUDA(cudaMemcpyAsync(scales, a->base + lay.sf, round_up(static_cast<size_t>(M), 128) * h->K / 16,
                             cudaMemcpyDeviceToDevice, st));
   if (ubr_bf16 && h->r > 0)
     QW_CUDA(cudaMemcpyAsync(ubr_bf16, a->base + lay.ub, static_cast<size_t>(M) * h->r * 2, cudaMemcpyDeviceToDevice, st));
-  if (g_x) QW_CUDA(cudaMemcpyAsync(g_x, arena_gx(*a), 4, cudaMemcpyDeviceToDevice, st));
+  if (g_x) {
+    static const float kOne = 1.0f;  // INT4 has no per-tensor scale
+    if (h->fmt == 2) QW_CUDA(cudaMemcpyAsync(g_x, &kOne, 4, cudaMemcpyHostToDevice, st));
+    else QW_CUDA(cudaMemcpyAsync(g_x, arena_gx(*a), 4, cudaMemcpyDeviceToDevice, st));
+  }
   return QWAM_OK;
 }
 
@@ -1207,6 +1444,14 @@ qwam_status qwam_debug_fp4_gemm_withheld(const void* a_codes, const void* a_scal
 qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* splits, int* bn) {
   if (!h || h->magic != kMagic) return fail(QWAM_ERR_INVALID_ARG, "invalid qwam handle");
   if (M < 0) return fail(QWAM_ERR_SHAPE, "M=%d must be >= 0", M);
+  if (h->fmt == 2) {  // Local prologue, group GEMM (+ the split-K sum)
+    const int sp = group_splits(std::max(M, 1), h->N, h->K, sm_count(h->dev));
+    if (kernels) *kernels = M == 0 ? 0 : (sp > 1 ? 3 : 2);
+    if (fused) *fused = 0;
+    if (splits) *splits = sp;
+    if (bn) *bn = 128;
+    return QWAM_OK;
+  }
   const bool f = use_fused(M);
   const Plan pl = plan_gemm(std::max(M, 1), h->N, h->K, sm_count(h->dev), h->fmt);
   const int form = prologue_form(std::max(M, 1), h->r, h->K, sm_count(h->dev));

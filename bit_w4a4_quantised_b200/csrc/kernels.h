@@ -42,14 +42,22 @@ struct PrologueParams {
   float* u_out;           // optional fp32 [rows, r] (debug export of c)
   uint32_t* err;          // device error word for bounded waits
   int fmt;                // element format: 0 NVFP4 (codes [rows, K/2] + tiled
-                          // scales), 1 FP8 E4M3 (codes [rows, K], no block scales)
+                          // scales), 1 FP8 E4M3 (codes [rows, K], no block scales),
+                          // 2 INT4 group 64 (levels as E4M3 bytes [rows, K]; sf
+                          // holds fp32 scales [K / 64][sf_pitch])
+  int sf_pitch;           // INT4: row pitch of the scale array, in scales
 };
 
-enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2 };
+// Local: the SVDQuant arm's activation side (b = 1, INT4): x * chan quantised
+// group by group as it is read, no deflation and no tensor-wide amax, so every
+// row tile is independent; c = x P still summed across the row tile's cluster
+// for the branch operand bf16(c).
+enum class PrologueMode { Fused = 0, Stats = 1, Quantise = 2, Local = 3 };
 
-// Grid: parts x ceil(rows / 128) CTAs; Fused and Stats (r > 0) launch the
-// parts of a row tile as one cluster.  Fused requires rows <= 128; Stats
-// requires *amax_glob == 0.
+// Grid: parts x ceil(rows / 128) CTAs; Fused, Stats and Local (r > 0) launch
+// the parts of a row tile as one cluster.  Fused requires rows <= 128 (INT4,
+// whose scales are local: any rows); Stats requires *amax_glob == 0; Local
+// requires fmt == INT4.
 cudaError_t launch_prologue(const ProMaps& maps, const PrologueParams& p, int r, PrologueMode mode,
                             cudaStream_t st);
 
@@ -137,6 +145,34 @@ GemmShape gemm_shape(int M, int N, bool fp8 = false);
 // CTAs per tile.
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, GemmShape shape, GemmEpilogue epi,
                         cudaStream_t st);
+
+// INT4 group-64 GEMM of the SVDQuant arm:
+//   y = sum_g sa[:, g] sb[:, g]^T * P_g + u' L^T + bias,  P_g the exact group sums
+// on E4M3-coded levels.  128 x 128 tiles, K in stages of 128 (two groups).
+struct GroupGemmParams {
+  int M, N, K;             // K % 128 == 0
+  int splits;              // K splits (grid z); the stages are shared out evenly
+  int branch_k;            // r of the bf16 branch (0: none); split 0 adds it
+  const void* bias;        // bf16 [N] or nullptr (bf16 output only)
+  void* y;                 // bf16 [M, N]; nullptr: fp32 partial tiles instead
+  float* partial;          // fp32 [splits][M][N] when y == nullptr
+  uint32_t* err;
+  uint64_t wait_ns;        // limit of every bounded wait (0: the default)
+};
+
+struct GroupGemmMaps {
+  CUtensorMap a;    // A levels [M, K] u8 (E4M3 bytes) as a 3-D map (bytes, rows, 1), box 128 B x 128 rows x 1, 128B swizzle
+  CUtensorMap b;    // B levels [N, K] u8, same form
+  CUtensorMap sa;   // A scales fp32 [K / 64][pitch >= M], box 128 rows x 2 groups
+  CUtensorMap sb;   // B scales fp32 [K / 64][N], same box
+  CUtensorMap u;    // branch A [M, r] bf16, box r x 128 rows (unread when r == 0)
+  CUtensorMap l;    // branch B [N, r] bf16, box r x 128 rows
+};
+
+cudaError_t launch_group_gemm(const GroupGemmMaps& maps, const GroupGemmParams& p, cudaStream_t st);
+// y = bf16(sum over splits of partial + bias), the splits summed in order.
+cudaError_t launch_splitk_finalize(const float* partial, int splits, int M, int N, const void* bias, void* y,
+                                   cudaStream_t st);
 
 // The warp-specialised kernels move registers between warpgroups with
 // setmaxnreg, a split that adds up to the registers the launch gives each

@@ -60,7 +60,7 @@ template <int R, int MODE, int W>
 struct PCfg {
   // Stats / Quantise: the rotation runs on the tensor core, Z = (A_hi + A_lo) H -
   // c V^T into TMEM, with A = T * chan * hscale split into bf16 hi/lo by the rows
-  static constexpr bool kTC = MODE != 0;
+  static constexpr bool kTC = MODE == 1 || MODE == 2;
   static constexpr bool kMMA = R > 0 || kTC;
   static constexpr bool kProj = R > 0 && MODE != 2;   // this launch computes c
   static constexpr bool kNeedA = kProj;               // cluster exchange of partial c
@@ -241,7 +241,10 @@ __device__ __forceinline__ void split_cols(uint8_t* xs, uint8_t* lo_tile, const 
 template <int W>
 __device__ __forceinline__ void quantise_cols(const PrologueParams& p, const float (&v)[W], int row, int col,
                                               float g, float y_g) {
-  if (p.fmt == FMT_FP8)
+  if (p.fmt == FMT_INT4) {
+    if constexpr (W == 64)  // the host never runs INT4 in the 32-column layout
+      quantise_store_int4<W>(v, row, col, p.K, p.sf_pitch, p.codes, reinterpret_cast<float*>(p.sf), p.z_out);
+  } else if (p.fmt == FMT_FP8)
     quantise_store_fp8<W>(v, row, col, p.K, y_g, p.codes, p.z_out);
   else
     quantise_store<W>(v, row, col, p.K, g, y_g, p.codes, p.sf, p.z_out);
@@ -280,14 +283,27 @@ __device__ __forceinline__ void write_branch(const PrologueParams& p, const floa
 //            order, so its first loads find the chunks the projection read last
 //            still in L2 (a row slab wider than L2 holds is otherwise read twice
 //            from DRAM)
+//   need_v : the loads of the Z sweeps carry V (not in Local: no deflation)
 struct Sched {
-  bool merged, rev;
+  bool merged, rev, need_v;
   int nproj, zsweeps, total;
 };
 
 template <int R, int MODE>
 __device__ __forceinline__ Sched schedule(int nch) {
   Sched s;
+  if constexpr (MODE == 3) {
+    // Local: one sweep; each load (T, P, chan) feeds the projection MMA and the
+    // quantiser at once, since nothing the rows compute waits for c
+    s.merged = R > 0;
+    s.rev = false;
+    s.need_v = false;
+    s.nproj = 0;
+    s.zsweeps = 1;
+    s.total = nch;
+    return s;
+  }
+  s.need_v = true;
   const bool proj = R > 0 && MODE != 2;
   s.merged = proj && nch == 1 && MODE == 0;  // the tensor-core rotation keeps P and V in one area
   s.nproj = (proj && !s.merged) ? nch : 0;
@@ -301,7 +317,7 @@ template <int R>
 __device__ __forceinline__ uint32_t load_kind(const Sched& s, int i) {
   if (i < s.nproj) return LD_X | LD_P;
   uint32_t k = LD_X | LD_CH;
-  if (R > 0) k |= LD_V;
+  if (R > 0 && s.need_v) k |= LD_V;
   if (s.merged) k |= LD_P;
   return k;
 }
@@ -479,7 +495,9 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
       }
     };
     for (int i = 0; i < sch.total; ++i) {
-      if (i == zs1 + 2) pass_a();
+      // (Local: the rows free every slot without a barrier, so the producers
+      // issue every load first)
+      if (MODE != 3 && i == zs1 + 2) pass_a();
       if (sch.zsweeps == 2 && i == zs2 + 2) pass_b();
       issue(i);
     }
@@ -517,7 +535,7 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
                 mma_bf16(u_tmem, a, b, idesc_bf16(128, 2 * R), acc);
                 acc = 1u;
               }
-            if (!sch.merged) {
+            if (!sch.merged || MODE == 3) {  // Local: the projection is the slot's only MMA
               tc_commit(&empty[slot]);
               ++i;
             }
@@ -580,7 +598,7 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
           for (int c = 0; ok && c < nch; ++c) ok = zmma(c);
         }
         __syncwarp();
-      } else {
+      } else if constexpr (MODE != 3) {
         // deflation of one chunk: D2[128 x 128] = c (hi/lo) . V_chunk^T (hi/lo)
         const uint32_t sbo_u = 8u * 2u * R;
         const uint32_t swz_u = umma_swizzle_code(2 * R);
@@ -704,10 +722,11 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
       if (lane == 0) mbar_arrive(&empty[i & 1]);
     }
 
-    if constexpr (C::kProj) {
-      // Partial c of this CTA's K range (T P_hi + T P_lo, from TMEM), summed
-      // over the cluster: reduce-scatter by row slice, then all-gather, both by
-      // remote stores (remote loads would cost a round trip each).
+    // Partial c of this CTA's K range (T P_hi + T P_lo, from TMEM), summed
+    // over the cluster: reduce-scatter by row slice, then all-gather, both by
+    // remote stores (remote loads would cost a round trip each).
+    auto gather_c = [&]() {
+      if constexpr (C::kProj) {
       mbar_wait(u_full, 0, p.err, DEVERR_EPILOGUE_WAIT);
       __syncwarp();
       tc_fence_after();
@@ -764,6 +783,28 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
           u[k] = v.x; u[k + 1] = v.y; u[k + 2] = v.z; u[k + 3] = v.w;
         }
       }
+      }
+    };
+    if constexpr (MODE == 3) {
+      // Local: every chunk quantised as it lands (x * chan, no deflation, the
+      // group scales local), then the cluster sum of c for the branch bf16(c)
+      float z[W];
+      for (int c = 0; c < nch; ++c, ++i) {
+        const int slot = i & 1;
+        mbar_wait(&full[slot], (i >> 1) & 1, p.err, DEVERR_EPILOGUE_WAIT);
+        const uint8_t* s = smem + slot * C::SLOT;
+        rotate_cols<W>(s, reinterpret_cast<const float*>(s + C::OFF_CH), zrow, s0, p.b, z);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (zvalid) quantise_cols<W>(p, z, zrow_g, col0 + c * kChunk + s0 * W, 1.0f, 1.0f);
+      }
+      if constexpr (C::kProj) {
+        gather_c();
+        if (part == 0 && uvalid) write_branch<C::UC>(p, u, R, urow_g, uc0, 1.0f);
+      }
+    } else {
+    if constexpr (C::kProj) {
+      gather_c();
       if (MODE == 1 && part == 0 && uvalid) {
         float4* o = reinterpret_cast<float4*>(p.u_glob + static_cast<size_t>(urow_g) * R + uc0);
 #pragma unroll
@@ -919,6 +960,7 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
     if constexpr (MODE == 2) {
       if (part == 0 && blockIdx.y == 0 && rw == 0 && lane == 0) *p.g_out = g;
     }
+    }  // MODE != 3
   }
   tc_fence_before();
   __syncthreads();
@@ -962,10 +1004,16 @@ template <int R>
 cudaError_t launch_r(const ProMaps& maps, const PrologueParams& p, PrologueMode mode, cudaStream_t st) {
   switch (mode) {
     case PrologueMode::Fused:
-      if (p.rows > kRows) return cudaErrorInvalidValue;
-      return p.rows <= 32 ? launch_one<R, 0, 32>(maps, p, st) : launch_one<R, 0, 64>(maps, p, st);
+      // one row tile, since the cluster's amax is the tensor's; INT4 scales are
+      // local, so its row tiles may run side by side
+      if (p.rows > kRows && p.fmt != FMT_INT4) return cudaErrorInvalidValue;
+      // the INT4 quantiser takes one 64-column group per thread
+      return p.rows <= 32 && p.fmt != FMT_INT4 ? launch_one<R, 0, 32>(maps, p, st) : launch_one<R, 0, 64>(maps, p, st);
     case PrologueMode::Stats: return launch_one<R, 1, 64>(maps, p, st);
     case PrologueMode::Quantise: return launch_one<R, 2, 64>(maps, p, st);
+    case PrologueMode::Local:
+      if (p.fmt != FMT_INT4 || p.b != 1) return cudaErrorInvalidValue;
+      return launch_one<R, 3, 64>(maps, p, st);
   }
   return cudaErrorInvalidValue;
 }

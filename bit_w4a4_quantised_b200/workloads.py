@@ -150,6 +150,22 @@ def c3_video_attn(r: int = 32, seed: int = 0, layer: int = 0) -> LayerCase:
                       n_outliers=outlier_count(3072, 0.005), outlier_scale=30.0, v_rank=32)
 
 
+def c3_video_attn_int4(seed: int = 0, layer: int = 0) -> LayerCase:
+    """The c3 layer (same x, W, bias and V as c3_video_attn(32)) for the
+    SVDQuant INT4 arm: no rotation (block 1), rank 32."""
+    return draw_layer("c3_video_attn_4096x3072x3072_r32_b1", 4096, 3072, 3072, 32, 1,
+                      seed=seed, config_id=3, layer=layer,
+                      n_outliers=outlier_count(3072, 0.005), outlier_scale=30.0, v_rank=32)
+
+
+def c2_action_attn_int4(seed: int = 0, layer: int = 0) -> LayerCase:
+    """The c2 layer (same draws as c2_action_attn) for the SVDQuant INT4 arm:
+    block 1, rank 32."""
+    return draw_layer("c2_action_attn_32x1024x1024_r32_b1", 32, 1024, 1024, 32, 1,
+                      seed=seed, config_id=2, layer=layer,
+                      n_outliers=outlier_count(1024, 0.01), outlier_scale=20.0)
+
+
 def c4_video_ffn_up(seed: int = 0) -> LayerCase:
     """Video-expert FFN up: 4096 tokens, 3072 -> 14336, rank 32, block 128."""
     return draw_layer("c4_video_ffn_up_4096x3072x14336_r32_b128", 4096, 3072, 14336, 32, 128,

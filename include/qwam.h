@@ -114,8 +114,40 @@ qwam_status qwam_prepare_weight_fp8(const void* W_bf16, int N, int K, const floa
                                     const void* bias_bf16, int hadamard_block, float* Wd_f32, void* stream,
                                     qwam_handle* out);
 
+/* ---------------------------------------------------------------------------
+ * The SVDQuant INT4 W4A4 arm ("FastWAM UR3 3-task -- 4-bit quantisations",
+ * top table, SVDQuant column: INT4 at group 64 on weights and activations,
+ * a low-rank branch, products on integer tensor cores, exact for 4-bit
+ * codes; section "Verification -- INT4 SVDQuant").  In this library's terms:
+ * smoothing x^ = x / s and W^ = W diag(s) with no rotation (b = 1); the
+ * branch from the rank-r basis V, L = W^ V (with V the top right singular
+ * vectors of W^, L V^T is its rank-r truncated SVD); the residual
+ * R = W^ - L V^T and the activation x^ itself (not deflated) quantised
+ * INT4 per group of 64 along K:
+ *
+ *   y = deq(Q(x^)) deq(Q(R))^T + (x^ V) L^T + bias
+ *
+ * Q: a = max |v| of the group, s = fp16_rn(a / 7) (saturated to 65504),
+ * level = clamp(rint(v * (1 / s)), -8, 7) (fp32, half to even; 0 when
+ * s == 0).  The levels reach the tensor core as E4M3 bytes (kind::f8f6f4
+ * gives the exact integer group sums); each group's sums are scaled by
+ * s_x s_w and added in fp32 in group order.
+ *
+ * Arguments as qwam_prepare_weight without hadamard_block (b = 1); Wd_f32
+ * (device fp32 [N, K] or NULL) receives the exact fp32 R the weight
+ * quantiser consumed.  The handle's weight export (qwam_export_weight): codes
+ * [N, K] E4M3 bytes of the levels; scales fp32 [K / 64][N] (N * K / 16 bytes).
+ * The activation export (qwam_debug_prologue): z = the fp32 x^ quantised,
+ * codes [M, K] E4M3 bytes, scales fp32 [K / 64][round_up(M, 128)], u' =
+ * bf16(u) (no scale to divide by), g_x = 1.  Every per-call entry point takes
+ * the handle; qwam_linear_noalloc within its scratch limit.
+ * ------------------------------------------------------------------------- */
+qwam_status qwam_prepare_weight_int4(const void* W_bf16, int N, int K, const float* s, const float* V, int r,
+                                     const void* bias_bf16, float* Wd_f32, void* stream, qwam_handle* out);
+
 /* Host outputs (each may be NULL): the element format of the handle (0 NVFP4,
- * 1 FP8 E4M3) and its weight arm (0 deflated, 1 shared-weight). */
+ * 1 FP8 E4M3, 2 INT4 group 64) and its weight arm (0 deflated, 1
+ * shared-weight, 2 SVDQuant). */
 qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant);
 
 /* ---------------------------------------------------------------------------
@@ -129,8 +161,10 @@ qwam_status qwam_handle_format(qwam_handle h, int* fmt, int* variant);
  * uint32 version = 1; uint32 header_bytes = 64; int32 N, K, r, b, fmt,
  * variant; uint32 flags (bit 0: bias present); float g_w; uint64
  * total_bytes; uint64 checksum}, then these arrays, each zero-padded to a
- * multiple of 16 bytes: codes (N * K/2 bytes; FP8: N * K), block scales
- * (NVFP4 only: round_up(N,256) * K/16 bytes, tiled as on the device), and
+ * multiple of 16 bytes: codes (N * K/2 bytes; FP8: N * K; INT4: the levels
+ * as 4-bit two's complement, two per byte, the even element in the low
+ * nibble), scales (NVFP4: round_up(N,256) * K/16 bytes, tiled as on the
+ * device; INT4: fp16 [K/64][N]; none for FP8), and
  * when r > 0: L bf16 [N, r], V hi and lo bf16 [K, r] each, P^T hi and lo
  * bf16 [r, K] each; then 1/s fp32 [K]; then bias bf16 [N] when flag bit 0
  * is set.  checksum = FNV-1a 64 (offset basis 0xcbf29ce484222325, prime
@@ -261,6 +295,16 @@ qwam_status qwam_debug_fp4_gemm_withheld(const void* a_codes, const void* a_scal
  * fused = 1 when the prologue is the single-launch cluster form for up to 128
  * rows, splits = K splits of the GEMM, bn = GEMM tile width. */
 qwam_status qwam_plan_info(int M, qwam_handle h, int* kernels, int* fused, int* splits, int* bn);
+
+/* The bare INT4 group GEMM of the SVDQuant arm, for tests: out_f32 [M, N] =
+ * sum over the K / 64 groups g of P_g (sa[g][m] sb[g][n]), with P_g the exact
+ * group sums of the levels, accumulated in fp32 in group order (no branch, no
+ * bias).  a_levels [M, K] and b_levels [N, K]: E4M3 bytes of INT4 levels;
+ * a_scales fp32 [K / 64][M], b_scales fp32 [K / 64][N].  M % 4 == 0,
+ * N % 16 == 0, K % 128 == 0 (QWAM_ERR_SHAPE otherwise); 16-byte aligned device
+ * buffers.  Expired waits are reported by qwam_device_error. */
+qwam_status qwam_int4_gemm(const void* a_levels, const float* a_scales, const void* b_levels, const float* b_scales,
+                           int M, int N, int K, float* out_f32, void* stream);
 
 /* Synchronise the current device, then return (and clear) the device error
  * word set by bounded waits: *code == 0 means none expired.  Returns

@@ -2,7 +2,8 @@
 with qwam_load_image computes exactly what the saved handle computes.
 
 Checks, through the C-ABI, for the deflated arm (r = 32 with bias, r = 0
-without), the shared-weight arm and the FP8 arm:
+without), the shared-weight arm, the FP8 arm and the SVDQuant INT4 arm (its
+levels stored 4-bit and its scales fp16 in the image):
 1. the image parsed by the documented layout holds the handle's exported
    codes, scales and L byte for byte, and g_w in its header;
 2. the loaded handle reports the same shape, format and g_w, exports the same
@@ -21,7 +22,12 @@ import pytest
 
 from bit_w4a4_quantised_b200 import workloads
 from gpu_util import codes_of, prepare
-from oracle import asp
+from oracle import asp, fp8
+
+
+def levels_of(dev_bytes):
+    """E4M3 bytes of INT4 levels -> int8 levels."""
+    return fp8.decode(np.asarray(dev_bytes)).astype(np.int8)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,6 +36,7 @@ CASES = {
     "deflated_r0": (lambda: workloads.custom(200, 512, 256, 0, 16, seed=102, n_outliers=5), "deflated", "nvfp4"),
     "shared_r16": (lambda: workloads.custom(260, 768, 384, 16, 64, seed=103, n_outliers=8), "shared", "nvfp4"),
     "fp8_r32": (lambda: workloads.custom(300, 1024, 512, 32, 128, seed=104, n_outliers=10), "deflated", "fp8"),
+    "int4_r32": (lambda: workloads.custom(300, 1024, 512, 32, 1, seed=106, n_outliers=10), "svdquant", "int4"),
 }
 
 
@@ -50,6 +57,8 @@ def parse_image(img: bytes):
     take("codes", N * (K if fmt == 1 else K // 2))
     if fmt == 0:
         take("scales", (N + 255) // 256 * 256 * K // 16)
+    if fmt == 2:
+        take("scales", K // 64 * N * 2)
     if r:
         take("L", N * r * 2)
         for name in ("v_hi", "v_lo", "px_hi", "px_lo"):
@@ -77,10 +86,21 @@ def test_image_round_trip(name):
     # 1. the documented layout
     p = parse_image(img)
     assert (p["N"], p["K"], p["r"], p["b"]) == (case.N, case.K, case.r, case.b)
-    assert p["fmt"] == (1 if fmt == "fp8" else 0) and p["variant"] == (1 if variant == "shared" else 0)
+    assert p["fmt"] == {"nvfp4": 0, "fp8": 1, "int4": 2}[fmt]
+    assert p["variant"] == {"deflated": 0, "shared": 1, "svdquant": 2}[variant]
     assert np.float32(p["g_w"]) == np.float32(h.g_w)
     w = qw.export_weight(h)
-    assert np.array_equal(p["codes"], w["codes"].cpu().numpy().reshape(-1))
+    if fmt == "int4":
+        # 4-bit two's complement, even element in the low nibble; fp16 scales
+        lo = (p["codes"] & 15).astype(np.int8)
+        hi = (p["codes"] >> 4).astype(np.int8)
+        lv = np.stack([np.where(lo >= 8, lo - 16, lo), np.where(hi >= 8, hi - 16, hi)], axis=1).reshape(case.N, case.K)
+        assert np.array_equal(lv, levels_of(w["codes"].cpu().numpy()))
+        sc = np.frombuffer(p["scales"].tobytes(), np.float16).astype(np.float32)
+        ws = w["scales"].cpu().view(torch.float32).numpy()[: sc.size]
+        assert np.array_equal(sc, ws)
+    else:
+        assert np.array_equal(p["codes"], w["codes"].cpu().numpy().reshape(-1))
     if fmt == "nvfp4":  # the image keeps the device's 256-row padding of the tiles
         ws = w["scales"].cpu().numpy().reshape(-1)
         assert np.array_equal(p["scales"][:ws.size], ws)
@@ -100,6 +120,9 @@ def test_image_round_trip(name):
     keys = ["codes", "L"] + (["scales"] if fmt == "nvfp4" else [])
     for k in keys:
         assert torch.equal(w[k], w2[k]), k
+    if fmt == "int4":  # the first N K / 16 scale bytes are the weight scales
+        nb = case.N * case.K // 16
+        assert torch.equal(w["scales"][:nb], w2["scales"][:nb])
     for rows in (min(37, case.M), case.M):
         xr = x[:rows].contiguous()
         y1, y2 = qw.linear(xr, h), qw.linear(xr, h2)
@@ -121,6 +144,8 @@ def test_image_round_trip(name):
         ref = asp.prepare_weight(case.W, case.s, case.V, case.b, fmt=fmt)
     if fmt == "fp8":
         got = p["codes"].reshape(case.N, case.K)
+    elif fmt == "int4":
+        got = lv
     else:
         got = codes_of(torch.from_numpy(p["codes"].reshape(case.N, case.K // 2).copy()))
     assert np.mean(got == ref["codes"]) >= 0.999

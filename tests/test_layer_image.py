@@ -25,9 +25,11 @@ def pad16(n):
 
 
 def image_len(N, K, r, fmt, bias):
-    n = 64 + pad16(N * (K if fmt == 1 else K // 2))
+    n = 64 + pad16(N * (K if fmt == 1 else K // 2))   # INT4: 4-bit levels, two per byte
     if fmt == 0:
         n += pad16((N + 255) // 256 * 256 * K // 16)
+    if fmt == 2:
+        n += pad16(K // 64 * N * 2)                   # fp16 group scales
     if r:
         n += pad16(N * r * 2) + 4 * pad16(K * r * 2)
     n += pad16(K * 4)
@@ -75,7 +77,7 @@ def test_header_is_64_bytes():
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(r=32, b=128, K=256, N=48, bias=True), dict(fmt=1, r=16, K=384, b=64),
-                                dict(variant=1, r=16, N=64)])
+                                dict(variant=1, r=16, N=64), dict(fmt=2, variant=2, r=32, K=256, N=32, bias=True)])
 def test_valid_image_passes_every_host_check(lib, kw):
     st, msg, h = load(lib, make_image(**kw))
     # no GPU here: the first device call fails, after the format checks
@@ -105,6 +107,9 @@ def test_any_flipped_byte_is_refused(lib, offset):
     (dict(b=3), "shape"),
     (dict(fmt=2), "out of range"),
     (dict(fmt=1, variant=1), "out of range"),
+    (dict(fmt=2, variant=0), "out of range"),
+    (dict(fmt=0, variant=2), "out of range"),
+    (dict(fmt=2, variant=2, b=16), "out of range"),
     (dict(g_w=0.0), "out of range"),
     (dict(g_w=float("nan")), "out of range"),
     (dict(total=3000), "bytes"),
