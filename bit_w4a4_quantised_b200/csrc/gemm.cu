@@ -54,7 +54,10 @@ constexpr int kScaleSlots = 4;  // TMEM scale ring, one stage per slot
 
 // F8: the FP8 W8A8 arm (E4M3 operands, kind::f8f6f4, one byte per element, no
 // block scales); otherwise NVFP4 (packed E2M1, E4M3 scale per 16 in TMEM).
-template <int BN, int KS, bool PAIR = false, bool F8 = false>
+// NB: no low-rank branch (r = 0); CTA pairs use the branch tiles' room for a
+// fifth operand stage (the stage ring is bound by its round trip, not by the
+// tensor core: more bytes in flight is more throughput).
+template <int BN, int KS, bool PAIR = false, bool F8 = false, bool NB = false>
 struct Cfg {
   static constexpr int TM = PAIR ? 2 * kBM : kBM;          // rows of an output tile
   static constexpr int HB = PAIR ? BN / 2 : BN;             // B (and L) rows held by one CTA
@@ -62,7 +65,7 @@ struct Cfg {
   static constexpr int KM = F8 ? KS / 32 : KS / 64;         // MMAs per stage (K 32 for FP8, 64 for FP4)
   static constexpr int K64 = KS / 64;                       // K64 steps of a stage (FP4 scale blocks)
   static constexpr uint32_t SWZ = ROWB == 128 ? 2u : 4u;    // UMMA layout: 128B / 64B swizzle
-  static constexpr int STAGES = PAIR ? 4 : (ROWB == 128 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
+  static constexpr int STAGES = PAIR ? (NB ? 5 : 4) : (ROWB == 128 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
   static constexpr int NSFB = F8 ? 0 : BN / 128;            // 128-row scale blocks of B
   static constexpr int SF_BLK = F8 ? 0 : K64 * 512;         // one 128-row scale block of a stage
   static constexpr int NBOX = F8 ? 2 : 4;                   // boxes per stage: A, B (, A scales, B scales)
@@ -78,8 +81,8 @@ struct Cfg {
   static constexpr int B_BYTES = HB * ROWB;
   static constexpr int SF_BYTES = F8 ? 0 : (1 + NSFB) * SF_BLK;
   static constexpr int STAGE_TX = A_BYTES + B_BYTES + SF_BYTES;
-  static constexpr int U_BYTES = kBM * 64;
-  static constexpr int L_BYTES = HB * 64;
+  static constexpr int U_BYTES = NB ? 0 : kBM * 64;
+  static constexpr int L_BYTES = NB ? 0 : HB * 64;
   static constexpr int SCOLS = PAIR ? 32 : 64;              // columns of one y store box
   static constexpr int STG_BYTES = 32 * SCOLS * 2;          // per epilogue warp: 32 rows x SCOLS bf16
   static constexpr int BIAS_BYTES = BN;                     // per epilogue warp: BN / 2 bf16
@@ -123,13 +126,13 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n,
   return {(rest % tiles_m) * tm, (rest / tiles_m % tiles_n) * bn, sp};
 }
 
-template <int BN, int KS, int EPI, bool PAIR, bool F8>
-__global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
+template <int BN, int KS, int EPI, bool PAIR, bool F8, bool NB>
+__global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8, NB>::THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmSA,
                     const __grid_constant__ CUtensorMap tmSB, const GemmParams p) {
-  using C = Cfg<BN, KS, PAIR, F8>;
+  using C = Cfg<BN, KS, PAIR, F8, NB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES] operands and scales landed
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
       tma_prefetch_desc(&tmB);
       tma_prefetch_desc(&tmSA);
       tma_prefetch_desc(&tmSB);
-      if (p.has_branch) {
+      if (!NB && p.has_branch) {
         tma_prefetch_desc(&tmU);
         tma_prefetch_desc(&tmL);
       }
@@ -280,7 +283,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
     for (int t = unit; ok && t < n_tiles; t += n_units) {
       const TileCoord tc = coord(t);
       const Range rg = range_of(tc.split);
-      if (p.has_branch && tc.split == 0 && warp == C::NPROD - 1) {
+      if (!NB && p.has_branch && tc.split == 0 && warp == C::NPROD - 1) {
         // branch operands of this tile, once the previous tile's branch MMAs are done
         int bok = 1;
         if (lane == 0) {
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
         if (!mbar_wait(acc_empty, (tl & 1) ^ 1u, p.err, DEVERR_MMA_WAIT, wlim)) break;
         tc_fence_after();
         uint32_t accum = 0;
-        if (p.has_branch && tc.split == 0) {
+        if (!NB && p.has_branch && tc.split == 0) {
           if (!mbar_wait(branch_full, nbranch & 1, p.err, DEVERR_BRANCH_WAIT, wlim)) break;
           tc_fence_after();
           for (int kk = 0; kk < p.branch_k / 16; ++kk) {
@@ -520,14 +523,21 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
                             fma_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]), gs, bw.w));
         };
         auto half_sync = [&]() { named_bar(1 + half, 128); };
+        // two 32-column loads in flight per wait (the round trip, not the
+        // bytes, sets the drain time; four serial rounds held the accumulator
+        // ~1.4 us per tile)
+        static_assert((HC / 32) % 2 == 0, "column pairs of 32");
         uint4 v[HC / 8];
 #pragma unroll
-        for (int qq = 0; qq < HC / 32; ++qq) {
-          uint32_t r[32];
+        for (int qq = 0; qq < HC / 32; qq += 2) {
+          uint32_t r[32], r1[32];
           tmem_ld_32x32b_x32(taddr + qq * 32, r);
+          tmem_ld_32x32b_x32(taddr + (qq + 1) * 32, r1);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 4; ++j) v[4 * qq + j] = convert(r, qq, j);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[4 * (qq + 1) + j] = convert(r1, qq + 1, j);
         }
         tc_fence_before();
         __syncwarp();
@@ -650,10 +660,11 @@ __global__ void __launch_bounds__(Cfg<BN, KS, PAIR, F8>::THREADS, 1)
   }
 }
 
-template <int BN, int KS, int EPI, bool PAIR, bool F8>
+template <int BN, int KS, int EPI, bool PAIR, bool F8, bool NB = false>
 cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
-  using C = Cfg<BN, KS, PAIR, F8>;
-  auto kern = fp4_gemm_kernel<BN, KS, EPI, PAIR, F8>;
+  using C = Cfg<BN, KS, PAIR, F8, NB>;
+  auto kern = fp4_gemm_kernel<BN, KS, EPI, PAIR, F8, NB>;
+  if (NB && p.has_branch) return cudaErrorInvalidValue;
   static const cudaError_t smem_attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (smem_attr != cudaSuccess) return smem_attr;
@@ -710,12 +721,12 @@ cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
 }
 
 // registers per thread at launch: the split's total over the 512 threads
-template <int BN, int KS, int EPI, bool PAIR, bool F8>
+template <int BN, int KS, int EPI, bool PAIR, bool F8, bool NB = false>
 bool split_ok(char* msg, size_t n) {
-  using C = Cfg<BN, KS, PAIR, F8>;
+  using C = Cfg<BN, KS, PAIR, F8, NB>;
   constexpr int want = (256 * C::REG_OTHER + 256 * C::REG_EPI) / C::THREADS;
   cudaFuncAttributes a{};
-  const cudaError_t e = cudaFuncGetAttributes(&a, fp4_gemm_kernel<BN, KS, EPI, PAIR, F8>);
+  const cudaError_t e = cudaFuncGetAttributes(&a, fp4_gemm_kernel<BN, KS, EPI, PAIR, F8, NB>);
   if (e != cudaSuccess) {
     snprintf(msg, n, "cudaFuncGetAttributes(fp4_gemm_kernel<%d,%d,%d,%d,%d>) failed: %s", BN, KS, EPI, int(PAIR),
              int(F8), cudaGetErrorString(e));
@@ -734,8 +745,14 @@ bool split_ok(char* msg, size_t n) {
 template <int BN, int KS, bool PAIR, bool F8>
 cudaError_t launch_bn(const GemmMaps& m, const GemmParams& p, GemmEpilogue epi, cudaStream_t st) {
   switch (epi) {
-    case GemmEpilogue::Bf16: return launch_t<BN, KS, 0, PAIR, F8>(m, p, st);
-    case GemmEpilogue::RawF32: return launch_t<BN, KS, 1, PAIR, F8>(m, p, st);
+    case GemmEpilogue::Bf16:
+      if constexpr (PAIR)
+        if (!p.has_branch) return launch_t<BN, KS, 0, PAIR, F8, true>(m, p, st);
+      return launch_t<BN, KS, 0, PAIR, F8>(m, p, st);
+    case GemmEpilogue::RawF32:
+      if constexpr (PAIR)
+        if (!p.has_branch) return launch_t<BN, KS, 1, PAIR, F8, true>(m, p, st);
+      return launch_t<BN, KS, 1, PAIR, F8>(m, p, st);
     case GemmEpilogue::SplitK:
       if constexpr (PAIR) return cudaErrorInvalidValue;
       else return launch_t<BN, KS, 2, false, F8>(m, p, st);
@@ -748,6 +765,7 @@ cudaError_t launch_bn(const GemmMaps& m, const GemmParams& p, GemmEpilogue epi, 
 template <bool F8, int KB, int KS>  // KB: K per stage of the large-M tiles, KS of the small-M ones
 bool format_split_ok(char* msg, size_t n) {
   return split_ok<256, KB, 0, true, F8>(msg, n) && split_ok<256, KB, 1, true, F8>(msg, n) &&
+         split_ok<256, KB, 0, true, F8, true>(msg, n) && split_ok<256, KB, 1, true, F8, true>(msg, n) &&
          split_ok<256, KB, 0, false, F8>(msg, n) && split_ok<256, KB, 1, false, F8>(msg, n) &&
          split_ok<256, KB, 2, false, F8>(msg, n) && split_ok<128, KB, 0, false, F8>(msg, n) &&
          split_ok<128, KB, 1, false, F8>(msg, n) && split_ok<128, KB, 2, false, F8>(msg, n) &&

@@ -11,22 +11,28 @@
 // most 64 * 64 in magnitude) are exact in its fp32 accumulator, so P_g is the
 // integer an INT8 tensor core would give, read out of TMEM as fp32 with no
 // conversion.  The scale sa sb changes from group to group, so it cannot stay
-// in the accumulator: each group's P_g goes to one of two TMEM buffers in turn
-// and eight rescale warps fold it into an fp32 accumulator in registers,
+// in the accumulator: each group's P_g goes to one of four TMEM buffers in turn
+// (the MMA warp runs up to three groups ahead of the barrier round trip that
+// frees a buffer) and sixteen rescale warps fold it into an fp32 accumulator in
+// registers,
 // acc = fma(P_g, RN(sa * sb), acc) in group order (sa * sb is exact in fp32:
 // both are fp16 values), while the MMA warp fills the other buffer.  The bf16
 // branch product u' L^T comes last, as one more group with scale 1.
 //
-// CTA = one 128 x 128 output tile (one K split of it), 10 warps:
+// CTA = one 128 x 128 output tile (one K split of it), 18 warps:
 //   warp 0    TMA producer.  A stage is K 128 (two groups): the A and B level
 //             boxes (128 rows x 128 bytes, 128B swizzle) and the two groups'
 //             fp32 scales of the tile's rows and of its columns; U and L once.
 //             The weight boxes of the first stage go out before the wait on
 //             the kernel that writes A.
-//   warp 1    TMEM owner and MMA issuer: two MMAs (K 32) per group.
-//   warps 2-9 rescale and epilogue: warp w reads TMEM lane quarter w % 4,
-//             columns [64 h, 64 h + 64), h = (w - 2) / 4: one thread = one
-//             output row x 64 columns.
+//   warp 1    TMEM owner and MMA issuer: two MMAs (K 32) per group into
+//             buffer g % 4.
+//   warps 2-17 rescale and epilogue: warp w reads TMEM lane quarter w % 4,
+//             columns [32 h, 32 h + 32), h = (w - 2) / 4: one thread = one
+//             output row x 32 columns.  The rescale is a chain of dependent
+//             loads and packed FMAs per group; four such warps per scheduler
+//             keep its issue slots busy where two left them idle two thirds of
+//             the time.
 // Split K (few output tiles): each split writes its fp32 partial tile and a
 // second kernel sums the splits in order, adds the bias and rounds to bf16.
 // Every mbarrier wait is bounded.  No TMA multicast.
@@ -50,9 +56,23 @@ constexpr int kOffL = kOffU + 8192;           // L tile: 128 rows x r bf16
 constexpr int kOffBar = kOffL + 8192;
 constexpr int kSmem = kOffBar + 256 + 1024;
 constexpr int kRescaleWarp0 = 2;
-constexpr int kRescaleWarps = 8;
+constexpr int kRescaleWarps = 16;
+constexpr int kCols = kTile * 4 / kRescaleWarps;  // output columns per rescale thread
+static_assert(kCols == 32, "one 32-column TMEM load per group per rescale thread");
 constexpr int kThreads = 32 * (kRescaleWarp0 + kRescaleWarps);
-constexpr uint32_t kTmemCols = 256;  // two 128-column group buffers
+constexpr int kBufs = 4;             // 128-column TMEM group buffers
+constexpr uint32_t kTmemCols = 128 * kBufs;
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 static_assert(kStageBytes % 1024 == 0, "128B-swizzled boxes stay 1024-byte aligned");
 
@@ -63,9 +83,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);  // [kStages] levels and scales landed
   uint64_t* empty = full + kStages;                               // [kStages] MMAs done with the levels
   uint64_t* sc_free = empty + kStages;                            // [kStages] rescale warps done with the scales
-  uint64_t* acc_full = sc_free + kStages;                         // [2] a group's P in the buffer
-  uint64_t* acc_empty = acc_full + 2;                             // [2] the buffer read out
-  uint64_t* branch_full = acc_empty + 2;
+  uint64_t* acc_full = sc_free + kStages;                         // [kBufs] a group's P in the buffer
+  uint64_t* acc_empty = acc_full + kBufs;                         // [kBufs] the buffer read out
+  uint64_t* branch_full = acc_empty + kBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(branch_full + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[i], 1);
       mbar_init(&sc_free[i], kRescaleWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kRescaleWarps);
     }
@@ -156,11 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_f8e4m3(kTile, kTile);
       bool ok = true;
-      // buffer g & 1 read out by the rescale warps since its last group
+      // buffer g % kBufs read out by the rescale warps since its last group
       auto take = [&](int g) {
-        const int use = g >> 1;
-        return use == 0 ||
-               mbar_wait(&acc_empty[g & 1], static_cast<uint32_t>(use - 1) & 1u, p.err, DEVERR_MMA_WAIT, wlim);
+        const int use = g / kBufs;
+        return use == 0 || mbar_wait(&acc_empty[g % kBufs], static_cast<uint32_t>(use - 1) & 1u, p.err,
+                                     DEVERR_MMA_WAIT, wlim);
       };
       int g = 0;
       for (int s = 0; ok && s < n_st; ++s) {
@@ -178,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + 128u * static_cast<uint32_t>(g & 1);
+          const uint32_t d = tmem + 128u * static_cast<uint32_t>(g % kBufs);
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             // 32 bytes of each operand row per MMA (K 32), inside the 128-byte swizzle atom
@@ -186,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = smem_desc(b_s + j * 64 + kk * 32, 16, 1024, 2);
             mma_f8(d, ad, bd, idesc, kk ? 1u : 0u);
           }
-          tc_commit(&acc_full[g & 1]);
+          tc_commit(&acc_full[g % kBufs]);
         }
         tc_commit(&empty[st]);
       }
@@ -195,38 +215,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t layout = p.branch_k == 32 ? 4u : 6u;  // 64B / 32B swizzle
         const uint32_t sbo = 8u * static_cast<uint32_t>(p.branch_k) * 2u;
         const uint32_t us = smem_u32(smem + kOffU), ls = smem_u32(smem + kOffL);
-        const uint32_t d = tmem + 128u * static_cast<uint32_t>(g & 1);
+        const uint32_t d = tmem + 128u * static_cast<uint32_t>(g % kBufs);
         for (int kk = 0; kk < p.branch_k / 16; ++kk)
           mma_bf16(d, smem_desc(us + kk * 32, 16, sbo, layout), smem_desc(ls + kk * 32, 16, sbo, layout),
                    idesc_bf16(kTile, kTile), kk ? 1u : 0u);
-        tc_commit(&acc_full[g & 1]);
+        tc_commit(&acc_full[g % kBufs]);
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------ rescale and epilogue
-    const int ew = warp - kRescaleWarp0;  // 0..7
+    const int ew = warp - kRescaleWarp0;  // 0..15
     const int qd = warp & 3;              // TMEM lane quarter this warp may access
-    const int h = ew >> 2;                // column half
+    const int h = ew >> 2;                // column quarter
     const int row_l = qd * 32 + lane;
     const int row = m0 + row_l;
-    const int c0 = n0 + h * 64;
-    const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(h * 64);
-    float2 acc[32];
+    const int c0 = n0 + h * kCols;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(h * kCols);
+    float2 acc[kCols / 2];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) acc[q] = make_float2(0.0f, 0.0f);
+    for (int q = 0; q < kCols / 2; ++q) acc[q] = make_float2(0.0f, 0.0f);
     griddep_wait();  // y / the partial tiles may still be read by the kernel before this one
     bool alive = true;
     for (int g = 0; alive && g < n_groups; ++g) {
-      const int b = g & 1;
+      const int b = g % kBufs;
       // warp-uniform outcome: the TMEM loads below are warp-collective
-      alive = __all_sync(0xffffffffu,
-                         mbar_wait(&acc_full[b], static_cast<uint32_t>(g >> 1) & 1u, p.err, DEVERR_EPILOGUE_WAIT, wlim));
+      alive = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], static_cast<uint32_t>(g / kBufs) & 1u, p.err,
+                                                DEVERR_EPILOGUE_WAIT, wlim));
       if (!alive) break;
       tc_fence_after();
-      uint32_t r0[32], r1[32];
+      uint32_t r0[32];
       tmem_ld_32x32b_x32(taddr + 128u * static_cast<uint32_t>(b), r0);
-      tmem_ld_32x32b_x32(taddr + 128u * static_cast<uint32_t>(b) + 32u, r1);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -234,16 +253,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < 2 * n_st) {
         const int s = g >> 1, j = g & 1, st = s % kStages;
         // the stage's TMA writes (the scales) are complete and visible
-        alive = __all_sync(0xffffffffu, mbar_wait(&full[st], static_cast<uint32_t>(s / kStages) & 1u, p.err,
-                                                   DEVERR_EPILOGUE_WAIT, wlim));
-        const float* sa = reinterpret_cast<const float*>(smem + st * kStageBytes + kOffSA) + j * kTile;
-        const float* sb = reinterpret_cast<const float*>(smem + st * kStageBytes + kOffSB) + j * kTile + h * 64;
-        const float a = sa[row_l];
+        if (j == 0)
+          alive = __all_sync(0xffffffffu, mbar_wait(&full[st], static_cast<uint32_t>(s / kStages) & 1u, p.err,
+                                                     DEVERR_EPILOGUE_WAIT, wlim));
+        const uint32_t sbase = smem_u32(smem + st * kStageBytes);
+        const uint32_t sa = sbase + kOffSA + 4u * static_cast<uint32_t>(j * kTile);
+        const uint32_t sb = sbase + kOffSB + 4u * static_cast<uint32_t>(j * kTile + h * kCols);
+        const float a = lds_f32(sa + 4u * static_cast<uint32_t>(row_l));
         const float2 a2 = make_float2(a, a);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float4 w4 = *reinterpret_cast<const float4*>(sb + 4 * q);
-          const uint32_t* r = q < 8 ? r0 + 4 * q : r1 + 4 * (q - 8);
+        for (int q = 0; q < kCols / 4; ++q) {
+          const float4 w4 = lds_f32x4(sb + 16u * q);
+          const uint32_t* r = r0 + 4 * q;
           const float2 w01 = f2_mul(make_float2(w4.x, w4.y), a2);  // exact: fp16 x fp16
           const float2 w23 = f2_mul(make_float2(w4.z, w4.w), a2);
           acc[2 * q] = f2_fma(make_float2(__uint_as_float(r[0]), __uint_as_float(r[1])), w01, acc[2 * q]);
@@ -254,10 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         // the branch u' L^T, scale 1
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < kCols / 2; ++q)
           acc[q] = f2_add(acc[q], make_float2(__uint_as_float(r0[2 * q]), __uint_as_float(r0[2 * q + 1])));
-          acc[16 + q] = f2_add(acc[16 + q], make_float2(__uint_as_float(r1[2 * q]), __uint_as_float(r1[2 * q + 1])));
-        }
       }
     }
     if (alive && row < p.M) {
@@ -266,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint16_t* bias = static_cast<const uint16_t*>(p.bias);
         uint16_t* yrow = static_cast<uint16_t*>(p.y) + static_cast<size_t>(row) * p.N;
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
+        for (int q8 = 0; q8 < kCols / 8; ++q8) {
           const int n = c0 + 8 * q8;
           if (n >= p.N) break;
           const uint4 bw = bias ? __ldg(reinterpret_cast<const uint4*>(bias + n)) : make_uint4(0u, 0u, 0u, 0u);
@@ -278,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         float* prow = p.partial + (static_cast<size_t>(split) * p.M + row) * p.N;
 #pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
+        for (int q4 = 0; q4 < kCols / 4; ++q4) {
           const int n = c0 + 4 * q4;
           if (n >= p.N) break;
           *reinterpret_cast<float4*>(prow + n) =
