@@ -63,6 +63,23 @@ constexpr int kThreads = 32 * (kRescaleWarp0 + kRescaleWarps);
 constexpr int kBufs = 4;             // 128-column TMEM group buffers
 constexpr uint32_t kTmemCols = 128 * kBufs;
 
+// acc0/1 += P0/1 * RN(w0/1 * a): two packed fp32 operations (RN(w a) is exact
+// here: w and a are fp16 values), written as one block so the pairs are formed
+// in registers once.
+__device__ __forceinline__ void rescale2(float& acc0, float& acc1, uint32_t p0, uint32_t p1, float w0, float w1,
+                                         float a) {
+  asm("{\n\t.reg .b64 pp, ww, aa, cc;\n\t"
+      "mov.b64 pp, {%2, %3};\n\t"
+      "mov.b64 ww, {%4, %5};\n\t"
+      "mov.b64 aa, {%6, %6};\n\t"
+      "mov.b64 cc, {%0, %1};\n\t"
+      "mul.rn.f32x2 ww, ww, aa;\n\t"
+      "fma.rn.f32x2 cc, pp, ww, cc;\n\t"
+      "mov.b64 {%0, %1}, cc;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(p0), "r"(p1), "f"(w0), "f"(w1), "f"(a));
+}
+
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
@@ -232,9 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = m0 + row_l;
     const int c0 = n0 + h * kCols;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(h * kCols);
-    float2 acc[kCols / 2];
+    float acc[kCols];
 #pragma unroll
-    for (int q = 0; q < kCols / 2; ++q) acc[q] = make_float2(0.0f, 0.0f);
+    for (int q = 0; q < kCols; ++q) acc[q] = 0.0f;
     griddep_wait();  // y / the partial tiles may still be read by the kernel before this one
     bool alive = true;
     for (int g = 0; alive && g < n_groups; ++g) {
@@ -260,23 +277,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sa = sbase + kOffSA + 4u * static_cast<uint32_t>(j * kTile);
         const uint32_t sb = sbase + kOffSB + 4u * static_cast<uint32_t>(j * kTile + h * kCols);
         const float a = lds_f32(sa + 4u * static_cast<uint32_t>(row_l));
-        const float2 a2 = make_float2(a, a);
 #pragma unroll
         for (int q = 0; q < kCols / 4; ++q) {
           const float4 w4 = lds_f32x4(sb + 16u * q);
-          const uint32_t* r = r0 + 4 * q;
-          const float2 w01 = f2_mul(make_float2(w4.x, w4.y), a2);  // exact: fp16 x fp16
-          const float2 w23 = f2_mul(make_float2(w4.z, w4.w), a2);
-          acc[2 * q] = f2_fma(make_float2(__uint_as_float(r[0]), __uint_as_float(r[1])), w01, acc[2 * q]);
-          acc[2 * q + 1] = f2_fma(make_float2(__uint_as_float(r[2]), __uint_as_float(r[3])), w23, acc[2 * q + 1]);
+          rescale2(acc[4 * q], acc[4 * q + 1], r0[4 * q], r0[4 * q + 1], w4.x, w4.y, a);
+          rescale2(acc[4 * q + 2], acc[4 * q + 3], r0[4 * q + 2], r0[4 * q + 3], w4.z, w4.w, a);
         }
         __syncwarp();
         if (j == 1 && lane == 0) mbar_arrive(&sc_free[st]);
       } else {
         // the branch u' L^T, scale 1
 #pragma unroll
-        for (int q = 0; q < kCols / 2; ++q)
-          acc[q] = f2_add(acc[q], make_float2(__uint_as_float(r0[2 * q]), __uint_as_float(r0[2 * q + 1])));
+        for (int q = 0; q < kCols; ++q) acc[q] = __fadd_rn(acc[q], __uint_as_float(r0[q]));
       }
     }
     if (alive && row < p.M) {
@@ -289,9 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = c0 + 8 * q8;
           if (n >= p.N) break;
           const uint4 bw = bias ? __ldg(reinterpret_cast<const uint4*>(bias + n)) : make_uint4(0u, 0u, 0u, 0u);
-          const float2* a4 = acc + 4 * q8;
-          const uint4 o = make_uint4(fma_bf16x2(a4[0].x, a4[0].y, 1.0f, bw.x), fma_bf16x2(a4[1].x, a4[1].y, 1.0f, bw.y),
-                                     fma_bf16x2(a4[2].x, a4[2].y, 1.0f, bw.z), fma_bf16x2(a4[3].x, a4[3].y, 1.0f, bw.w));
+          const float* a8 = acc + 8 * q8;
+          const uint4 o = make_uint4(fma_bf16x2(a8[0], a8[1], 1.0f, bw.x), fma_bf16x2(a8[2], a8[3], 1.0f, bw.y),
+                                     fma_bf16x2(a8[4], a8[5], 1.0f, bw.z), fma_bf16x2(a8[6], a8[7], 1.0f, bw.w));
           *reinterpret_cast<uint4*>(yrow + n) = o;
         }
       } else {
@@ -300,8 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q4 = 0; q4 < kCols / 4; ++q4) {
           const int n = c0 + 4 * q4;
           if (n >= p.N) break;
-          *reinterpret_cast<float4*>(prow + n) =
-              make_float4(acc[2 * q4].x, acc[2 * q4].y, acc[2 * q4 + 1].x, acc[2 * q4 + 1].y);
+          *reinterpret_cast<float4*>(prow + n) = make_float4(acc[4 * q4], acc[4 * q4 + 1], acc[4 * q4 + 2], acc[4 * q4 + 3]);
         }
       }
     }
