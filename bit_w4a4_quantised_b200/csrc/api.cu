@@ -285,12 +285,15 @@ qwam_status arena_get(int dev, size_t need, Arena** out) {
 }
 
 // CTAs along K per 128-row tile of the prologue: the largest power of two
-// that divides the chunk count (K / 128), is at most 8 (one portable cluster)
-// and keeps the grid within one wave of the SMs (at least one part).
+// that divides the chunk count (K / 128), is at most 8 (one portable cluster;
+// 16 for a single row tile) and keeps the grid within one wave of the SMs (at
+// least one part).
 int cluster_parts(int K, int rows, int sms) {
   const int chunks = K / 128;
   const int tiles = (rows + 127) / 128;
-  for (int c = 8; c > 1; c >>= 1)
+  // one row tile (the 32-token layers): up to 16 CTAs (non-portable cluster
+  // size; the launch falls back to 8 where the device cannot place 16)
+  for (int c = tiles == 1 ? 16 : 8; c > 1; c >>= 1)
     if (chunks % c == 0 && tiles * c <= sms) return c;
   return 1;
 }

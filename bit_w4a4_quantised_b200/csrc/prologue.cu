@@ -50,7 +50,7 @@ constexpr int kRows = 128;
 constexpr int kChunk = 128;
 constexpr int kRowWarps = 8;
 constexpr int kRowThreads = 32 * kRowWarps;
-constexpr int kMaxParts = 8;
+constexpr int kMaxParts = 16;  // 16: a non-portable cluster size (one 128-row tile only)
 
 // What one ring load brings in.
 enum : uint32_t { LD_X = 1u, LD_P = 2u, LD_V = 4u, LD_CH = 8u };
@@ -105,7 +105,7 @@ struct PCfg {
   static constexpr int OFF_RS = kTC ? OFF_ALO : OFF_UA + UA_BYTES;
   static constexpr int OFF_UG = kTC ? SLOT + OFF_ALO : OFF_RS + RS_BYTES;
   static constexpr int OFF_BAR = kTC ? OFF_UA + UA_BYTES : OFF_UG + UG_BYTES;
-  static constexpr int OFF_RED = OFF_BAR + 128;       // warp maxima [0, 8), CTA maxima by rank [8, 16)
+  static constexpr int OFF_RED = OFF_BAR + 128;       // warp maxima [0, 8), CTA maxima by rank [8, 8 + kMaxParts)
   static constexpr int SMEM = OFF_RED + 128 + 1024;
   // TMEM: D2 [0, 128) (TC: two Z accumulators [0, 256)), then T P^T hi | lo (2R columns)
   static constexpr uint32_t U_COL = kTC ? 256 : 128;
@@ -973,15 +973,16 @@ __global__ void __launch_bounds__(PCfg<R, MODE, W>::THREADS, 1)
 }
 
 template <int R, int MODE, int W>
-cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p, cudaStream_t st) {
+cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p_in, cudaStream_t st) {
   using C = PCfg<R, MODE, W>;
   auto kern = prologue_kernel<R, MODE, W>;
   static const cudaError_t smem_attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (smem_attr != cudaSuccess) return smem_attr;
+  PrologueParams p = p_in;
   if (p.parts < 1 || p.parts > kMaxParts || (p.parts & (p.parts - 1))) return cudaErrorInvalidValue;
+  static_assert(8 + kMaxParts <= 32, "per-rank maxima fit the reduction area");
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.parts, (p.rows + kRows - 1) / kRows, 1);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
@@ -990,6 +991,37 @@ cudaError_t launch_one(const ProMaps& maps, const PrologueParams& p, cudaStream_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (C::kCluster && p.parts > 8) {
+    // 16 CTAs per cluster is beyond the portable size: allowed per kernel, and
+    // used only when the device can place such a cluster (else 8 CTAs with
+    // twice the chunks each)
+    static const bool ok16 = [&]() {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+      }
+      cudaLaunchConfig_t q = cfg;
+      cudaLaunchAttribute a = {};
+      a.id = cudaLaunchAttributeClusterDimension;
+      a.val.clusterDim.x = 16;
+      a.val.clusterDim.y = 1;
+      a.val.clusterDim.z = 1;
+      q.attrs = &a;
+      q.numAttrs = 1;
+      q.gridDim = dim3(16, 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+      }
+      return n > 0;
+    }();
+    if (!ok16) {
+      p.parts = 8;
+      p.chunks *= 2;
+    }
+  }
+  cfg.gridDim = dim3(p.parts, (p.rows + kRows - 1) / kRows, 1);
   if (C::kCluster) {
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = p.parts;
