@@ -54,9 +54,10 @@ constexpr int kScaleSlots = 4;  // TMEM scale ring, one stage per slot
 
 // F8: the FP8 W8A8 arm (E4M3 operands, kind::f8f6f4, one byte per element, no
 // block scales); otherwise NVFP4 (packed E2M1, E4M3 scale per 16 in TMEM).
-// NB: no low-rank branch (r = 0); CTA pairs use the branch tiles' room for a
-// fifth operand stage (the stage ring is bound by its round trip, not by the
-// tensor core: more bytes in flight is more throughput).
+// NB: no low-rank branch (r = 0): no room for the branch tiles.  CTA pairs
+// keep five operand stages (the stage ring is bound by its round trip, not by
+// the tensor core: more bytes in flight is more throughput), which just fit
+// beside the branch tiles too.
 template <int BN, int KS, bool PAIR = false, bool F8 = false, bool NB = false>
 struct Cfg {
   static constexpr int TM = PAIR ? 2 * kBM : kBM;          // rows of an output tile
@@ -65,7 +66,7 @@ struct Cfg {
   static constexpr int KM = F8 ? KS / 32 : KS / 64;         // MMAs per stage (K 32 for FP8, 64 for FP4)
   static constexpr int K64 = KS / 64;                       // K64 steps of a stage (FP4 scale blocks)
   static constexpr uint32_t SWZ = ROWB == 128 ? 2u : 4u;    // UMMA layout: 128B / 64B swizzle
-  static constexpr int STAGES = PAIR ? (NB ? 5 : 4) : (ROWB == 128 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
+  static constexpr int STAGES = PAIR ? 5 : (ROWB == 128 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 6 : 8));
   static constexpr int NSFB = F8 ? 0 : BN / 128;            // 128-row scale blocks of B
   static constexpr int SF_BLK = F8 ? 0 : K64 * 512;         // one 128-row scale block of a stage
   static constexpr int NBOX = F8 ? 2 : 4;                   // boxes per stage: A, B (, A scales, B scales)
