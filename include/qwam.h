@@ -220,7 +220,9 @@ qwam_status qwam_linear(const void* x_bf16, int M, qwam_handle h, void* y_bf16, 
  * same GEMM plan), but all scratch lives in one fixed 2 MiB array compiled
  * into the library (one copy per device) instead of the growable workspace.
  * Limits: M <= 128 rows and K <= 16384 (QWAM_ERR_SHAPE beyond them, before
- * anything is launched); within them every N, r and b that qwam_linear takes.
+ * anything is launched); within them every N, r and b that qwam_linear takes,
+ * except that an INT4 handle's split-K partial tiles (splits x M x N x 4
+ * bytes) must fit the array too (QWAM_ERR_SHAPE otherwise).
  * The first call on a device does the set-up (looks up the array's device
  * address and clears its header, whose error word must start at zero,
  * synchronising the device); make that first call before any latency-critical

@@ -60,3 +60,19 @@ def test_argument_errors_need_no_device(lib):
 def test_built_for_sm100a_only():
     src = open(os.path.join(ROOT, "bit_w4a4_quantised_b200", "build.py")).read()
     assert "arch=compute_100a,code=sm_100a" in src
+
+
+def test_int4_and_image_entry_points_check_arguments_first(lib):
+    import ctypes
+    assert lib.qwam_status_string(8) == b"QWAM_ERR_FORMAT"
+    out = ctypes.c_void_p()
+    # NULL out pointer / NULL weight: refused before any device call
+    assert lib.qwam_prepare_weight_int4(None, 16, 128, None, None, 0, None, None, None, None) == 1
+    assert lib.qwam_prepare_weight_int4(None, 16, 128, None, None, 0, None, None, None, ctypes.byref(out)) == 1
+    # the bare group GEMM: NULL buffers, then shapes, before any device call
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks stop first
+    assert lib.qwam_int4_gemm(None, fake, fake, fake, 4, 16, 128, fake, None) == 1
+    assert lib.qwam_int4_gemm(fake, fake, fake, fake, 3, 16, 128, fake, None) == 2   # M % 4
+    assert lib.qwam_int4_gemm(fake, fake, fake, fake, 4, 24, 128, fake, None) == 2   # N % 16
+    assert lib.qwam_int4_gemm(fake, fake, fake, fake, 4, 16, 192, fake, None) == 2   # K % 128
+    assert b"multiple" in lib.qwam_last_error()
