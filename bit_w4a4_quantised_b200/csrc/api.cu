@@ -884,12 +884,16 @@ uint8_t e4m3_of_level(int v) {
   return static_cast<uint8_t>((v < 0 ? 0x80 : 0) | ((e + 7) << 3) | m);
 }
 bool level_of_e4m3(uint8_t b, int* v) {
-  for (int l = -8; l <= 7; ++l)
-    if (e4m3_of_level(l) == b || (l == 0 && b == 0x80)) {
-      *v = l;
-      return true;
-    }
-  return false;
+  // byte -> level + 8 (0..15), or -1 for a byte that is no level
+  static const std::vector<int8_t> lut = [] {
+    std::vector<int8_t> t(256, -1);
+    for (int l = -8; l <= 7; ++l) t[e4m3_of_level(l)] = static_cast<int8_t>(l + 8);
+    t[0x80] = 8;  // -0
+    return t;
+  }();
+  if (lut[b] < 0) return false;
+  *v = lut[b] - 8;
+  return true;
 }
 // fp16 bits of an fp32 value that fp16 holds exactly (false otherwise), and back.
 bool half_bits_exact(float f, uint16_t* out) {

@@ -16,7 +16,7 @@
 // frees a buffer) and sixteen rescale warps fold it into an fp32 accumulator in
 // registers,
 // acc = fma(P_g, RN(sa * sb), acc) in group order (sa * sb is exact in fp32:
-// both are fp16 values), while the MMA warp fills the other buffer.  The bf16
+// both are fp16 values), while the MMA warp fills the other buffers.  The bf16
 // branch product u' L^T comes last, as one more group with scale 1.
 //
 // CTA = one 128 x 128 output tile (one K split of it), 18 warps:
@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = sc_free + kStages;                         // [kBufs] a group's P in the buffer
   uint64_t* acc_empty = acc_full + kBufs;                         // [kBufs] the buffer read out
   uint64_t* branch_full = acc_empty + kBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(branch_full + 1);
+  uint64_t* mma_done = branch_full + 1;  // every MMA of this CTA complete (before TMEM is freed)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t wlim = p.wait_ns ? p.wait_ns : kWaitLimitNs;
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], kRescaleWarps);
     }
     mbar_init(branch_full, 1);
+    mbar_init(mma_done, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -238,6 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                    idesc_bf16(kTile, kTile), kk ? 1u : 0u);
         tc_commit(&acc_full[g % kBufs]);
       }
+      // on every path (an expired wait included) no MMA may still be writing
+      // TMEM when it is freed
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, p.err, DEVERR_DRAIN_WAIT, wlim);
     }
     __syncwarp();
   } else {
