@@ -98,6 +98,14 @@ WORKLOADS = {
     "c4down": dict(make=lambda i, seed: workloads.c4_video_ffn_down(seed=seed + i),
                    desc="video-expert FFN down, 4096 tokens, 14336->3072, r=32, b=128",
                    unit="TFLOP/s", steps=500, warmup=5),
+    # the video FFN layers as the denoising step holds them (r = 0): --workload only, for
+    # per-shape evidence on the step's video GEMM group
+    "c5ffn0": dict(make=lambda i, seed: workloads.c5_layer(8, seed=seed + i),
+                   desc="video-expert FFN up as in the denoising step, 4096 tokens, 3072->14336, r=0, b=128",
+                   unit="TFLOP/s", steps=500, warmup=5),
+    "c5ffn2": dict(make=lambda i, seed: workloads.c5_layer(9, seed=seed + i),
+                   desc="video-expert FFN down as in the denoising step, 4096 tokens, 14336->3072, r=0, b=128",
+                   unit="TFLOP/s", steps=500, warmup=5),
     # the other arms of the boundary on the same layers
     "c3r0fp8": dict(make=lambda i, seed: workloads.c3_video_attn(0, seed=seed, layer=i), fmt="fp8",
                     desc="FP8 W8A8 arm: video-expert attention projection, 4096 tokens, 3072->3072, r=0, b=128",
@@ -732,7 +740,7 @@ def bench_set(ctx, args, name, steps, warmup, cpu_budget):
     value = per_unit(set_bytes * steps * ctx.world, ms / 1e3, unit)
     groups = _group_roofs(layers, pro, gem, peaks, timed_alone=False)
     dom = max(groups, key=lambda k: groups[k]["share"])
-    roof = dict(groups[dom], group=dom, traffic=None,
+    roof = dict(groups[dom], group=dom, traffic=recorded_traffic("c5", dom),
                 duration_note="CUDA events around each kernel of every layer, one replay of the set's graph with "
                               "event nodes added, right after the timed region",
                 set_frac=value / ctx.world / peaks["hbm_gbs"])
