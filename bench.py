@@ -740,7 +740,7 @@ def bench_set(ctx, args, name, steps, warmup, cpu_budget):
     value = per_unit(set_bytes * steps * ctx.world, ms / 1e3, unit)
     groups = _group_roofs(layers, pro, gem, peaks, timed_alone=False)
     dom = max(groups, key=lambda k: groups[k]["share"])
-    roof = dict(groups[dom], group=dom, traffic=recorded_traffic("c5", dom),
+    roof = dict(groups[dom], group=dom, traffic=recorded_traffic(name, dom),
                 duration_note="CUDA events around each kernel of every layer, one replay of the set's graph with "
                               "event nodes added, right after the timed region",
                 set_frac=value / ctx.world / peaks["hbm_gbs"])
@@ -852,7 +852,7 @@ def bench_step(ctx, args, steps, warmup, cpu_budget):
     value = per_unit(step_flops * steps * ctx.world, ms / 1e3, "TFLOP/s")
     groups = _group_roofs(layers, pro, gem, peaks, timed_alone=False)
     dom = max(groups, key=lambda k: groups[k]["share"])
-    roof = dict(groups[dom], group=dom, traffic=None,
+    roof = dict(groups[dom], group=dom, traffic=recorded_traffic("c5", dom),
                 duration_note="CUDA events around each kernel of every layer, one replay of the step's graph with "
                               "event nodes added, right after the timed region; achieved = the group's algorithmic "
                               "flops (or bytes) over its summed durations")
