@@ -223,26 +223,43 @@ def fp4_peak(peaks, timed_alone):
                          f"against 4 x the burst figure")
 
 
-def csrc_digest():
-    files = sorted(glob.glob(os.path.join(ROOT, "bit_w4a4_quantised_b200", "csrc", "*")))
+# Sources every kernel's traffic depends on (launch planning included), and the
+# file that builds each kernel family.
+SHARED_SOURCES = ("common.cuh", "quant.cuh", "kernels.h", "api.cu")
+KERNEL_SOURCES = {"fp4_gemm": ("gemm.cu",), "prologue": ("prologue.cu",), "onepass": ("prologue_wide.cu",),
+                  "wide_prologue": ("prologue_wide.cu",), "group_gemm": ("group_gemm.cu",)}
+
+
+def sources_digest(names):
+    """sha256 over the named files of csrc/ (name and bytes, in sorted order)."""
     h = hashlib.sha256()
-    for p in files:
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
+    for name in sorted(names):
+        with open(os.path.join(ROOT, "bit_w4a4_quantised_b200", "csrc", name), "rb") as f:
+            h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()
 
 
+def traffic_sources(family):
+    return sorted(set(SHARED_SOURCES) | set(KERNEL_SOURCES[family]))
+
+
 def recorded_traffic(workload, kernel):
     """DRAM bytes per launch from a committed ncu summary, or None when the
-    kernel sources changed since those counters were taken."""
+    sources of the captured kernel (its .cu file, the shared headers and the
+    launch planning) changed since those counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{workload}:{kernel}")
-    if not e or e.get("csrc_sha256") != csrc_digest():
+    if not e or not e.get("sources"):
+        return None
+    try:
+        if e.get("sources_sha256") != sources_digest(e["sources"]):
+            return None
+    except OSError:
         return None
     return e.get("bytes_per_launch")
 

@@ -6,6 +6,7 @@ The per-layer bytes follow the minimal-traffic definition (x, packed W_d with
 its E4M3 scales, L, V, s, bias, y) and are checked against values worked out by
 hand for the configs' shapes, so a dropped or doubled term fails here."""
 import json
+import os
 
 import pytest
 
@@ -71,17 +72,43 @@ def test_action_set_members_are_the_step_specs():
 
 
 def test_recorded_traffic_needs_the_same_sources(tmp_path, monkeypatch):
+    import shutil
+    src = os.path.join(bench.ROOT, "bit_w4a4_quantised_b200", "csrc")
+    csrc = tmp_path / "bit_w4a4_quantised_b200" / "csrc"
+    shutil.copytree(src, csrc)
     prof = tmp_path / "profiles"
     prof.mkdir()
-    entry = {"bytes_per_launch": 1234, "csrc_sha256": bench.csrc_digest(), "from": "x.md"}
-    (prof / "traffic.json").write_text(json.dumps({"c2:prologue_kernel": entry,
-                                                   "c3:prologue_kernel": dict(entry, csrc_sha256="0" * 64)}))
-    digest = entry["csrc_sha256"]  # of the real sources, taken before ROOT moves
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "csrc_digest", lambda: digest)
+    pro, gem = bench.traffic_sources("prologue"), bench.traffic_sources("fp4_gemm")
+    assert "prologue.cu" in pro and "gemm.cu" not in pro and "api.cu" in pro
+    entry = {"bytes_per_launch": 1234, "sources": pro, "sources_sha256": bench.sources_digest(pro)}
+    (prof / "traffic.json").write_text(json.dumps({
+        "c2:prologue_kernel": entry,
+        "c3:prologue_kernel": dict(entry, sources_sha256="0" * 64),
+        "c3r0:fp4_gemm_kernel": {"bytes_per_launch": 99, "sources": gem, "sources_sha256": bench.sources_digest(gem)},
+        "c4down:prologue_kernel": {"bytes_per_launch": 7, "csrc_sha256": "0" * 64}}))
     assert bench.recorded_traffic("c2", "prologue_kernel") == 1234
-    assert bench.recorded_traffic("c3", "prologue_kernel") is None
-    assert bench.recorded_traffic("c4up", "fp4_gemm_kernel") is None
+    assert bench.recorded_traffic("c3", "prologue_kernel") is None       # other sources
+    assert bench.recorded_traffic("c4up", "fp4_gemm_kernel") is None     # not recorded
+    assert bench.recorded_traffic("c4down", "prologue_kernel") is None   # no source list
+    # a change to the GEMM's file leaves the prologue's figure valid, and not the reverse
+    with open(csrc / "gemm.cu", "a") as f:
+        f.write("// edited\n")
+    assert bench.recorded_traffic("c2", "prologue_kernel") == 1234
+    assert bench.recorded_traffic("c3r0", "fp4_gemm_kernel") is None
+    # a shared header invalidates both
+    with open(csrc / "common.cuh", "a") as f:
+        f.write("// edited\n")
+    assert bench.recorded_traffic("c2", "prologue_kernel") is None
+
+
+def test_committed_traffic_entries_name_their_sources():
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    for key, e in d.items():
+        assert e["bytes_per_launch"] > 0, key
+        assert set(bench.SHARED_SOURCES) <= set(e["sources"]), key
+        assert len(e["sources_sha256"]) == 64, key
 
 
 def test_per_unit():
