@@ -77,3 +77,12 @@ def device_operand_reference(case, h, x, rows=None, variant="deflated"):
             L = asp.prepare_weight(case.W, case.s, case.V, case.b, fp4=False)["L"]
         y = y + u @ L.T
     return y + np.asarray(case.bias, dtype=np.float64)[None, :]
+
+
+def sample_rows(M: int, n: int = 48, seed: int = 7) -> np.ndarray:
+    """Rows checked at full size: the first and last rows of the first, a middle
+    and the last 128-row tiles, plus n seeded random rows."""
+    rng = np.random.default_rng(seed)
+    edge = [0, 1, 127, 128, 255, 256, M // 2, M - 129, M - 128, M - 2, M - 1]
+    rows = np.concatenate([np.array(edge), rng.integers(0, M, n)])
+    return np.unique(np.clip(rows, 0, M - 1))

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 from bit_w4a4_quantised_b200 import workloads
-from gpu_util import bf16_to_np, codes_of, device_operand_reference, local_rel_errors, prepare
+from gpu_util import bf16_to_np, codes_of, device_operand_reference, local_rel_errors, prepare, sample_rows
 from oracle import asp, nvfp4
 
 pytestmark = pytest.mark.gpu
@@ -28,14 +28,12 @@ CASES = {
     "c3_r32": lambda: workloads.c3_video_attn(32),
     "c4_up": lambda: workloads.c4_video_ffn_up(),
     "c4_down": lambda: workloads.c4_video_ffn_down(),
+    # the video FFN pair as the denoising step holds it (r = 0): FFN up through
+    # the one-launch rank-0 prologue, FFN down (K = 14336, 32 row tiles per CTA)
+    # through the two-launch rank-0 form, both into CTA-pair tiles without a branch
+    "c5_video_ffn0_r0": lambda: workloads.c5_layer(8),
+    "c5_video_ffn2_r0": lambda: workloads.c5_layer(9),
 }
-
-
-def sample_rows(M: int, n: int = 48, seed: int = 7) -> np.ndarray:
-    rng = np.random.default_rng(seed)
-    edge = [0, 1, 127, 128, 255, 256, M // 2, M - 129, M - 128, M - 2, M - 1]
-    rows = np.concatenate([np.array(edge), rng.integers(0, M, n)])
-    return np.unique(np.clip(rows, 0, M - 1))
 
 
 @pytest.mark.parametrize("name", sorted(CASES))

@@ -68,3 +68,40 @@ def test_fp8_arm_matches_oracle(name):
     own = own + case.bias.astype(np.float64)[None, :]
     row_err, blk_err = local_rel_errors(got, own)
     assert row_err <= LOCAL_TOL and blk_err <= LOCAL_TOL, (row_err, blk_err)
+
+
+def test_fp8_full_size_on_sampled_rows():
+    """The FP8 arm on the 4096 x 3072 -> 3072 rank-0 layer, as the benchmark
+    runs it (one-launch rank-0 prologue, CTA-pair FP8 tiles): quantisers
+    bit-exact on the device's own full inputs, the per-tensor scales from the
+    whole input, the output on sampled rows against the oracle."""
+    import torch
+    from bit_w4a4_quantised_b200 import binding as qw
+    from gpu_util import sample_rows
+    case = workloads.c3_video_attn(0)
+    h, x, wd = prepare(case, wd_out=True, fmt="fp8")
+    y = qw.linear(x, h)
+    d = qw.debug_prologue(x, h)
+    w = qw.export_weight(h)
+    torch.cuda.synchronize()
+    assert qw.device_error() == 0
+
+    z = d["z"].cpu().numpy()
+    ca, ga = fp8.quantize(z)
+    assert np.float32(d["g_x"].item()) == ga
+    assert np.array_equal(d["codes"].cpu().numpy(), ca)
+    cb, gb = fp8.quantize(wd.cpu().numpy())
+    assert np.float32(h.g_w) == gb
+    assert np.array_equal(w["codes"].cpu().numpy(), cb)
+
+    rows = sample_rows(case.M)
+    wp = asp.prepare_weight(case.W, case.s, case.V, case.b, fmt="fp8")
+    ap = asp.activation_prologue(case.x, case.s, case.V, case.b, fmt="fp8")
+    assert np.mean(ca[rows] == ap["codes"][rows]) >= 0.999
+    bias = case.bias.astype(np.float64)[None, :]
+    ref = asp.nvfp4_gemm(ap["deq"][rows], wp["deq"]) + bias
+    got = bf16_to_np(y)[rows]
+    assert asp.rel_fro(got, ref) <= TOL
+    own = fp8.dequantize(ca[rows], ga) @ fp8.dequantize(cb, gb).T + bias
+    row_err, blk_err = local_rel_errors(got, own)
+    assert row_err <= LOCAL_TOL and blk_err <= LOCAL_TOL, (row_err, blk_err)
