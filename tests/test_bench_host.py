@@ -114,3 +114,21 @@ def test_committed_traffic_entries_name_their_sources():
 def test_per_unit():
     assert bench.per_unit(2e9, 2.0, "GB/s") == pytest.approx(1.0)
     assert bench.per_unit(3e12, 1.5, "TFLOP/s") == pytest.approx(2.0)
+
+
+def test_reference_arm_line_on_the_cpu():
+    """bench.py --impl reference runs the float64 oracle on the host: its line
+    carries the contract's keys and the steps and warm-up it actually ran."""
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "c2", "--steps", "4", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "GB/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert (line["steps"], line["warmup"]) == (4, 3)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
